@@ -1,0 +1,218 @@
+/*
+ * svdq.h -- C ABI of the B200-native SVDQuant W4A4 (NVFP4) linear layer.
+ *
+ * What the layer computes ("Bringing Nunchaku 4-bit diffusion inference to
+ * Diffusers", section "Background: SVDQuant and Nunchaku"; the Hacker News
+ * thread on "SVDQuant: 4-Bit Quantization Powers 12B Flux on a 16GB 4090
+ * GPU with 3x Speedup"): activation outliers are smoothed into the weight,
+ * the smoothed weight W~ is split into a 16-bit rank-r branch L1 L2 plus a
+ * residual R, and only R (and the activation) is held in 4 bits:
+ *
+ *     Y = Q(X_hat) Q(R)^T + (X_hat L1) L2 + bias,   Q = NVFP4.
+ *
+ * NVFP4 (the svdq_w4a4 precision on Blackwell, hardware-support table of
+ * the same article): E2M1 values, one E4M3 scale per 16 consecutive
+ * elements along K, one fp32 tensor scale.
+ *
+ * Kernel fusion follows the Korean rendering of the article (section
+ * "SVDQuant and the Nunchaku engine"): the low-rank down-projection runs
+ * inside the activation-quantization kernel and the up-projection inside
+ * the 4-bit GEMM kernel, so the 16-bit branch adds no separate pass over
+ * memory.
+ *
+ * Conventions for every call:
+ *   - All pointers are caller-owned.  The library never allocates, frees or
+ *     retains device or host memory and never synchronizes a stream.
+ *   - "device" pointers must be global memory of the current CUDA device;
+ *     "host" pointers are ordinary host memory.
+ *   - bf16 tensors are passed as uint16_t bit patterns.
+ *   - Matrices are row-major; ld* is the row stride in elements.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  GPU calls
+ *     are asynchronous; errors found on the host are returned before any
+ *     launch; a device-side fault surfaces on the caller's next synchronize.
+ *   - Inputs must be finite; NaN/Inf activations give unspecified codes.
+ *   - The GPU entry points require an sm_100 device (B200); any other device
+ *     gives SVDQ_ERR_UNSUPPORTED_ARCH and launches nothing (the article's
+ *     rule: validate GPU capability and refuse rather than compute wrongly).
+ */
+#ifndef SVDQ_H
+#define SVDQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum svdq_status {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,      /* null pointer, bad shape or rank        */
+  SVDQ_ERR_UNSUPPORTED_ARCH = 2, /* no CUDA device, or not sm_100          */
+  SVDQ_ERR_MISALIGNED = 3,       /* pointer / leading dimension alignment  */
+  SVDQ_ERR_WORKSPACE = 4,        /* workspace smaller than required        */
+  SVDQ_ERR_CUDA = 5,             /* a CUDA runtime call or launch failed   */
+  SVDQ_ERR_TIMEOUT = 6,          /* a kernel gave up waiting (see below)   */
+  SVDQ_ERR_NUMERIC = 7           /* pack: non-finite weight or statistics  */
+} svdq_status;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* svdq_status_string(svdq_status s);
+
+/* Library version, e.g. "svdq-b200 0.1". */
+const char* svdq_version(void);
+
+/* ---------------------------------------------------------------- sizes --
+ * Buffer sizes (bytes) for an N x K weight with rank r.
+ *   r must be 0 or a multiple of 16 in [16, 128]; K a multiple of 64;
+ *   N a multiple of 16.
+ *   klr = round_up(2 r, 64): the padded K extent of the low-rank operands.
+ */
+typedef struct svdq_sizes {
+  int N, K, r, klr;
+  size_t smooth_bytes;   /* fp32 [K]                                       */
+  size_t l1_bytes;       /* bf16 [K][r]       plain factor L1              */
+  size_t l2_bytes;       /* bf16 [r][N]       plain factor L2              */
+  size_t l1_mma_bytes;   /* bf16 [2r][K]      kernel operand, see pack     */
+  size_t l2_mma_bytes;   /* bf16 [N][klr]     kernel operand, see pack     */
+  size_t codes_w_bytes;  /* u8   [N][K/2]     E2M1 codes of R              */
+  size_t sf_w_bytes;     /* u8   MMA tiles    E4M3 scales of R (rows padded to 256) */
+  size_t bias_bytes;     /* bf16 [N]                                       */
+} svdq_sizes;
+
+svdq_status svdq_query_sizes(int N, int K, int r, svdq_sizes* out);
+
+/* ------------------------------------------------------------------ pack --
+ * svdq_pack_weight: the offline quantization of one linear (host only,
+ * synchronous, re-entrant; OpenMP threads).  Steps, in the article's order
+ * ("Background: SVDQuant and Nunchaku"):
+ *   1. smoothing: lambda_j = (x_absmax_j / max_n |W_nj|)^alpha (lambda = 1
+ *      where either maximum is 0); stored as smooth_j = fp32(1/lambda_j), the
+ *      activation multiplier (x_hat = fp32(x * smooth_j)); W~ = W / smooth
+ *      in float64.
+ *   2. low-rank branch: top-r SVD of W~ (randomized subspace iteration with
+ *      Rayleigh-Ritz, seeded): L1 = V sqrt(S) [K x r], L2 = sqrt(S) U^T
+ *      [r x N], each rounded once to bf16.
+ *   3. residual R = fp32(W~ - (L1 L2)^T) (float64 sum over rank ascending).
+ *   4. NVFP4 of R: g_w = 2688 / max|R|; per 16 along K:
+ *      sf = E4M3(fp32(a/6) * g_w), code = E2M1(R * fp32(g_w / sf)).
+ *   5. activation tensor scale from calibration:
+ *      g_x = 2688 / max_j fp32(x_absmax_j * smooth_j).
+ *   6. lr_scale = fp32(g_x * g_w), alpha = fp32(1 / lr_scale).
+ *   7. kernel operands: l1_mma[i][k] = bf16 hi part and l1_mma[r+i][k] =
+ *      bf16 lo part of smooth_k * L1[k][i] (exact product in float64, hi =
+ *      bf16(p), lo = bf16(p - hi)); l2_mma[n][i] = l2_mma[n][r+i] = L2[i][n],
+ *      zero beyond 2r.
+ * Arguments:
+ *   W         host fp32 [N][K] (out x in, the PyTorch Linear layout)
+ *   x_absmax  host fp32 [K], per-input-channel max |x| of calibration data
+ *   smooth_alpha  smoothing exponent (0.5 in the workloads here)
+ *   seed      seed of the SVD's random start (the result is deterministic
+ *             for a given seed and build)
+ *   out       host buffers sized by svdq_query_sizes; every pointer field
+ *             except bias must be non-NULL; the scalars are written.
+ * Errors: INVALID_ARG for shapes/NULLs, NUMERIC for non-finite input.
+ */
+typedef struct svdq_packed_host {
+  float*    smooth;      /* [K]        */
+  uint16_t* l1;          /* [K][r]     */
+  uint16_t* l2;          /* [r][N]     */
+  uint16_t* l1_mma;      /* [2r][K]    */
+  uint16_t* l2_mma;      /* [N][klr]   */
+  uint8_t*  codes_w;     /* [N][K/2], even k in the low nibble             */
+  uint8_t*  sf_w;        /* MMA tile layout (svdq_sf_tile_offset)          */
+  float g_x, g_w, alpha, lr_scale;
+} svdq_packed_host;
+
+svdq_status svdq_pack_weight(const float* W, const float* x_absmax, int N,
+                             int K, int r, float smooth_alpha, uint64_t seed,
+                             svdq_packed_host* out);
+
+/* ---------------------------------------------------------------- layout --
+ * Byte offset of the E4M3 scale of (row, group g = k/16) in the MMA tile
+ * layout used for sf_w and sf_x: atoms of 128 rows x 4 scales (512 bytes),
+ * atom (row/128, g/4) at ((row/128) * (K/64) + g/4) * 512, and inside the
+ * atom byte (row%32)*16 + ((row%128)/32)*4 + g%4.  Returns -1 on bad args.
+ * This is the scale arrangement the block-scaled tensor-core MMA reads.
+ */
+int64_t svdq_sf_tile_offset(int row, int g, int K);
+
+/* -------------------------------------------------------------- forward --
+ * Device-side weight: a plain struct of device pointers (filled by the
+ * caller after copying the packed host buffers to the GPU).
+ */
+typedef struct svdq_weight {
+  int N, K, r;
+  float g_x, g_w, alpha, lr_scale;
+  const float*    smooth;   /* device fp32 [K], 16-byte aligned            */
+  const uint16_t* l1_mma;   /* device bf16 [2r][K]        (NULL if r == 0) */
+  const uint16_t* l2_mma;   /* device bf16 [N][klr]       (NULL if r == 0) */
+  const uint16_t* bias;     /* device bf16 [N] or NULL                     */
+  const uint8_t*  codes_w;  /* device u8 [N][K/2]                          */
+  const uint8_t*  sf_w;     /* device u8, MMA tiles, rows padded to 256    */
+} svdq_weight;
+
+/* Bytes of the activation workspace for M tokens: codes_x [M][K/2],
+ * sf_x (MMA tiles, rows padded to 128) and xl1 [M][klr] bf16, each region
+ * 256-byte aligned.  0 on bad arguments. */
+size_t svdq_act_workspace_bytes(int M, int K, int r);
+
+/* svdq_quantize_act: activation kernel (one launch).  For every row of X:
+ * x_hat = fp32(x * smooth); NVFP4 with the static g_x (per 16-group max by
+ * warp shuffles, E4M3 scale, E2M1 codes, two per byte); and, fused, the
+ * down-projection X_hat L1 on the tensor cores, written pre-multiplied by
+ * lr_scale as a bf16 hi/lo pair: xl1[m][i] + xl1[m][r+i] ~= lr_scale *
+ * (X_hat L1)[m][i], zeros in columns [2r, klr).
+ *   X        device bf16 [M][ldx], 16-byte aligned, ldx % 8 == 0, ldx >= K
+ *   codes_x  device u8 [M][K/2]
+ *   sf_x     device u8, MMA tiles, round_up(M,128) * K/16 bytes (pad rows 0)
+ *   xl1      device bf16 [M][klr] (may be NULL if r == 0)
+ * Reads X exactly once.
+ */
+svdq_status svdq_quantize_act(const svdq_weight* w, const uint16_t* X, int M,
+                              int64_t ldx, uint8_t* codes_x, uint8_t* sf_x,
+                              uint16_t* xl1, void* stream);
+
+/* svdq_gemm: the 4-bit GEMM kernel (one launch): block-scaled FP4 x FP4
+ * tensor-core MMA into an fp32 accumulator in tensor memory, the low-rank
+ * up-projection xl1 * L2 accumulated into the same accumulator, epilogue
+ * Y = bf16(alpha * acc + bias).
+ *   Y  device bf16 [M][ldy], 16-byte aligned, ldy % 8 == 0, ldy >= N
+ */
+svdq_status svdq_gemm(const svdq_weight* w, const uint8_t* codes_x,
+                      const uint8_t* sf_x, const uint16_t* xl1, int M,
+                      uint16_t* Y, int64_t ldy, void* stream);
+
+/* svdq_linear_forward: svdq_quantize_act then svdq_gemm on one stream, with
+ * the intermediates in `workspace` (device, >= svdq_act_workspace_bytes,
+ * 256-byte aligned). */
+svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t* X,
+                                int M, int64_t ldx, uint16_t* Y, int64_t ldy,
+                                void* workspace, size_t ws_bytes,
+                                void* stream);
+
+/* ------------------------------------------------------------- failure --
+ * Every wait inside the kernels is bounded (about one second).  A kernel
+ * that gives up records a code in a device-side word and exits cleanly
+ * (outstanding copies drained, tensor memory released); the CUDA context
+ * stays usable.  svdq_device_error synchronizes `stream`, returns the
+ * recorded code in *code (0 = none) and clears it.  Returns SVDQ_ERR_TIMEOUT
+ * when a code was set, SVDQ_OK otherwise.
+ */
+svdq_status svdq_device_error(void* stream, int* code);
+
+/* Test hook: launches a one-CTA kernel whose mbarrier wait can never be
+ * satisfied, with the wait limit set to `timeout_us`; it must end with the
+ * device error code set (exercises the bounded-wait path without a hang). */
+svdq_status svdq_selftest_timeout(int timeout_us, void* stream);
+
+/* Diagnostic: device float32 -> E2M1 (n codes, one per byte) and float32 ->
+ * E4M3 (one per byte, inputs >= 0) with the same hardware conversions the
+ * activation kernel uses.  in/out device pointers, n >= 0. */
+svdq_status svdq_debug_convert(const float* in, uint8_t* e2m1_out,
+                               uint8_t* e4m3_out, int64_t n, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SVDQ_H */

@@ -1,0 +1,352 @@
+"""Python binding of libsvdq.so, the B200-native SVDQuant W4A4 (NVFP4) linear.
+
+Argument marshalling only: every step of the layer runs inside the C/CUDA
+library (include/svdq.h).  PyTorch is used for device memory and streams.
+There is no fallback: if the library cannot be loaded, importing the
+binding raises, and the GPU calls raise SvdqError on any non-OK status.
+
+The functions keep the C names:
+  svdq_pack_weight      host-side smoothing, SVD, residual NVFP4 packing
+  svdq_quantize_act     activation kernel (+ fused low-rank down-projection)
+  svdq_gemm             4-bit GEMM kernel (+ fused up-projection, bias)
+  svdq_linear_forward   both kernels on one stream
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import numpy as np
+
+from . import build as _build
+
+__all__ = [
+    "SvdqError", "PackedWeight", "DeviceWeight", "svdq_query_sizes", "svdq_pack_weight",
+    "svdq_quantize_act", "svdq_gemm", "svdq_linear_forward", "svdq_act_workspace_bytes",
+    "svdq_device_error", "svdq_selftest_timeout", "svdq_debug_convert", "svdq_sf_tile_offset",
+    "svdq_status_string", "SVDQW4A4Linear", "lib", "STATUS",
+]
+
+STATUS = {
+    0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_UNSUPPORTED_ARCH",
+    3: "SVDQ_ERR_MISALIGNED", 4: "SVDQ_ERR_WORKSPACE", 5: "SVDQ_ERR_CUDA",
+    6: "SVDQ_ERR_TIMEOUT", 7: "SVDQ_ERR_NUMERIC",
+}
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS.get(status, status)} ({svdq_status_string(status)})")
+
+
+class SvdqSizes(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int), ("K", ctypes.c_int), ("r", ctypes.c_int),
+                ("klr", ctypes.c_int), ("smooth_bytes", ctypes.c_size_t),
+                ("l1_bytes", ctypes.c_size_t), ("l2_bytes", ctypes.c_size_t),
+                ("l1_mma_bytes", ctypes.c_size_t), ("l2_mma_bytes", ctypes.c_size_t),
+                ("codes_w_bytes", ctypes.c_size_t), ("sf_w_bytes", ctypes.c_size_t),
+                ("bias_bytes", ctypes.c_size_t)]
+
+
+class SvdqPackedHost(ctypes.Structure):
+    _fields_ = [("smooth", ctypes.c_void_p), ("l1", ctypes.c_void_p), ("l2", ctypes.c_void_p),
+                ("l1_mma", ctypes.c_void_p), ("l2_mma", ctypes.c_void_p),
+                ("codes_w", ctypes.c_void_p), ("sf_w", ctypes.c_void_p),
+                ("g_x", ctypes.c_float), ("g_w", ctypes.c_float), ("alpha", ctypes.c_float),
+                ("lr_scale", ctypes.c_float)]
+
+
+class SvdqWeight(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int), ("K", ctypes.c_int), ("r", ctypes.c_int),
+                ("g_x", ctypes.c_float), ("g_w", ctypes.c_float), ("alpha", ctypes.c_float),
+                ("lr_scale", ctypes.c_float), ("smooth", ctypes.c_void_p),
+                ("l1_mma", ctypes.c_void_p), ("l2_mma", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p), ("codes_w", ctypes.c_void_p),
+                ("sf_w", ctypes.c_void_p)]
+
+
+def _load() -> ctypes.CDLL:
+    path = _build.build()          # no-op when the in-tree library is current
+    if not os.path.exists(path):
+        raise ImportError(f"libsvdq.so missing at {path}")
+    L = ctypes.CDLL(path)
+    P, I, I64, SZ, F, U64 = (ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t,
+                             ctypes.c_float, ctypes.c_uint64)
+    sig = {
+        "svdq_status_string": (ctypes.c_char_p, [I]),
+        "svdq_version": (ctypes.c_char_p, []),
+        "svdq_query_sizes": (I, [I, I, I, ctypes.POINTER(SvdqSizes)]),
+        "svdq_pack_weight": (I, [P, P, I, I, I, F, U64, ctypes.POINTER(SvdqPackedHost)]),
+        "svdq_sf_tile_offset": (I64, [I, I, I]),
+        "svdq_act_workspace_bytes": (SZ, [I, I, I]),
+        "svdq_quantize_act": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P, P, P]),
+        "svdq_gemm": (I, [ctypes.POINTER(SvdqWeight), P, P, P, I, P, I64, P]),
+        "svdq_linear_forward": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P, SZ, P]),
+        "svdq_device_error": (I, [P, ctypes.POINTER(I)]),
+        "svdq_selftest_timeout": (I, [I, P]),
+        "svdq_debug_convert": (I, [P, P, P, I64, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    return L
+
+
+lib = _load()
+
+
+def svdq_status_string(status: int) -> str:
+    return lib.svdq_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise SvdqError(status, what)
+
+
+def svdq_query_sizes(N: int, K: int, r: int) -> SvdqSizes:
+    out = SvdqSizes()
+    _check(lib.svdq_query_sizes(N, K, r, ctypes.byref(out)), "svdq_query_sizes")
+    return out
+
+
+def svdq_sf_tile_offset(row: int, g: int, K: int) -> int:
+    return int(lib.svdq_sf_tile_offset(row, g, K))
+
+
+def svdq_act_workspace_bytes(M: int, K: int, r: int) -> int:
+    return int(lib.svdq_act_workspace_bytes(M, K, r))
+
+
+# ---------------------------------------------------------------- pack ----
+
+@dataclass
+class PackedWeight:
+    """Host result of svdq_pack_weight (numpy arrays, bf16 as uint16)."""
+    N: int
+    K: int
+    r: int
+    klr: int
+    smooth: np.ndarray       # fp32 [K]
+    l1: np.ndarray           # bf16 [K, r]
+    l2: np.ndarray           # bf16 [r, N]
+    l1_mma: np.ndarray       # bf16 [2r, K]
+    l2_mma: np.ndarray       # bf16 [N, klr]
+    codes_w: np.ndarray      # u8 [N, K/2]
+    sf_w: np.ndarray         # u8, MMA tiles
+    g_x: float
+    g_w: float
+    alpha: float
+    lr_scale: float
+
+    def to_device(self, device="cuda", bias_bf16: Optional[np.ndarray] = None) -> "DeviceWeight":
+        import torch
+
+        def up(a):
+            return torch.from_numpy(np.ascontiguousarray(a)).to(device)
+
+        t = {"smooth": up(self.smooth), "codes_w": up(self.codes_w), "sf_w": up(self.sf_w)}
+        if self.r > 0:
+            t["l1_mma"] = up(self.l1_mma.view(np.int16))
+            t["l2_mma"] = up(self.l2_mma.view(np.int16))
+        if bias_bf16 is not None:
+            t["bias"] = up(np.asarray(bias_bf16, np.uint16).view(np.int16))
+        return DeviceWeight(self, t)
+
+
+class DeviceWeight:
+    """Device copies of a packed weight plus the C struct pointing at them."""
+
+    def __init__(self, packed: PackedWeight, tensors: dict):
+        self.packed = packed
+        self.tensors = tensors
+        s = SvdqWeight()
+        s.N, s.K, s.r = packed.N, packed.K, packed.r
+        s.g_x, s.g_w, s.alpha, s.lr_scale = packed.g_x, packed.g_w, packed.alpha, packed.lr_scale
+        for name in ("smooth", "l1_mma", "l2_mma", "bias", "codes_w", "sf_w"):
+            t = tensors.get(name)
+            setattr(s, name, t.data_ptr() if t is not None else None)
+        self.struct = s
+
+    @property
+    def N(self):
+        return self.packed.N
+
+    @property
+    def K(self):
+        return self.packed.K
+
+    @property
+    def r(self):
+        return self.packed.r
+
+
+def svdq_pack_weight(W: np.ndarray, x_absmax: np.ndarray, r: int, smooth_alpha: float = 0.5,
+                     seed: int = 0) -> PackedWeight:
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    x_absmax = np.ascontiguousarray(x_absmax, dtype=np.float32)
+    N, K = W.shape
+    if x_absmax.shape != (K,):
+        raise ValueError("x_absmax must have shape [K]")
+    sz = svdq_query_sizes(N, K, r)
+    smooth = np.empty(K, np.float32)
+    l1 = np.empty((K, r), np.uint16)
+    l2 = np.empty((r, N), np.uint16)
+    l1m = np.empty((2 * r, K), np.uint16)
+    l2m = np.empty((N, sz.klr), np.uint16)
+    codes = np.empty((N, K // 2), np.uint8)
+    sf = np.empty(sz.sf_w_bytes, np.uint8)
+    out = SvdqPackedHost()
+    out.smooth = smooth.ctypes.data
+    out.l1 = l1.ctypes.data if r else None
+    out.l2 = l2.ctypes.data if r else None
+    out.l1_mma = l1m.ctypes.data if r else None
+    out.l2_mma = l2m.ctypes.data if r else None
+    out.codes_w = codes.ctypes.data
+    out.sf_w = sf.ctypes.data
+    _check(lib.svdq_pack_weight(W.ctypes.data, x_absmax.ctypes.data, N, K, r,
+                                float(smooth_alpha), int(seed), ctypes.byref(out)),
+           "svdq_pack_weight")
+    return PackedWeight(N, K, r, sz.klr, smooth, l1, l2, l1m, l2m, codes, sf,
+                        float(out.g_x), float(out.g_w), float(out.alpha), float(out.lr_scale))
+
+
+# ------------------------------------------------------------- forward ----
+
+def _stream_ptr(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _act_shapes(M: int, K: int, r: int):
+    klr = ((2 * r + 63) // 64) * 64
+    sf_bytes = ((M + 127) // 128) * 128 * (K // 16)
+    return klr, sf_bytes
+
+
+def _check_x(X, K):
+    import torch
+    if X.dtype != torch.bfloat16 or X.dim() != 2 or X.shape[1] != K or X.stride(1) != 1:
+        raise ValueError("X must be a bf16 [M, K] tensor with unit column stride")
+
+
+def svdq_quantize_act(w: DeviceWeight, X, codes_x=None, sf_x=None, xl1=None, stream=None):
+    """Returns (codes_x u8 [M, K/2], sf_x u8 tiles, xl1 bf16 [M, klr] or None)."""
+    import torch
+    _check_x(X, w.K)
+    M = X.shape[0]
+    klr, sf_bytes = _act_shapes(M, w.K, w.r)
+    dev = X.device
+    if codes_x is None:
+        codes_x = torch.empty((M, w.K // 2), dtype=torch.uint8, device=dev)
+    if sf_x is None:
+        sf_x = torch.empty(sf_bytes, dtype=torch.uint8, device=dev)
+    if xl1 is None and w.r > 0:
+        xl1 = torch.empty((M, klr), dtype=torch.bfloat16, device=dev)
+    _check(lib.svdq_quantize_act(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
+                                 codes_x.data_ptr(), sf_x.data_ptr(), _ptr(xl1),
+                                 _stream_ptr(stream)), "svdq_quantize_act")
+    return codes_x, sf_x, xl1
+
+
+def svdq_gemm(w: DeviceWeight, codes_x, sf_x, xl1, M: int, Y=None, stream=None):
+    import torch
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=codes_x.device)
+    _check(lib.svdq_gemm(ctypes.byref(w.struct), codes_x.data_ptr(), sf_x.data_ptr(),
+                         _ptr(xl1), M, Y.data_ptr(), Y.stride(0), _stream_ptr(stream)),
+           "svdq_gemm")
+    return Y
+
+
+def svdq_linear_forward(w: DeviceWeight, X, Y=None, workspace=None, stream=None):
+    import torch
+    _check_x(X, w.K)
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+    need = svdq_act_workspace_bytes(M, w.K, w.r)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+    _check(lib.svdq_linear_forward(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
+                                   Y.data_ptr(), Y.stride(0), workspace.data_ptr(),
+                                   workspace.numel(), _stream_ptr(stream)),
+           "svdq_linear_forward")
+    return Y
+
+
+def svdq_linear_forward_host(w: DeviceWeight, X_host, Y_host, X_dev, Y_dev, workspace,
+                             stream=None):
+    """The host-buffer form of the forward: copy X (pinned host) to the
+    device, run the layer, copy Y back into pinned host memory, all on
+    `stream` (asynchronous)."""
+    X_dev.copy_(X_host, non_blocking=True)
+    svdq_linear_forward(w, X_dev, Y_dev, workspace, stream)
+    Y_host.copy_(Y_dev, non_blocking=True)
+    return Y_host
+
+
+def svdq_device_error(stream=None) -> int:
+    code = ctypes.c_int(0)
+    st = lib.svdq_device_error(_stream_ptr(stream), ctypes.byref(code))
+    if st not in (0, 6):
+        raise SvdqError(st, "svdq_device_error")
+    return code.value
+
+
+def svdq_selftest_timeout(timeout_us: int, stream=None):
+    _check(lib.svdq_selftest_timeout(int(timeout_us), _stream_ptr(stream)),
+           "svdq_selftest_timeout")
+
+
+def svdq_debug_convert(x):
+    import torch
+    x = x.contiguous()
+    e2 = torch.empty(x.numel(), dtype=torch.uint8, device=x.device)
+    e4 = torch.empty(x.numel(), dtype=torch.uint8, device=x.device)
+    _check(lib.svdq_debug_convert(x.data_ptr(), e2.data_ptr(), e4.data_ptr(), x.numel(),
+                                  _stream_ptr(None)), "svdq_debug_convert")
+    return e2, e4
+
+
+# ------------------------------------------------------------ module ----
+
+def _linear_module_base():
+    import torch
+    return torch.nn.Module
+
+
+class SVDQW4A4Linear(_linear_module_base()):
+    """Drop-in analogue of the runtime layer the article names
+    (SVDQW4A4Linear replaces nn.Linear): built from a float weight, a bias and
+    calibration statistics; forward runs svdq_linear_forward."""
+
+    def __init__(self, weight: np.ndarray, bias_bf16: Optional[np.ndarray], x_absmax: np.ndarray,
+                 rank: int = 32, smooth_alpha: float = 0.5, seed: int = 0, device="cuda"):
+        super().__init__()
+        self.packed = svdq_pack_weight(weight, x_absmax, rank, smooth_alpha, seed)
+        self.dev = self.packed.to_device(device, bias_bf16)
+        self.in_features = self.packed.K
+        self.out_features = self.packed.N
+        self._ws = None
+
+    def forward(self, X):
+        import torch
+        lead = X.shape[:-1]
+        X2 = X.reshape(-1, X.shape[-1])
+        M = X2.shape[0]
+        need = svdq_act_workspace_bytes(M, self.packed.K, self.packed.r)
+        if self._ws is None or self._ws.numel() < need or self._ws.device != X.device:
+            self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+        Y = svdq_linear_forward(self.dev, X2, workspace=self._ws)
+        return Y.reshape(*lead, self.out_features)

@@ -1,0 +1,359 @@
+// C ABI of the B200 SVDQuant W4A4 linear: argument checks, tensor-map
+// (TMA descriptor) encoding and kernel launches.  See include/svdq.h for the
+// contract of every entry point.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/svdq.h"
+#include "ptx.cuh"
+#include "quantize_act.cuh"
+#include "w4a4_gemm.cuh"
+
+namespace svdq_dev {
+
+// Never satisfied wait: exercises the bounded-wait error path.
+__global__ void selftest_timeout_kernel(uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    mbar_wait(smem_u32(&bar), 0, timeout_ns, &abort_flag, (7u << 8) | 3u);
+  __syncthreads();
+}
+
+// The hardware conversions of the activation kernel, one value per thread.
+__global__ void debug_convert_kernel(const float* in, uint8_t* e2m1, uint8_t* e4m3, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float x = in[i];
+  if (e2m1) {
+    const float v[8] = {x, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    e2m1[i] = (uint8_t)(cvt_e2m1x8(v) & 0xF);
+  }
+  if (e4m3) e4m3[i] = (uint8_t)(cvt_e4m3x2(fabsf(x), 0.0f) & 0xFF);
+}
+}  // namespace svdq_dev
+
+using namespace svdq_dev;
+
+namespace {
+
+constexpr uint64_t kDefaultTimeoutNs = 1000000000ull;  // 1 s per wait
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+struct DeviceInfo {
+  bool checked = false;
+  bool ok = false;
+  int num_sms = 0;
+  bool attrs_set = false;
+};
+constexpr int kMaxDevices = 64;
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+EncodeTiledFn g_encode = nullptr;
+
+svdq_status device_check(int* sms) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SVDQ_ERR_UNSUPPORTED_ARCH;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.checked) {
+    int major = 0, minor = 0, n = 0;
+    const bool q = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) == cudaSuccess &&
+                   cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) == cudaSuccess &&
+                   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess;
+    cudaGetLastError();
+    d.checked = true;
+    d.ok = q && major == 10 && minor == 0;
+    d.num_sms = n;
+  }
+  if (!d.ok) return SVDQ_ERR_UNSUPPORTED_ARCH;
+  if (!d.attrs_set) {
+    if (cudaFuncSetAttribute(quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)qa_smem_bytes(128)) != cudaSuccess ||
+        cudaFuncSetAttribute(w4a4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)gemm_smem_bytes()) != cudaSuccess) {
+      cudaGetLastError();
+      return SVDQ_ERR_CUDA;
+    }
+    d.attrs_set = true;
+  }
+  if (!g_encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult qres;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &qres) !=
+            cudaSuccess ||
+        qres != cudaDriverEntryPointSuccess || !fn) {
+      cudaGetLastError();
+      return SVDQ_ERR_CUDA;
+    }
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  }
+  if (sms) *sms = d.num_sms;
+  return SVDQ_OK;
+}
+
+// 2D tensor map over a row-major [rows][inner] matrix, 128-byte swizzle.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
+              uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+inline size_t rup(size_t x, size_t m) { return (x + m - 1) / m * m; }
+
+svdq_status check_weight(const svdq_weight* w) {
+  if (!w) return SVDQ_ERR_INVALID_ARG;
+  svdq_sizes sz;
+  if (svdq_query_sizes(w->N, w->K, w->r, &sz) != SVDQ_OK) return SVDQ_ERR_INVALID_ARG;
+  if (!w->smooth || !w->codes_w || !w->sf_w) return SVDQ_ERR_INVALID_ARG;
+  if (w->r > 0 && (!w->l1_mma || !w->l2_mma)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(w->smooth) || !aligned16(w->codes_w) || !aligned16(w->sf_w) ||
+      (w->bias && !aligned16(w->bias)) || (w->l1_mma && !aligned16(w->l1_mma)) ||
+      (w->l2_mma && !aligned16(w->l2_mma)))
+    return SVDQ_ERR_MISALIGNED;
+  return SVDQ_OK;
+}
+
+int klr_of(int r) { return (int)rup((size_t)2 * r, 64); }
+
+svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int64_t ldx,
+                            uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, cudaStream_t s,
+                            int sms) {
+  const int K = w->K, r = w->r;
+  const int RB = (M + 127) / 128;
+  const int KC = K / 64;
+  int S = std::max(1, std::min(8, sms / std::max(1, RB)));
+  S = std::min(S, KC);
+  const int cps = (KC + S - 1) / S;
+  S = (KC + cps - 1) / cps;
+
+  CUtensorMap tm_x, tm_l1;
+  std::memset(&tm_l1, 0, sizeof(tm_l1));
+  if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M,
+                (uint64_t)ldx * 2, 64, 128))
+    return SVDQ_ERR_CUDA;
+  if (r > 0 && !make_map(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l1_mma, (uint64_t)K,
+                         (uint64_t)(2 * r), (uint64_t)K * 2, 64, (uint32_t)(2 * r)))
+    return SVDQ_ERR_CUDA;
+
+  QAParams p;
+  p.smooth = w->smooth;
+  p.codes_x = codes_x;
+  p.sf_x = sf_x;
+  p.xl1 = xl1;
+  p.M = M;
+  p.K = K;
+  p.r = r;
+  p.klr = klr_of(r);
+  p.chunks_per_split = cps;
+  p.num_splits = S;
+  p.stage_bytes = qa_stage_bytes(r);
+  uint32_t cols = 32;
+  while (cols < (uint32_t)(2 * r)) cols <<= 1;
+  p.tmem_cols = cols;
+  p.g_x = w->g_x;
+  p.lr_scale = w->lr_scale;
+  p.timeout_ns = kDefaultTimeoutNs;
+
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)S, (unsigned)RB, 1);
+  cfg.blockDim = dim3(QA_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = qa_smem_bytes(r);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  cfg.attrs = attr;
+  cfg.numAttrs = 0;
+  if (r > 0 && S > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.numAttrs = 1;
+  }
+  if (cudaLaunchKernelEx(&cfg, quantize_act_kernel, tm_x, tm_l1, p) != cudaSuccess) {
+    cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
+}
+
+svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint8_t* sf_x,
+                        const uint16_t* xl1, int M, uint16_t* Y, int64_t ldy, cudaStream_t s,
+                        int sms) {
+  const int N = w->N, K = w->K, r = w->r, klr = klr_of(r);
+  CUtensorMap ta, tb, talr, tblr;
+  std::memset(&talr, 0, sizeof(talr));
+  std::memset(&tblr, 0, sizeof(tblr));
+  if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_x, (uint64_t)K / 2, (uint64_t)M,
+                (uint64_t)K / 2, 128, G_BM) ||
+      !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes_w, (uint64_t)K / 2, (uint64_t)N,
+                (uint64_t)K / 2, 128, G_BN))
+    return SVDQ_ERR_CUDA;
+  if (r > 0) {
+    if (!make_map(&talr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xl1, (uint64_t)klr, (uint64_t)M,
+                  (uint64_t)klr * 2, 64, G_BM) ||
+        !make_map(&tblr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l2_mma, (uint64_t)klr, (uint64_t)N,
+                  (uint64_t)klr * 2, 64, G_BN))
+      return SVDQ_ERR_CUDA;
+  }
+  GemmParams p;
+  p.sf_x = sf_x;
+  p.sf_w = w->sf_w;
+  p.bias = w->bias;
+  p.Y = Y;
+  p.ldy = ldy;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.r = r;
+  p.klr = klr;
+  p.alpha = w->alpha;
+  p.timeout_ns = kDefaultTimeoutNs;
+  const int tiles = ((M + G_BM - 1) / G_BM) * ((N + G_BN - 1) / G_BN);
+  const int grid = std::max(1, std::min(tiles, sms));
+  w4a4_gemm_kernel<<<grid, G_THREADS, gemm_smem_bytes(), s>>>(ta, tb, talr, tblr, p);
+  if (cudaGetLastError() != cudaSuccess) return SVDQ_ERR_CUDA;
+  return SVDQ_OK;
+}
+
+size_t ws_codes(int M, int K) { return rup((size_t)M * (K / 2), 256); }
+size_t ws_sf(int M, int K) { return rup(rup((size_t)M, 128) * (K / 16), 256); }
+size_t ws_xl1(int M, int r) { return rup((size_t)M * klr_of(r) * 2, 256); }
+
+}  // namespace
+
+extern "C" const char* svdq_status_string(svdq_status s) {
+  switch (s) {
+    case SVDQ_OK: return "ok";
+    case SVDQ_ERR_INVALID_ARG: return "invalid argument";
+    case SVDQ_ERR_UNSUPPORTED_ARCH: return "unsupported device (an sm_100 B200 is required)";
+    case SVDQ_ERR_MISALIGNED: return "misaligned pointer or leading dimension";
+    case SVDQ_ERR_WORKSPACE: return "workspace too small";
+    case SVDQ_ERR_CUDA: return "CUDA runtime error";
+    case SVDQ_ERR_TIMEOUT: return "a kernel wait timed out";
+    case SVDQ_ERR_NUMERIC: return "non-finite input";
+  }
+  return "unknown status";
+}
+
+extern "C" const char* svdq_version(void) { return "svdq-b200 0.1"; }
+
+extern "C" size_t svdq_act_workspace_bytes(int M, int K, int r) {
+  if (M < 0 || K <= 0 || K % 64 || r < 0 || r > 128 || (r && r % 16)) return 0;
+  return ws_codes(M, K) + ws_sf(M, K) + (r > 0 ? ws_xl1(M, r) : 0);
+}
+
+extern "C" svdq_status svdq_quantize_act(const svdq_weight* w, const uint16_t* X, int M,
+                                         int64_t ldx, uint8_t* codes_x, uint8_t* sf_x,
+                                         uint16_t* xl1, void* stream) {
+  svdq_status st = check_weight(w);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || ldx < w->K) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !codes_x || !sf_x || (w->r > 0 && !xl1)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || ldx % 8 || !aligned16(codes_x) || !aligned16(sf_x) ||
+      (xl1 && !aligned16(xl1)))
+    return SVDQ_ERR_MISALIGNED;
+  int sms = 0;
+  if ((st = device_check(&sms)) != SVDQ_OK) return st;
+  return launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, (cudaStream_t)stream, sms);
+}
+
+extern "C" svdq_status svdq_gemm(const svdq_weight* w, const uint8_t* codes_x,
+                                 const uint8_t* sf_x, const uint16_t* xl1, int M, uint16_t* Y,
+                                 int64_t ldy, void* stream) {
+  svdq_status st = check_weight(w);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || ldy < w->N) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!codes_x || !sf_x || !Y || (w->r > 0 && !xl1)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(codes_x) || !aligned16(sf_x) || !aligned16(Y) || ldy % 8 ||
+      (xl1 && !aligned16(xl1)))
+    return SVDQ_ERR_MISALIGNED;
+  int sms = 0;
+  if ((st = device_check(&sms)) != SVDQ_OK) return st;
+  return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, (cudaStream_t)stream, sms);
+}
+
+extern "C" svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t* X, int M,
+                                           int64_t ldx, uint16_t* Y, int64_t ldy,
+                                           void* workspace, size_t ws_bytes, void* stream) {
+  svdq_status st = check_weight(w);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || ldx < w->K || ldy < w->N) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !Y || !workspace) return SVDQ_ERR_INVALID_ARG;
+  if (ws_bytes < svdq_act_workspace_bytes(M, w->K, w->r)) return SVDQ_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return SVDQ_ERR_MISALIGNED;
+  if (!aligned16(X) || !aligned16(Y) || ldx % 8 || ldy % 8) return SVDQ_ERR_MISALIGNED;
+  int sms = 0;
+  if ((st = device_check(&sms)) != SVDQ_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint8_t* codes_x = base;
+  uint8_t* sf_x = codes_x + ws_codes(M, w->K);
+  uint16_t* xl1 = w->r > 0 ? reinterpret_cast<uint16_t*>(sf_x + ws_sf(M, w->K)) : nullptr;
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((st = launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, s, sms)) != SVDQ_OK) return st;
+  return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, s, sms);
+}
+
+extern "C" svdq_status svdq_device_error(void* stream, int* code) {
+  if (!code) return SVDQ_ERR_INVALID_ARG;
+  *code = 0;
+  svdq_status st = device_check(nullptr);
+  if (st != SVDQ_OK) return st;
+  if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return SVDQ_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_svdq_error, sizeof(v)) != cudaSuccess ||
+      cudaMemcpyToSymbol(g_svdq_error, &zero, sizeof(zero)) != cudaSuccess)
+    return SVDQ_ERR_CUDA;
+  *code = (int)v;
+  return v ? SVDQ_ERR_TIMEOUT : SVDQ_OK;
+}
+
+extern "C" svdq_status svdq_selftest_timeout(int timeout_us, void* stream) {
+  if (timeout_us <= 0 || timeout_us > 10000000) return SVDQ_ERR_INVALID_ARG;
+  svdq_status st = device_check(nullptr);
+  if (st != SVDQ_OK) return st;
+  selftest_timeout_kernel<<<1, 32, 0, (cudaStream_t)stream>>>((uint64_t)timeout_us * 1000ull);
+  return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+extern "C" svdq_status svdq_debug_convert(const float* in, uint8_t* e2m1_out, uint8_t* e4m3_out,
+                                          int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && !in)) return SVDQ_ERR_INVALID_ARG;
+  if (n == 0) return SVDQ_OK;
+  svdq_status st = device_check(nullptr);
+  if (st != SVDQ_OK) return st;
+  const int64_t blocks = (n + 255) / 256;
+  if (blocks > 0x7FFFFFFF) return SVDQ_ERR_INVALID_ARG;
+  debug_convert_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(in, e2m1_out, e4m3_out, n);
+  return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}

@@ -1,0 +1,284 @@
+// 4-bit GEMM kernel of the SVDQuant W4A4 linear with the fused low-rank
+// up-projection, bias and bf16 store.
+//
+// The fusion follows the Nunchaku engine as described in the Korean
+// rendering of "Bringing Nunchaku 4-bit diffusion inference to Diffusers"
+// (section "SVDQuant and the Nunchaku engine"): the low-rank up projection is
+// merged into the 4-bit compute kernel.  The B200 design:
+//
+//   * persistent CTAs (one per SM) walk 128 x 256 output tiles;
+//   * warp 0 (one lane) streams, per 256-wide K step, the E2M1 code tiles of
+//     X [128 x 128 B] and of R [256 x 128 B] with TMA (128-byte swizzle) and
+//     the matching E4M3 scale atoms (512 B each, already in the MMA layout)
+//     with bulk copies, into a 4-deep shared-memory ring;
+//   * warp 1 (one lane) copies the scale atoms into tensor memory
+//     (tcgen05.cp, 32x128b x4) and issues tcgen05.mma kind::mxf4nvf4 with
+//     block16 UE4M3 scales, K = 64 per instruction, into a 128 x 256 fp32
+//     accumulator in tensor memory; after the K loop it streams the low-rank
+//     operands (xl1 hi|lo [128 x 2r] and L2 [256 x 2r], bf16) through the
+//     same ring and accumulates xl1 . L2 into the SAME accumulator with
+//     kind::f16 MMAs (xl1 was pre-multiplied by g_x g_w = 1/alpha);
+//   * warps 2..5 drain the accumulator (tcgen05.ld), compute
+//     Y = bf16(alpha * acc + bias) and store it.
+#pragma once
+#include "ptx.cuh"
+
+namespace svdq_dev {
+
+constexpr int G_STAGES = 4;
+constexpr int G_THREADS = 192;
+constexpr int G_BM = 128, G_BN = 256;
+constexpr uint32_t G_A_BYTES = 128 * 128;    // 128 rows x 128 B
+constexpr uint32_t G_B_BYTES = 256 * 128;    // 256 rows x 128 B
+constexpr uint32_t G_SFA_BYTES = 4 * 512;    // 4 atoms (K = 256)
+constexpr uint32_t G_SFB_BYTES = 8 * 512;    // 2 row blocks x 4 atoms
+constexpr uint32_t G_STAGE_BYTES = G_A_BYTES + G_B_BYTES + G_SFA_BYTES + G_SFB_BYTES;
+constexpr uint32_t G_TMEM_COLS = 512;
+constexpr uint32_t G_SF_TMEM = 256;          // scale buffers after the accumulator
+constexpr uint32_t G_SF_TMEM_STRIDE = 48;    // 16 cols SFA + 32 cols SFB
+
+__host__ __device__ inline uint32_t gemm_smem_bytes() {
+  return 1024u + G_STAGES * G_STAGE_BYTES + 256u;
+}
+
+struct GemmParams {
+  const uint8_t* sf_x;
+  const uint8_t* sf_w;
+  const uint16_t* bias;
+  uint16_t* Y;
+  long long ldy;
+  int M, N, K, r, klr;
+  float alpha;
+  uint64_t timeout_ns;
+};
+
+__global__ void __launch_bounds__(G_THREADS, 1)
+    w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
+                     const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_alr,
+                     const __grid_constant__ CUtensorMap tm_blr, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G_STAGES * G_STAGE_BYTES);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * G_STAGES;
+  const uint32_t acc_full = full0 + 16 * G_STAGES;
+  const uint32_t acc_empty = acc_full + 8;
+  const uint32_t drain_bar = acc_full + 16;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * G_STAGES + 3);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const uint32_t warp = warp_id(), lane = lane_id();
+  const int M = p.M, N = p.N, K = p.K, r = p.r;
+  const bool has_lr = r > 0;
+  const int num_m = (M + G_BM - 1) / G_BM;
+  const int num_n = (N + G_BN - 1) / G_BN;
+  const int num_tiles = num_m * num_n;
+  const int k64 = K >> 6;
+  const int kb_total = (k64 + 3) >> 2;
+  const int lr_chunks = has_lr ? (p.klr >> 6) : 0;
+  const unsigned int kid = 2;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < G_STAGES; ++i) {
+      mbar_init(full0 + 8 * i, 1);
+      mbar_init(empty0 + 8 * i, 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 128);
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tm_a);
+    prefetch_tensormap(&tm_b);
+    if (has_lr) {
+      prefetch_tensormap(&tm_alr);
+      prefetch_tensormap(&tm_blr);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), G_TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  int issued = 0;
+  if (warp == 0) {
+    // ---------------------------------------------------- TMA producer ----
+    if (lane == 0) {
+      int it = 0;
+      bool stop = false;
+      for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
+        const int mb = tile % num_m, nb = tile / num_m;
+        for (int kb = 0; kb < kb_total; ++kb, ++it) {
+          const int st = it % G_STAGES;
+          const uint32_t ph = (it / G_STAGES) & 1;
+          if (!mbar_wait(empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) {
+            stop = true;
+            break;
+          }
+          const int nk = min(4, k64 - 4 * kb);
+          const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
+          const uint32_t fb = full0 + 8 * st;
+          mbar_arrive_expect_tx(fb, G_A_BYTES + G_B_BYTES + 3u * 512u * nk);
+          tma_load_2d(sb, &tm_a, kb * 128, mb * G_BM, fb);
+          tma_load_2d(sb + G_A_BYTES, &tm_b, kb * 128, nb * G_BN, fb);
+          bulk_load(sb + G_A_BYTES + G_B_BYTES, p.sf_x + ((size_t)mb * k64 + 4 * kb) * 512,
+                    512u * nk, fb);
+          for (int hh = 0; hh < 2; ++hh)
+            bulk_load(sb + G_A_BYTES + G_B_BYTES + G_SFA_BYTES + hh * 2048,
+                      p.sf_w + ((size_t)(2 * nb + hh) * k64 + 4 * kb) * 512, 512u * nk, fb);
+          issued = it + 1;
+        }
+        for (int c = 0; c < lr_chunks && !stop; ++c, ++it) {
+          const int st = it % G_STAGES;
+          const uint32_t ph = (it / G_STAGES) & 1;
+          if (!mbar_wait(empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) {
+            stop = true;
+            break;
+          }
+          const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
+          const uint32_t fb = full0 + 8 * st;
+          mbar_arrive_expect_tx(fb, G_A_BYTES + G_B_BYTES);
+          tma_load_2d(sb, &tm_alr, c * 64, mb * G_BM, fb);
+          tma_load_2d(sb + G_A_BYTES, &tm_blr, c * 64, nb * G_BN, fb);
+          issued = it + 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer ----
+    if (lane == 0) {
+      const uint32_t id_fp4 = idesc_nvfp4(G_BM, G_BN);
+      const uint32_t id_lr = idesc_bf16(G_BM, G_BN);
+      int it = 0, tcount = 0;
+      bool stop = false;
+      for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x, ++tcount) {
+        if (!mbar_wait(acc_empty, (tcount & 1) ^ 1, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
+        tc_fence_after();
+        uint32_t accumulate = 0;
+        for (int kb = 0; kb < kb_total; ++kb, ++it) {
+          const int st = it % G_STAGES;
+          const uint32_t ph = (it / G_STAGES) & 1;
+          if (!mbar_wait(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const int nk = min(4, k64 - 4 * kb);
+          const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
+          const uint32_t sfa_s = sb + G_A_BYTES + G_B_BYTES;
+          const uint32_t sfb_s = sfa_s + G_SFA_BYTES;
+          const uint32_t sfa_t = tmem + G_SF_TMEM + (it & 1) * G_SF_TMEM_STRIDE;
+          const uint32_t sfb_t = sfa_t + 16;
+          for (int kk = 0; kk < nk; ++kk) {
+            tmem_copy_32x128b_x4(sfa_t + 4 * kk, sdesc_sf_block(sfa_s + 512 * kk));
+            tmem_copy_32x128b_x4(sfb_t + 8 * kk, sdesc_sf_block(sfb_s + 512 * kk));
+            tmem_copy_32x128b_x4(sfb_t + 8 * kk + 4, sdesc_sf_block(sfb_s + 2048 + 512 * kk));
+          }
+          const uint64_t da = sdesc_sw128(sb), db = sdesc_sw128(sb + G_A_BYTES);
+          for (int kk = 0; kk < nk; ++kk) {  // K = 64 E2M1 = 32 bytes per MMA
+            mma_nvfp4(tmem, da + 2 * kk, db + 2 * kk, id_fp4, sfa_t + 4 * kk, sfb_t + 8 * kk,
+                      accumulate);
+            accumulate = 1;
+          }
+          tc_commit(empty0 + 8 * st);
+        }
+        for (int c = 0; c < lr_chunks && !stop; ++c, ++it) {
+          const int st = it % G_STAGES;
+          const uint32_t ph = (it / G_STAGES) & 1;
+          if (!mbar_wait(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) {
+            stop = true;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
+          const uint64_t da = sdesc_sw128(sb), db = sdesc_sw128(sb + G_A_BYTES);
+          const int nks = min(4, (2 * r - 64 * c) >> 4);  // K = 16 bf16 per MMA
+          for (int kk = 0; kk < nks; ++kk) {
+            mma_bf16(tmem, da + 2 * kk, db + 2 * kk, id_lr, accumulate);
+            accumulate = 1;
+          }
+          tc_commit(empty0 + 8 * st);
+        }
+        tc_commit(acc_full);
+      }
+    }
+  } else {
+    // -------------------------------------------------------- epilogue ----
+    const int quad = warp & 3;
+    const float alpha = p.alpha;
+    int tcount = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
+      const int mb = tile % num_m, nb = tile / num_m;
+      if (!mbar_wait(acc_full, tcount & 1, p.timeout_ns, abort_flag, (4u << 8) | kid)) break;
+      tc_fence_after();
+      const int row = mb * G_BM + quad * 32 + lane;
+      const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
+      uint16_t* yrow = p.Y + (size_t)row * p.ldy;
+      for (int ch = 0; ch < G_BN / 16; ++ch) {
+        uint32_t acc[16];
+        tmem_ld16(tbase + 16 * ch, acc);
+        tmem_wait_ld();
+        const int n0 = nb * G_BN + 16 * ch;
+        if (n0 >= N) continue;
+        float b[16];
+        if (p.bias) {
+          const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0);
+          const uint4 b0 = __ldg(bp), b1 = __ldg(bp + 1);
+          const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            b[2 * j] = bf16_lo_f32(bw[j]);
+            b[2 * j + 1] = bf16_hi_f32(bw[j]);
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) b[j] = 0.0f;
+        }
+        uint32_t out[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float y0 = fmaf(alpha, __uint_as_float(acc[2 * j]), b[2 * j]);
+          const float y1 = fmaf(alpha, __uint_as_float(acc[2 * j + 1]), b[2 * j + 1]);
+          __nv_bfloat162 v = __floats2bfloat162_rn(y0, y1);
+          out[j] = *reinterpret_cast<uint32_t*>(&v);
+        }
+        if (row < M) {
+          uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
+          dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
+          dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(acc_empty);
+    }
+  }
+
+  // ------------------------------------------------------------ teardown ----
+  tc_fence_before();
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == 0 && lane == 0) {
+      for (int i = max(0, issued - G_STAGES); i < issued; ++i)
+        mbar_wait_drain(full0 + 8 * (i % G_STAGES), (i / G_STAGES) & 1, p.timeout_ns);
+    }
+    if (warp == 1 && lane == 0) {
+      tc_commit(drain_bar);
+      mbar_wait_drain(drain_bar, 0, p.timeout_ns);
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, G_TMEM_COLS);
+  }
+}
+
+}  // namespace svdq_dev
