@@ -1,0 +1,425 @@
+"""Throughput of the SVDQuant W4A4 (NVFP4) linear on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload flux_qkv] [--sets 4] [--no-e2e] [--no-cpu-baseline]
+
+One step = one pass of the whole hot path over one batch: the activation
+kernel (smoothing, NVFP4 quantization, fused low-rank down-projection) and
+the 4-bit GEMM kernel (fused up-projection, bias, bf16 store) of one
+Flux-shaped linear.  Default workload: the fused QKV projection, M = 4608
+tokens, K = 3072, N = 9216, rank 32, synthetic seeded data.
+
+With N > 1 (launched by torchrun) every rank runs its own batch of tokens
+through a replica of the layer (weak scaling, no data-path collective); the
+time is the max over ranks.  Rank 0 prints one JSON line.
+
+--impl reference runs the CPU oracle (the test reference implementation)
+on the host cores instead, on a bounded sample of rows per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import svdq_inputs as SI  # noqa: E402
+
+METRIC = "svdq W4A4 linear effective TFLOPS & % of dense NVFP4 peak; µs/layer @M=4608"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0            # nominal dense ratio 9 / 2.25 PFLOP/s
+KERNEL_SOURCES = ["w4a4_rank_corrected_b200/csrc/w4a4_gemm.cuh",
+                  "w4a4_rank_corrected_b200/csrc/quantize_act.cuh",
+                  "w4a4_rank_corrected_b200/csrc/ptx.cuh",
+                  "w4a4_rank_corrected_b200/csrc/svdq_api.cu"]
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="flux_qkv")
+    ap.add_argument("--sets", type=int, default=4, help="rotating input/weight/output sets")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=50)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------- helpers ----
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_activations(spec, rank: int, M: int, K: int) -> np.ndarray:
+    """Rank 0 uses the workload's own draw; rank r > 0 its own batch of
+    tokens with the same value model (independent seed)."""
+    if rank == 0:
+        return SI.make_workload(spec.name).X_bf16
+    rng = np.random.default_rng(spec.seed * 1000003 + rank)
+    return SI.draw_activations(rng, M, K, spec.x_dist, spec.x_outliers, spec.x_scale)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary of `kernel`,
+    or None when there is none or the kernel sources changed since."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if "=" in line and not line.lstrip().startswith("#"):
+            k, v = line.split("=", 1)
+            vals[k.strip()] = v.strip()
+    if vals.get("source_sha") != kernel_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons in the
+    background while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"svdq_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.gpu)], stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                rows.append({"sm": float(parts[1]), "max": float(parts[2]), "util": float(parts[4]),
+                             "hw": parts[6], "hwt": parts[7], "swt": parts[8], "pc": parts[9]})
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        load = [r for r in rows if r["util"] > 0] or rows
+        if not load:
+            return {"samples": 0}
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pc", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load),
+                "sm_max_mhz": max(r["max"] for r in load), "reasons": sorted(reasons),
+                "samples": len(load)}
+
+
+# --------------------------------------------------------------- ours ----
+
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    import w4a4_rank_corrected_b200 as S
+
+    spec = SI.workload_specs()[args.workload]
+    ls = spec.layers[0]
+    M, K, N, r = ls.M, ls.K, ls.N, ls.r
+    wl = SI.make_workload(spec.name)
+    W, bias = wl.layers[0].W, wl.layers[0].bias_bf16
+    X0 = wl.X_bf16 if rank == 0 else rank_activations(spec, rank, M, K)
+    cx = SI.channel_absmax(X0)
+    packed = S.svdq_pack_weight(W, cx, r)
+
+    nsets = max(1, args.sets)
+    weights = [packed.to_device(dev, bias) for _ in range(nsets)]
+    Xs = [torch.from_numpy(X0.view(np.int16)).to(dev).view(torch.bfloat16) for _ in range(nsets)]
+    Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(nsets)]
+    klr = ((2 * r + 63) // 64) * 64
+    sf_bytes = ((M + 127) // 128) * 128 * (K // 16)
+    codes = [torch.empty((M, K // 2), dtype=torch.uint8, device=dev) for _ in range(nsets)]
+    sfs = [torch.empty(sf_bytes, dtype=torch.uint8, device=dev) for _ in range(nsets)]
+    xl1s = [torch.empty((M, klr), dtype=torch.bfloat16, device=dev) if r else None
+            for _ in range(nsets)]
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        j = i % nsets
+        S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j], stream)
+        S.svdq_gemm(weights[j], codes[j], sfs[j], xl1s[j], M, Ys[j], stream)
+
+    sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ
+                           else int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local]))
+    sampler.start()
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+
+    K_steps = args.steps
+    stride = max(1, K_steps // 1000)
+    ev_start = torch.cuda.Event(enable_timing=True)
+    ev_end = torch.cuda.Event(enable_timing=True)
+    marks = []
+    ev_start.record(stream)
+    for i in range(K_steps):
+        if i % stride == 0:
+            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            j = i % nsets
+            e0.record(stream)
+            S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j], stream)
+            e1.record(stream)
+            S.svdq_gemm(weights[j], codes[j], sfs[j], xl1s[j], M, Ys[j], stream)
+            e2.record(stream)
+            marks.append((e0, e1, e2))
+        else:
+            step(i)
+    ev_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    elapsed_ms = max_over_ranks(ev_start.elapsed_time(ev_end), world, dev)
+    err = S.svdq_device_error(stream)
+    if err:
+        raise SystemExit(f"device error code {err:#x}")
+
+    q_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in marks)
+    g_ms = statistics.mean(b.elapsed_time(c) for _, b, c in marks)
+    ms_per_step = elapsed_ms / K_steps
+    flops = 2.0 * M * N * K
+    value = world * flops * K_steps / (elapsed_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    fp4_sust = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]) * FP4_OVER_BF16
+    fp4_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]) * FP4_OVER_BF16
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    gemm_tflops = flops / (g_ms * 1e-3) / 1e12
+    q_bytes = M * K * 2 + M * K // 2 + M * K // 16 + (M * klr * 2 + 2 * r * K * 2 if r else 0) + K * 4
+    q_gbs = q_bytes / (q_ms * 1e-3) / 1e9
+    traffic = profiled_traffic("w4a4_gemm", args.workload)
+
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOPS", "n_gpus": world,
+        "steps": K_steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
+        "data": "synthetic",
+        "config": {
+            "workload": f"{spec.name}: {spec.description}", "M": M, "K": K, "N": N, "r": r,
+            "global_batch": M * world, "parallelism": f"dp{world} (independent replicas, no collective)",
+            "l2": f"{nsets} rotating input/weight/output sets (~{nsets * (M * K * 2 + M * N * 2 + N * K // 2) / 1e6:.0f} MB > 126 MB L2)",
+            "us_per_layer": round(ms_per_step * 1e3, 2),
+            "us_quantize_act": round(q_ms * 1e3, 2), "us_gemm": round(g_ms * 1e3, 2),
+            "gemm_tflops": round(gemm_tflops, 1),
+            "pct_fp4_peak_sustained": round(100 * gemm_tflops / fp4_sust, 1),
+            "pct_fp4_peak_burst": round(100 * gemm_tflops / fp4_burst, 1),
+            "pct_fp4_datasheet_9pf": round(100 * gemm_tflops / 9000.0, 1),
+            "quantize_act_gbs": round(q_gbs, 1), "quantize_act_pct_hbm": round(100 * q_gbs / hbm, 1),
+            "layer_roofline_frac": round(max(flops / (fp4_sust * 1e12), (q_bytes + M * N * 2) / (hbm * 1e9)) / (ms_per_step * 1e-3), 3),
+        },
+        "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_sust, 1),
+                     "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_sust, 4), "traffic": traffic,
+                     "kernel": "w4a4_gemm_kernel",
+                     "peak_source": f"{peak_src} bf16_tflops_sustained x {FP4_OVER_BF16:g} (nominal FP4/BF16 dense ratio)"},
+        "gpu_launches": 2 * K_steps,
+        "clocks": clocks,
+    }
+
+    if not args.no_e2e:
+        out["e2e"] = e2e_leg(S, weights[0], X0, M, K, N, r, dev, stream, args.e2e_steps, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(spec, W, bias, X0, packed, r, budget_s=15.0)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def e2e_leg(S, w, X0, M, K, N, r, dev, stream, steps, world):
+    """The same metric through the public forward call with host buffers:
+    every step copies X from pinned host memory and Y back to it."""
+    import torch
+    Xh = torch.from_numpy(X0.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    Xd = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+    Yd = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(S.svdq_act_workspace_bytes(M, K, r), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        S.svdq_linear_forward_host(w, Xh, Yh, Xd, Yd, ws, stream)
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        S.svdq_linear_forward_host(w, Xh, Yh, Xd, Yd, ws, stream)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(a.elapsed_time(b), world, dev) / steps
+    return {"value": round(world * 2.0 * M * N * K / (ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
+            "ms_per_step": round(ms, 4), "h2d_bytes_per_step": M * K * 2,
+            "d2h_bytes_per_step": M * N * 2}
+
+
+def _oracle_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def cpu_baseline(spec, W, bias, X0, packed, r, budget_s=15.0, rows=None):
+    """The oracle as it stands, on a bounded sample of rows of the same
+    workload, timed on the host cores; scaled to effective TFLOPS."""
+    from oracle import svdq as O
+    cx = SI.channel_absmax(X0)
+    op = O.pack(W, cx, r, L1=packed.l1, L2=packed.l2) if r else O.pack(W, cx, 0)
+    M, K = X0.shape
+    N = W.shape[0]
+    if rows is None:
+        t0 = time.perf_counter()
+        O.linear_reference(X0, op, bias, rows=np.arange(8))
+        per_row = (time.perf_counter() - t0) / 8
+        rows = int(max(8, min(M, budget_s / max(per_row, 1e-6))))
+    idx = np.arange(rows)
+    t0 = time.perf_counter()
+    O.linear_reference(X0, op, bias, rows=idx)
+    dt = time.perf_counter() - t0
+    return {"value": round(2.0 * rows * N * K / dt / 1e12, 6), "unit": "TFLOPS",
+            "cores": _oracle_threads(), "kind": "oracle",
+            "sample": f"first {rows} of {M} rows of {spec.name} (activation NVFP4 + float64 dequantized GEMM + low-rank branch + bias), {dt:.2f} s"}
+
+
+# ---------------------------------------------------------- reference ----
+
+def run_reference(args):
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    import w4a4_rank_corrected_b200 as S  # host pack only (the oracle takes its factors)
+    from oracle import svdq as O
+    spec = SI.workload_specs()[args.workload]
+    ls = spec.layers[0]
+    M, K, N, r = ls.M, ls.K, ls.N, ls.r
+    wl = SI.make_workload(spec.name)
+    W, bias, X0 = wl.layers[0].W, wl.layers[0].bias_bf16, wl.X_bf16
+    cx = SI.channel_absmax(X0)
+    packed = S.svdq_pack_weight(W, cx, r)
+    op = O.pack(W, cx, r, L1=packed.l1, L2=packed.l2) if r else O.pack(W, cx, 0)
+    t0 = time.perf_counter()
+    O.linear_reference(X0, op, bias, rows=np.arange(4))
+    per_row = (time.perf_counter() - t0) / 4
+    total_budget = 120.0
+    rows = int(max(1, min(M, total_budget / max(1, args.steps + args.warmup) / max(per_row, 1e-6))))
+    for i in range(args.warmup):
+        O.linear_reference(X0, op, bias, rows=(np.arange(rows) + i * rows) % M)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        O.linear_reference(X0, op, bias, rows=(np.arange(rows) + i * rows) % M)
+    dt = time.perf_counter() - t0
+    value = 2.0 * rows * N * K * args.steps / dt / 1e12
+    cores = _oracle_threads()
+    out = {"metric": METRIC, "value": round(value, 6), "unit": "TFLOPS", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "impl": "reference",
+           "config": {"workload": f"{spec.name}: {spec.description}", "M": M, "K": K, "N": N,
+                      "r": r, "rows_per_step": rows},
+           "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": cores,
+                            "kind": "oracle",
+                            "sample": f"{rows} rows of {M} per step (activation NVFP4 + float64 dequantized GEMM + low-rank branch + bias)"},
+           "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()
