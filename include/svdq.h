@@ -94,10 +94,11 @@ svdq_status svdq_query_sizes(int N, int K, int r, svdq_sizes* out);
  *      Rayleigh-Ritz, seeded): L1 = V sqrt(S) [K x r], L2 = sqrt(S) U^T
  *      [r x N], each rounded once to bf16.
  *   3. residual R = fp32(W~ - (L1 L2)^T) (float64 sum over rank ascending).
- *   4. NVFP4 of R: g_w = 2688 / max|R|; per 16 along K:
- *      sf = E4M3(fp32(a/6) * g_w), code = E2M1(R * fp32(g_w / sf)).
+ *   4. NVFP4 of R with A_w = max|R|: g_w = 2688/A_w, gs_w = 448/A_w; per
+ *      16 along K: sf = E4M3(a * gs_w), code = E2M1(R * fp32(g_w / sf)).
  *   5. activation tensor scale from calibration:
- *      g_x = 2688 / max_j fp32(x_absmax_j * smooth_j).
+ *      A_x = max_j fp32(x_absmax_j * smooth_j); g_x = 2688/A_x,
+ *      gs_x = 448/A_x (g = gs = 1 when A = 0).
  *   6. lr_scale = fp32(g_x * g_w), alpha = fp32(1 / lr_scale).
  *   7. kernel operands: l1_mma[i][k] = bf16 hi part and l1_mma[r+i][k] =
  *      bf16 lo part of smooth_k * L1[k][i] (exact product in float64, hi =
@@ -121,7 +122,8 @@ typedef struct svdq_packed_host {
   uint16_t* l2_mma;      /* [N][klr]   */
   uint8_t*  codes_w;     /* [N][K/2], even k in the low nibble             */
   uint8_t*  sf_w;        /* MMA tile layout (svdq_sf_tile_offset)          */
-  float g_x, g_w, alpha, lr_scale;
+  float amax_x, amax_w;  /* static activation absmax A_x, residual absmax A_w */
+  float g_x, gs_x, g_w, alpha, lr_scale;
 } svdq_packed_host;
 
 svdq_status svdq_pack_weight(const float* W, const float* x_absmax, int N,
@@ -143,7 +145,7 @@ int64_t svdq_sf_tile_offset(int row, int g, int K);
  */
 typedef struct svdq_weight {
   int N, K, r;
-  float g_x, g_w, alpha, lr_scale;
+  float g_x, gs_x, g_w, alpha, lr_scale;
   const float*    smooth;   /* device fp32 [K], 16-byte aligned            */
   const uint16_t* l1_mma;   /* device bf16 [2r][K]        (NULL if r == 0) */
   const uint16_t* l2_mma;   /* device bf16 [N][klr]       (NULL if r == 0) */
@@ -158,8 +160,9 @@ typedef struct svdq_weight {
 size_t svdq_act_workspace_bytes(int M, int K, int r);
 
 /* svdq_quantize_act: activation kernel (one launch).  For every row of X:
- * x_hat = fp32(x * smooth); NVFP4 with the static g_x (per 16-group max by
- * warp shuffles, E4M3 scale, E2M1 codes, two per byte); and, fused, the
+ * x_hat = fp32(x * smooth); NVFP4 with the static tensor scales g_x, gs_x
+ * (per 16-group max, sf = E4M3(a * gs_x), codes = E2M1(x_hat * g_x / sf),
+ * two per byte); and, fused, the
  * down-projection X_hat L1 on the tensor cores, written pre-multiplied by
  * lr_scale as a bf16 hi/lo pair: xl1[m][i] + xl1[m][r+i] ~= lr_scale *
  * (X_hat L1)[m][i], zeros in columns [2r, klr).

@@ -27,17 +27,19 @@ Readings of what the pages leave open (each is also listed in the design doc):
   R3 residual: R_nk = fp32( W~_nk - sum_{i ascending} L1_ki * L2_in ), the
      sum in float64.
   R4 NVFP4 recipe for a tensor T with tensor absmax A (fp32):
-       g   = fp32(2688 / A)            (2688 = 6 * 448; g = 1 if A = 0)
+       g   = fp32(2688 / A)            element encode scale (2688 = 6 * 448)
+       gs  = fp32(448 / A)             block-scale encode scale (= g / 6)
+       (g = gs = 1 if A = 0)
        per group G of 16 consecutive elements along K:
        a   = max_{t in G} |t|
-       sf  = E4M3_rn_satfinite( fp32( fp32(a / 6) * g ) )
+       sf  = E4M3_rn_satfinite( fp32(a * gs) )
        q   = 0 if sf == 0 else fp32( g / e4m3(sf) )
        code= E2M1_rn_satfinite( fp32(t * q) )
      dequantized value = e2m1(code) * e4m3(sf) / g.
   R5 activation tensor scale is static (from calibration):
      A_x = max_j fp32(cx_j * s_j), which equals max |x_hat| over the
-     calibration batch (rounding is monotone).  Run-time values beyond it
-     saturate (satfinite).
+     calibration batch (rounding is monotone); g_x, gs_x follow R4.
+     Run-time values beyond it saturate (satfinite).
   R6 reference output: Y_ref = D / (g_x g_w) + (X_hat L1) L2 + bias in
      float64, D = deq(codes_x, sf_x) deq(codes_w, sf_w)^T (the codes are
      the method's own 4-bit encodings; 1/(g_x g_w) undoes both tensor
@@ -137,18 +139,26 @@ def tensor_encode_scale(amax) -> np.float32:
     return F32(NVFP4_AMAX_TARGET / amax)
 
 
-def nvfp4_quantize(T: np.ndarray, g) -> Tuple[np.ndarray, np.ndarray]:
-    """Reading R4.  T: float32 [rows, K] (K % 16 == 0), g: fp32 tensor
-    encode scale.  Returns (codes uint8 [rows, K] one code per byte,
-    sf uint8 [rows, K/16] E4M3 codes)."""
+def block_scale_factor(amax) -> np.float32:
+    """gs = fp32(448 / A); gs = 1 when A = 0 (reading R4)."""
+    amax = F32(amax)
+    if amax == 0:
+        return F32(1.0)
+    return F32(F32(448.0) / amax)
+
+
+def nvfp4_quantize(T: np.ndarray, amax) -> Tuple[np.ndarray, np.ndarray]:
+    """Reading R4.  T: float32 [rows, K] (K % 16 == 0), amax: the fp32
+    tensor absmax A that fixes the tensor scales.  Returns (codes uint8
+    [rows, K] one code per byte, sf uint8 [rows, K/16] E4M3 codes)."""
     T = np.asarray(T, dtype=F32)
     rows, K = T.shape
     assert K % NVFP4_GROUP == 0
-    g = F32(g)
+    g = tensor_encode_scale(amax)
+    gs = block_scale_factor(amax)
     grp = T.reshape(rows, K // NVFP4_GROUP, NVFP4_GROUP)
     a = np.abs(grp).max(axis=2).astype(F32)
-    scaled = ((a / F32(6.0)).astype(F32) * g).astype(F32)
-    sf = e4m3_encode_nonneg(scaled)
+    sf = e4m3_encode_nonneg((a * gs).astype(F32))
     dec = e4m3_decode(sf).astype(F32)
     with np.errstate(divide="ignore"):
         q = np.where(sf == 0, F32(0.0), (g / np.where(sf == 0, F32(1.0), dec)).astype(F32)).astype(F32)
@@ -226,25 +236,32 @@ class OraclePack:
     R: np.ndarray            # fp32 [N, K]
     g_w: np.float32
     g_x: np.float32
+    A_w: np.float32          # tensor absmax of R
+    A_x: np.float32          # static activation absmax (reading R5)
     codes_w: np.ndarray      # uint8 [N, K] (one code per byte)
     sf_w: np.ndarray         # uint8 [N, K/16]
 
 
-def activation_tensor_scale(x_absmax: np.ndarray, s: np.ndarray) -> np.float32:
-    """Reading R5: g_x from A_x = max_j fp32(cx_j * s_j)."""
+def activation_absmax(x_absmax: np.ndarray, s: np.ndarray) -> np.float32:
+    """Reading R5: A_x = max_j fp32(cx_j * s_j)."""
     a = (np.asarray(x_absmax, F32) * np.asarray(s, F32)).astype(F32)
-    return tensor_encode_scale(np.abs(a).max() if a.size else F32(0))
+    return F32(np.abs(a).max()) if a.size else F32(0)
+
+
+def activation_tensor_scale(x_absmax: np.ndarray, s: np.ndarray) -> np.float32:
+    """g_x = fp32(2688 / A_x) (readings R4, R5)."""
+    return tensor_encode_scale(activation_absmax(x_absmax, s))
 
 
 def quantize_weight(W: np.ndarray, s: np.ndarray, L1: np.ndarray,
                     L2: np.ndarray):
     """Steps 2-3 for given smoothing factors and low-rank factors:
-    R, g_w, codes_w, sf_w."""
+    R, A_w, codes_w, sf_w."""
     Wt = smooth_weight(W, s)
     R = residual(Wt, L1, L2)
-    g_w = tensor_encode_scale(np.abs(R).max() if R.size else F32(0))
-    codes, sf = nvfp4_quantize(R, g_w)
-    return R, g_w, codes, sf
+    A_w = F32(np.abs(R).max()) if R.size else F32(0)
+    codes, sf = nvfp4_quantize(R, A_w)
+    return R, A_w, codes, sf
 
 
 def pack(W: np.ndarray, x_absmax: np.ndarray, r: int,
@@ -260,16 +277,17 @@ def pack(W: np.ndarray, x_absmax: np.ndarray, r: int,
             K, N = W.shape[1], W.shape[0]
             L1 = np.zeros((K, 0), np.uint16)
             L2 = np.zeros((0, N), np.uint16)
-    R, g_w, codes, sf = quantize_weight(W, s, L1, L2)
-    g_x = activation_tensor_scale(x_absmax, s)
-    return OraclePack(s, L1, L2, R, g_w, g_x, codes, sf)
+    R, A_w, codes, sf = quantize_weight(W, s, L1, L2)
+    A_x = activation_absmax(x_absmax, s)
+    return OraclePack(s, L1, L2, R, tensor_encode_scale(A_w), tensor_encode_scale(A_x),
+                      A_w, A_x, codes, sf)
 
 
-def quantize_activation(X_bf16: np.ndarray, s: np.ndarray, g_x):
-    """The activation step: smoothing then NVFP4 with the static g_x.
-    Returns (x_hat fp32, codes [M, K], sf [M, K/16])."""
+def quantize_activation(X_bf16: np.ndarray, s: np.ndarray, A_x):
+    """The activation step: smoothing then NVFP4 with the static tensor
+    absmax A_x.  Returns (x_hat fp32, codes [M, K], sf [M, K/16])."""
     xh = smooth_activation(X_bf16, s)
-    codes, sf = nvfp4_quantize(xh, g_x)
+    codes, sf = nvfp4_quantize(xh, A_x)
     return xh, codes, sf
 
 
@@ -284,7 +302,7 @@ def linear_reference(X_bf16: np.ndarray, p: OraclePack,
     """Reading R6: the float64 reference output Y_ref [M, N] (or only the
     listed rows).  Returns (Y_ref, codes_x, sf_x, xl1)."""
     X = X_bf16 if rows is None else X_bf16[rows]
-    xh, cx, sfx = quantize_activation(X, p.s, p.g_x)
+    xh, cx, sfx = quantize_activation(X, p.s, p.A_x)
     D = nvfp4_dequantize(cx, sfx) @ nvfp4_dequantize(p.codes_w, p.sf_w).T
     Y = D / (np.float64(p.g_x) * np.float64(p.g_w))
     xl1 = lowrank_down(xh, p.L1)

@@ -54,7 +54,7 @@ def check_activation(codes_dev, sf_dev, xl1_dev, X_bits, op, M, K, r, rows=None)
     """Bit-exact codes and scales; xl1 hi+lo against lr_scale * X_hat L1."""
     torch = torch_mod()
     idx = np.arange(M) if rows is None else np.asarray(rows)
-    xh, codes, sf = O.quantize_activation(X_bits[idx], op.s, op.g_x)
+    xh, codes, sf = O.quantize_activation(X_bits[idx], op.s, op.A_x)
     got_codes = codes_dev.cpu().numpy()[idx]
     assert np.array_equal(got_codes, O.pack_nibbles(codes)), "activation codes differ"
     tiles = sf_dev.cpu().numpy()

@@ -73,7 +73,7 @@ def test_workspace_bytes():
 def _fake_weight(N=256, K=256, r=32, base=0x10000000):
     w = S.SvdqWeight()
     w.N, w.K, w.r = N, K, r
-    w.g_x = w.g_w = w.alpha = w.lr_scale = 1.0
+    w.g_x = w.gs_x = w.g_w = w.alpha = w.lr_scale = 1.0
     w.smooth, w.l1_mma, w.l2_mma = base, base + 0x1000, base + 0x2000
     w.bias, w.codes_w, w.sf_w = base + 0x3000, base + 0x4000, base + 0x8000
     return w

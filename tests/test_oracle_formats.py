@@ -113,7 +113,7 @@ def test_nvfp4_hand_worked_groups(golden_dir):
     gold = _load_golden(golden_dir)
     for ex in gold["groups"]:
         t = np.array(ex["t"], np.float32)[None, :]
-        codes, sf = O.nvfp4_quantize(t, np.float32(ex["g"]))
+        codes, sf = O.nvfp4_quantize(t, np.float32(ex["amax"]))
         assert int(sf[0, 0]) == ex["sf"], ex["name"]
         assert codes[0].tolist() == ex["codes"], ex["name"]
 
@@ -122,6 +122,7 @@ def test_nvfp4_hand_worked_tensor_scales(golden_dir):
     gold = _load_golden(golden_dir)
     for ex in gold["tensor_scales"]:
         assert O.tensor_encode_scale(np.float32(ex["amax"])) == np.float32(ex["g"])
+        assert O.block_scale_factor(np.float32(ex["amax"])) == np.float32(ex["gs"])
 
 
 def test_nvfp4_error_bound_random():
@@ -130,8 +131,9 @@ def test_nvfp4_error_bound_random():
     v = t * q is the scaled value of reading R4."""
     rng = np.random.default_rng(3)
     T = (rng.standard_normal((64, 256)) * np.exp(rng.standard_normal((64, 1)) * 3)).astype(np.float32)
-    g = O.tensor_encode_scale(np.abs(T).max())
-    codes, sf = O.nvfp4_quantize(T, g)
+    A = np.abs(T).max()
+    g = O.tensor_encode_scale(A)
+    codes, sf = O.nvfp4_quantize(T, A)
     dec = F.e4m3_decode(sf).astype(np.float32)
     q = np.where(sf == 0, 0, g / np.where(sf == 0, 1, dec)).astype(np.float32)
     v = (T.reshape(64, 16, 16) * q[:, :, None]).astype(np.float64).reshape(64, 256)
@@ -140,8 +142,8 @@ def test_nvfp4_error_bound_random():
     bound = np.where(av <= 2, 0.25, np.where(av <= 4, 0.5, 1.0)) + np.maximum(av - 6, 0)
     assert np.all(err <= bound + 1e-12)
     # the group maximum lands within one E4M3 rounding of 6: a normal
-    # (unsaturated) scale is within 2^-4 relative of a*g/6, so
-    # v_max = 6 (a g / 6) / sf lies in [6/(1+2^-4), 6/(1-2^-4)]
+    # (unsaturated) scale is within 2^-4 relative of a*gs = a*g/6 (up to
+    # float32 rounding), so v_max = a g / sf lies in [6/(1+2^-4), 6/(1-2^-4)]
     vmax = av.reshape(64, 16, 16).max(axis=2)
     normal = (sf > 8) & (sf < 126)      # code 8 may be reached from a subnormal y
     assert normal.sum() > 500

@@ -116,9 +116,9 @@ def test_r0_unit_smoothing_is_plain_nvfp4():
     Y, _, _, _ = O.linear_reference(X, p)
     xf = F.bf16_bits_to_f64(X).astype(np.float32)
     gx = O.tensor_encode_scale(np.abs(cx).max())
-    cxq, sxq = O.nvfp4_quantize(xf, gx)
+    cxq, sxq = O.nvfp4_quantize(xf, np.abs(cx).max())
     gw = O.tensor_encode_scale(np.abs(W).max())
-    cwq, swq = O.nvfp4_quantize(W, gw)
+    cwq, swq = O.nvfp4_quantize(W, np.abs(W).max())
     D = O.nvfp4_dequantize(cxq, sxq) @ O.nvfp4_dequantize(cwq, swq).T
     assert np.array_equal(Y, D / (np.float64(gx) * np.float64(gw)))
 

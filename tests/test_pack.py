@@ -19,8 +19,11 @@ def _check_pack(W, cx, r, svd_quality=True):
     s = O.smoothing_factors(cx, W)
     assert np.array_equal(p.smooth, s)
     assert np.float32(p.g_x) == O.activation_tensor_scale(cx, s)
-    R, g_w, codes, sf = O.quantize_weight(W, p.smooth, p.l1, p.l2)
-    assert np.float32(p.g_w) == g_w
+    assert np.float32(p.amax_x) == O.activation_absmax(cx, s)
+    assert np.float32(p.gs_x) == O.block_scale_factor(O.activation_absmax(cx, s))
+    R, A_w, codes, sf = O.quantize_weight(W, p.smooth, p.l1, p.l2)
+    assert np.float32(p.amax_w) == A_w
+    assert np.float32(p.g_w) == O.tensor_encode_scale(A_w)
     assert np.array_equal(p.codes_w, O.pack_nibbles(codes))
     assert np.array_equal(p.sf_w, O.sf_to_mma_tiles(sf, row_multiple=256))
     assert np.float32(p.lr_scale) == np.float32(np.float32(p.g_x) * np.float32(p.g_w))

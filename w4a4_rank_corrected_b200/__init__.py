@@ -55,14 +55,15 @@ class SvdqPackedHost(ctypes.Structure):
     _fields_ = [("smooth", ctypes.c_void_p), ("l1", ctypes.c_void_p), ("l2", ctypes.c_void_p),
                 ("l1_mma", ctypes.c_void_p), ("l2_mma", ctypes.c_void_p),
                 ("codes_w", ctypes.c_void_p), ("sf_w", ctypes.c_void_p),
-                ("g_x", ctypes.c_float), ("g_w", ctypes.c_float), ("alpha", ctypes.c_float),
-                ("lr_scale", ctypes.c_float)]
+                ("amax_x", ctypes.c_float), ("amax_w", ctypes.c_float),
+                ("g_x", ctypes.c_float), ("gs_x", ctypes.c_float), ("g_w", ctypes.c_float),
+                ("alpha", ctypes.c_float), ("lr_scale", ctypes.c_float)]
 
 
 class SvdqWeight(ctypes.Structure):
     _fields_ = [("N", ctypes.c_int), ("K", ctypes.c_int), ("r", ctypes.c_int),
-                ("g_x", ctypes.c_float), ("g_w", ctypes.c_float), ("alpha", ctypes.c_float),
-                ("lr_scale", ctypes.c_float), ("smooth", ctypes.c_void_p),
+                ("g_x", ctypes.c_float), ("gs_x", ctypes.c_float), ("g_w", ctypes.c_float),
+                ("alpha", ctypes.c_float), ("lr_scale", ctypes.c_float), ("smooth", ctypes.c_void_p),
                 ("l1_mma", ctypes.c_void_p), ("l2_mma", ctypes.c_void_p),
                 ("bias", ctypes.c_void_p), ("codes_w", ctypes.c_void_p),
                 ("sf_w", ctypes.c_void_p)]
@@ -138,7 +139,10 @@ class PackedWeight:
     l2_mma: np.ndarray       # bf16 [N, klr]
     codes_w: np.ndarray      # u8 [N, K/2]
     sf_w: np.ndarray         # u8, MMA tiles
+    amax_x: float
+    amax_w: float
     g_x: float
+    gs_x: float
     g_w: float
     alpha: float
     lr_scale: float
@@ -166,7 +170,8 @@ class DeviceWeight:
         self.tensors = tensors
         s = SvdqWeight()
         s.N, s.K, s.r = packed.N, packed.K, packed.r
-        s.g_x, s.g_w, s.alpha, s.lr_scale = packed.g_x, packed.g_w, packed.alpha, packed.lr_scale
+        s.g_x, s.gs_x, s.g_w = packed.g_x, packed.gs_x, packed.g_w
+        s.alpha, s.lr_scale = packed.alpha, packed.lr_scale
         for name in ("smooth", "l1_mma", "l2_mma", "bias", "codes_w", "sf_w"):
             t = tensors.get(name)
             setattr(s, name, t.data_ptr() if t is not None else None)
@@ -212,7 +217,8 @@ def svdq_pack_weight(W: np.ndarray, x_absmax: np.ndarray, r: int, smooth_alpha: 
                                 float(smooth_alpha), int(seed), ctypes.byref(out)),
            "svdq_pack_weight")
     return PackedWeight(N, K, r, sz.klr, smooth, l1, l2, l1m, l2m, codes, sf,
-                        float(out.g_x), float(out.g_w), float(out.alpha), float(out.lr_scale))
+                        float(out.amax_x), float(out.amax_w), float(out.g_x), float(out.gs_x),
+                        float(out.g_w), float(out.alpha), float(out.lr_scale))
 
 
 # ------------------------------------------------------------- forward ----

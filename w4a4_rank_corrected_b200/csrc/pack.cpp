@@ -94,6 +94,9 @@ static inline float e4m3_value(uint8_t c) {
 static inline float tensor_scale(float amax) {
   return amax > 0.0f ? 2688.0f / amax : 1.0f;
 }
+static inline float block_scale_factor(float amax) {
+  return amax > 0.0f ? 448.0f / amax : 1.0f;
+}
 
 // --------------------------------------------------------------- rng ----
 
@@ -293,7 +296,7 @@ int64_t sf_tile_offset(int row, int g, int K) {
 
 // NVFP4 of rows x K float32 (row-major): codes two per byte (even k low
 // nibble) and E4M3 scales in the MMA tile layout.
-static void quantize_nvfp4_rows(const float* T, int rows, int K, float g,
+static void quantize_nvfp4_rows(const float* T, int rows, int K, float g, float gs,
                                 uint8_t* codes, uint8_t* sf_tiled) {
 #pragma omp parallel for schedule(static)
   for (int n = 0; n < rows; ++n) {
@@ -301,8 +304,7 @@ static void quantize_nvfp4_rows(const float* T, int rows, int K, float g,
     for (int gi = 0; gi < K / 16; ++gi) {
       float a = 0.0f;
       for (int j = 0; j < 16; ++j) a = std::max(a, std::fabs(t[gi * 16 + j]));
-      const float y = (a / 6.0f) * g;
-      const uint8_t s = e4m3_code(y);
+      const uint8_t s = e4m3_code(a * gs);
       const float q = (s == 0) ? 0.0f : g / e4m3_value(s);
       sf_tiled[sf_tile_offset(n, gi, K)] = s;
       for (int j = 0; j < 16; j += 2) {
@@ -416,7 +418,7 @@ extern "C" svdq_status svdq_pack_weight(const float* W, const float* x_absmax,
   // 4. NVFP4 of R
   const float g_w = tensor_scale(amax);
   std::memset(out->sf_w, 0, sz.sf_w_bytes);
-  quantize_nvfp4_rows(R.data(), N, K, g_w, out->codes_w, out->sf_w);
+  quantize_nvfp4_rows(R.data(), N, K, g_w, block_scale_factor(amax), out->codes_w, out->sf_w);
 
   // 5. static activation tensor scale
   float ax = 0.0f;
@@ -425,7 +427,10 @@ extern "C" svdq_status svdq_pack_weight(const float* W, const float* x_absmax,
 
   // 6. output scale and its inverse for the low-rank branch
   const float lr_scale = g_x * g_w;
+  out->amax_x = ax;
+  out->amax_w = amax;
   out->g_x = g_x;
+  out->gs_x = block_scale_factor(ax);
   out->g_w = g_w;
   out->lr_scale = lr_scale;
   out->alpha = 1.0f / lr_scale;

@@ -61,6 +61,13 @@ struct DeviceInfo {
   bool ok = false;
   int num_sms = 0;
   bool attrs_set = false;
+  // max co-resident clusters of the activation kernel, per rank r/16 (0..8)
+  // and cluster size S (1..8); -1 = not queried yet
+  int max_clusters[9][9];
+  DeviceInfo() {
+    for (auto& a : max_clusters)
+      for (int& v : a) v = -1;
+  }
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -87,8 +94,10 @@ svdq_status device_check(int* sms) {
   }
   if (!d.ok) return SVDQ_ERR_UNSUPPORTED_ARCH;
   if (!d.attrs_set) {
+    uint32_t qa_max = 0;
+    for (int rr = 0; rr <= 128; rr += 16) qa_max = std::max(qa_max, qa_smem_bytes(rr));
     if (cudaFuncSetAttribute(quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)qa_smem_bytes(128)) != cudaSuccess ||
+                             (int)qa_max) != cudaSuccess ||
         cudaFuncSetAttribute(w4a4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)gemm_smem_bytes()) != cudaSuccess) {
       cudaGetLastError();
@@ -142,21 +151,66 @@ svdq_status check_weight(const svdq_weight* w) {
 
 int klr_of(int r) { return (int)rup((size_t)2 * r, 64); }
 
+cudaLaunchAttribute pdl_attr() {
+  cudaLaunchAttribute a;
+  a.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  a.val.programmaticStreamSerializationAllowed = 1;
+  return a;
+}
+
+// Largest K split S (cluster size when the low-rank branch needs the
+// cross-CTA reduction) such that the whole grid is resident in one wave.
+int choose_splits(int tiles, int kchunks, int r, int sms) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int best = 1;
+  for (int S = 2; S <= 8; ++S) {
+    if (S > kchunks || tiles * S > sms) break;
+    if (r > 0) {
+      int& cached = g_dev[dev].max_clusters[r / 16][S];
+      if (cached < 0) {
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3((unsigned)S, 1, 1);
+        cfg.blockDim = dim3(QA_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = qa_smem_bytes(r);
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = (unsigned)S;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, quantize_act_kernel, &cfg) != cudaSuccess) {
+          cudaGetLastError();
+          n = 0;
+        }
+        cached = n;
+      }
+      if (tiles > cached) continue;
+    }
+    best = S;
+  }
+  return best;
+}
+
 svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int64_t ldx,
                             uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, cudaStream_t s,
                             int sms) {
   const int K = w->K, r = w->r;
-  const int RB = (M + 127) / 128;
+  // 64-row tiles covering whole 128-row scale atoms (padding rows get zero
+  // scales)
+  const int tiles = 2 * ((M + 127) / 128);
   const int KC = K / 64;
-  int S = std::max(1, std::min(8, sms / std::max(1, RB)));
-  S = std::min(S, KC);
+  int S = choose_splits(tiles, KC, r, sms);
   const int cps = (KC + S - 1) / S;
   S = (KC + cps - 1) / cps;
 
   CUtensorMap tm_x, tm_l1;
   std::memset(&tm_l1, 0, sizeof(tm_l1));
   if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M,
-                (uint64_t)ldx * 2, 64, 128))
+                (uint64_t)ldx * 2, 64, QA_BM))
     return SVDQ_ERR_CUDA;
   if (r > 0 && !make_map(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l1_mma, (uint64_t)K,
                          (uint64_t)(2 * r), (uint64_t)K * 2, 64, (uint32_t)(2 * r)))
@@ -173,29 +227,32 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
   p.klr = klr_of(r);
   p.chunks_per_split = cps;
   p.num_splits = S;
+  p.stages = qa_stages(r);
   p.stage_bytes = qa_stage_bytes(r);
   uint32_t cols = 32;
   while (cols < (uint32_t)(2 * r)) cols <<= 1;
   p.tmem_cols = cols;
   p.g_x = w->g_x;
+  p.gs_x = w->gs_x;
   p.lr_scale = w->lr_scale;
   p.timeout_ns = kDefaultTimeoutNs;
 
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3((unsigned)S, (unsigned)RB, 1);
+  cfg.gridDim = dim3((unsigned)S, (unsigned)tiles, 1);
   cfg.blockDim = dim3(QA_THREADS, 1, 1);
   cfg.dynamicSmemBytes = qa_smem_bytes(r);
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
+  attr[0] = pdl_attr();
   cfg.attrs = attr;
-  cfg.numAttrs = 0;
+  cfg.numAttrs = 1;
   if (r > 0 && S > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)S;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.numAttrs = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)S;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
   }
   if (cudaLaunchKernelEx(&cfg, quantize_act_kernel, tm_x, tm_l1, p) != cudaSuccess) {
     cudaGetLastError();
@@ -238,8 +295,20 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   p.timeout_ns = kDefaultTimeoutNs;
   const int tiles = ((M + G_BM - 1) / G_BM) * ((N + G_BN - 1) / G_BN);
   const int grid = std::max(1, std::min(tiles, sms));
-  w4a4_gemm_kernel<<<grid, G_THREADS, gemm_smem_bytes(), s>>>(ta, tb, talr, tblr, p);
-  if (cudaGetLastError() != cudaSuccess) return SVDQ_ERR_CUDA;
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.blockDim = dim3(G_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = gemm_smem_bytes();
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0] = pdl_attr();
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, w4a4_gemm_kernel, ta, tb, talr, tblr, p) != cudaSuccess) {
+    cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
   return SVDQ_OK;
 }
 

@@ -18,15 +18,19 @@
 //     operands (xl1 hi|lo [128 x 2r] and L2 [256 x 2r], bf16) through the
 //     same ring and accumulates xl1 . L2 into the SAME accumulator with
 //     kind::f16 MMAs (xl1 was pre-multiplied by g_x g_w = 1/alpha);
-//   * warps 2..5 drain the accumulator (tcgen05.ld), compute
-//     Y = bf16(alpha * acc + bias) and store it.
+//   * warps 2..9 (two per tensor-memory lane quarter, 128 columns each)
+//     drain the accumulator with four 32-column tcgen05.ld and ONE wait,
+//     release it to the MMA warp at once, and only then compute
+//     Y = bf16(alpha * acc + bias) (bias staged per tile in shared memory)
+//     and store, overlapping the next tile's main loop.
 #pragma once
 #include "ptx.cuh"
 
 namespace svdq_dev {
 
 constexpr int G_STAGES = 4;
-constexpr int G_THREADS = 192;
+constexpr int G_EPI_WARPS = 8;
+constexpr int G_THREADS = 32 * (2 + G_EPI_WARPS);
 constexpr int G_BM = 128, G_BN = 256;
 constexpr uint32_t G_A_BYTES = 128 * 128;    // 128 rows x 128 B
 constexpr uint32_t G_B_BYTES = 256 * 128;    // 256 rows x 128 B
@@ -37,8 +41,10 @@ constexpr uint32_t G_TMEM_COLS = 512;
 constexpr uint32_t G_SF_TMEM = 256;          // scale buffers after the accumulator
 constexpr uint32_t G_SF_TMEM_STRIDE = 48;    // 16 cols SFA + 32 cols SFB
 
+constexpr uint32_t G_BIAS_BYTES = 2 * G_BN * 4;   // two fp32 bias tiles
+
 __host__ __device__ inline uint32_t gemm_smem_bytes() {
-  return 1024u + G_STAGES * G_STAGE_BYTES + 256u;
+  return 1024u + G_STAGES * G_STAGE_BYTES + G_BIAS_BYTES + 256u;  // + barriers
 }
 
 struct GemmParams {
@@ -60,13 +66,15 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G_STAGES * G_STAGE_BYTES);
+  float* bias_s = reinterpret_cast<float*>(smem + G_STAGES * G_STAGE_BYTES);  // [2][256]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G_STAGES * G_STAGE_BYTES + G_BIAS_BYTES);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * G_STAGES;
   const uint32_t acc_full = full0 + 16 * G_STAGES;
   const uint32_t acc_empty = acc_full + 8;
   const uint32_t drain_bar = acc_full + 16;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * G_STAGES + 3);
+  const uint32_t bias_bar0 = acc_full + 24;  // two: one per bias buffer
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * G_STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const uint32_t warp = warp_id(), lane = lane_id();
@@ -86,8 +94,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       mbar_init(empty0 + 8 * i, 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 128);
+    mbar_init(acc_empty, 32 * G_EPI_WARPS);
     mbar_init(drain_bar, 1);
+    mbar_init(bias_bar0, 32 * G_EPI_WARPS);
+    mbar_init(bias_bar0 + 8, 32 * G_EPI_WARPS);
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -107,6 +117,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // The prologue above overlaps the previous kernel; the activation codes,
+  // scales and low-rank operand it produced are read only after this.
+  grid_dependency_wait();
+  grid_launch_dependents();
 
   int issued = 0;
   if (warp == 0) {
@@ -212,52 +226,58 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     }
   } else {
     // -------------------------------------------------------- epilogue ----
-    const int quad = warp & 3;
+    const int quad = warp & 3;                 // tensor-memory lane quarter
+    const int half = (warp - 2) >> 2;          // columns [128 half, 128 half + 128)
+    const int et = threadIdx.x - 64;           // 0..255
     const float alpha = p.alpha;
     int tcount = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
       const int mb = tile % num_m, nb = tile / num_m;
-      if (!mbar_wait(acc_full, tcount & 1, p.timeout_ns, abort_flag, (4u << 8) | kid)) break;
+      // stage this tile's bias (fp32) while the main loop runs.  Buffer
+      // tcount&1 was last read for tile tcount-2, which every thread had
+      // finished before arriving on the other buffer's barrier.
+      float* bt = bias_s + (tcount & 1) * G_BN;
+      const uint32_t bb = bias_bar0 + 8 * (tcount & 1);
+      {
+        const int n = nb * G_BN + et;
+        bt[et] = (p.bias && n < N) ? bf16_lo_f32(p.bias[n]) : 0.0f;
+      }
+      mbar_arrive(bb);
+      if (!mbar_wait_warp(bb, (tcount >> 1) & 1, p.timeout_ns, abort_flag, (5u << 8) | kid)) break;
+      if (!mbar_wait_warp(acc_full, tcount & 1, p.timeout_ns, abort_flag, (4u << 8) | kid)) break;
       tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + half * 128;
+      uint32_t acc[4][32];
+      tmem_ld32(tbase, acc[0]);
+      tmem_ld32(tbase + 32, acc[1]);
+      tmem_ld32(tbase + 64, acc[2]);
+      tmem_ld32(tbase + 96, acc[3]);
+      tmem_wait_ld();
+      tc_fence_before();
+      mbar_arrive(acc_empty);                  // the accumulator is free again
       const int row = mb * G_BM + quad * 32 + lane;
-      const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
       uint16_t* yrow = p.Y + (size_t)row * p.ldy;
-      for (int ch = 0; ch < G_BN / 16; ++ch) {
-        uint32_t acc[16];
-        tmem_ld16(tbase + 16 * ch, acc);
-        tmem_wait_ld();
-        const int n0 = nb * G_BN + 16 * ch;
-        if (n0 >= N) continue;
-        float b[16];
-        if (p.bias) {
-          const uint4* bp = reinterpret_cast<const uint4*>(p.bias + n0);
-          const uint4 b0 = __ldg(bp), b1 = __ldg(bp + 1);
-          const uint32_t bw[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            b[2 * j] = bf16_lo_f32(bw[j]);
-            b[2 * j + 1] = bf16_hi_f32(bw[j]);
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) b[j] = 0.0f;
-        }
-        uint32_t out[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float y0 = fmaf(alpha, __uint_as_float(acc[2 * j]), b[2 * j]);
-          const float y1 = fmaf(alpha, __uint_as_float(acc[2 * j + 1]), b[2 * j + 1]);
-          __nv_bfloat162 v = __floats2bfloat162_rn(y0, y1);
-          out[j] = *reinterpret_cast<uint32_t*>(&v);
-        }
+      for (int ch = 0; ch < 4; ++ch) {
+        const int c0 = half * 128 + ch * 32;
+        const int n0 = nb * G_BN + c0;
         if (row < M) {
-          uint4* dst = reinterpret_cast<uint4*>(yrow + n0);
-          dst[0] = make_uint4(out[0], out[1], out[2], out[3]);
-          dst[1] = make_uint4(out[4], out[5], out[6], out[7]);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {      // 8 columns = one 16-byte store
+            if (n0 + 8 * v < N) {
+              uint32_t out[4];
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const int c = 8 * v + 2 * j;
+                const float y0 = fmaf(alpha, __uint_as_float(acc[ch][c]), bt[c0 + c]);
+                const float y1 = fmaf(alpha, __uint_as_float(acc[ch][c + 1]), bt[c0 + c + 1]);
+                out[j] = pack_bf16x2(y0, y1);
+              }
+              *reinterpret_cast<uint4*>(yrow + n0 + 8 * v) = make_uint4(out[0], out[1], out[2], out[3]);
+            }
+          }
         }
       }
-      tc_fence_before();
-      mbar_arrive(acc_empty);
     }
   }
 
