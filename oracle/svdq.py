@@ -298,12 +298,16 @@ def lowrank_down(x_hat: np.ndarray, L1: np.ndarray) -> np.ndarray:
 
 def linear_reference(X_bf16: np.ndarray, p: OraclePack,
                      bias_bf16: Optional[np.ndarray] = None,
-                     rows: Optional[np.ndarray] = None):
+                     rows: Optional[np.ndarray] = None,
+                     deq_w: Optional[np.ndarray] = None):
     """Reading R6: the float64 reference output Y_ref [M, N] (or only the
-    listed rows).  Returns (Y_ref, codes_x, sf_x, xl1)."""
+    listed rows).  `deq_w` may pass nvfp4_dequantize(p.codes_w, p.sf_w)
+    computed once for many calls.  Returns (Y_ref, codes_x, sf_x, xl1)."""
     X = X_bf16 if rows is None else X_bf16[rows]
     xh, cx, sfx = quantize_activation(X, p.s, p.A_x)
-    D = nvfp4_dequantize(cx, sfx) @ nvfp4_dequantize(p.codes_w, p.sf_w).T
+    if deq_w is None:
+        deq_w = nvfp4_dequantize(p.codes_w, p.sf_w)
+    D = nvfp4_dequantize(cx, sfx) @ deq_w.T
     Y = D / (np.float64(p.g_x) * np.float64(p.g_w))
     xl1 = lowrank_down(xh, p.L1)
     if p.L1.shape[1]:

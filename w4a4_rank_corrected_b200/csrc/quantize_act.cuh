@@ -13,14 +13,16 @@
 //   * warp 0 streams X chunks [64 x 64] bf16, the matching chunk of the
 //     low-rank operand and 64 smoothing factors into a deep shared-memory
 //     ring with TMA (128-byte swizzle);
-//   * warps 2..9 (256 threads) quantize: thread t owns row t/4, 16-group t%4
-//     of every chunk.  It multiplies by the smoothing factors, takes the group
-//     maximum in registers, forms the E4M3 block scale with one multiply and
-//     the hardware conversion, looks up g/scale in a 127-entry table (the
-//     IEEE quotients, computed once per CTA), forms the E2M1 codes with the
-//     hardware conversion and stores 8 code bytes; the four scale bytes of a
-//     row are gathered with shuffles into one 32-bit store in the MMA tile
-//     layout;
+//   * W quantize warps (W = number of ring stages, up to 8): warp w owns ring
+//     stage w and processes every chunk that lands there, whole.  Lane l
+//     handles rows l and l + 32 (all four 16-groups), so the warps work on
+//     different chunks at the same time instead of in lockstep and each lane
+//     has 8 independent groups in flight.  Per group: multiply by the
+//     smoothing factors, take the maximum in registers, form the E4M3 block
+//     scale with one multiply and the hardware conversion, look up g/scale in
+//     a 127-entry table (the IEEE quotients, computed once per CTA), form the
+//     E2M1 codes with the hardware conversion; per row: 32 code bytes and one
+//     32-bit word of scales straight into the MMA tile layout;
 //   * warp 1 issues tcgen05 bf16 MMAs (M = 64) on the SAME shared-memory X
 //     tile: X [64 x 64] times L1' [2r x 64]^T into a 64 x 2r fp32 accumulator
 //     in tensor memory.  L1' holds smooth * L1 split into bf16 hi and lo
@@ -37,7 +39,7 @@ namespace svdq_dev {
 
 constexpr int QA_BM = 64;
 constexpr int QA_MAX_STAGES = 8;
-constexpr int QA_QWARPS = 8;
+constexpr int QA_QWARPS = QA_MAX_STAGES;                 // one per ring stage (at most)
 constexpr int QA_THREADS = 32 * (2 + QA_QWARPS);
 constexpr uint32_t QA_X_BYTES = QA_BM * 128;  // 64 rows x 64 bf16
 constexpr uint32_t QA_RING_BUDGET = 180 * 1024;
@@ -137,7 +139,7 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < ST; ++i) {
       mbar_init(full0 + 8 * i, 1);
-      mbar_init(empty0 + 8 * i, QA_QWARPS + (has_lr ? 1 : 0));
+      mbar_init(empty0 + 8 * i, 1 + (has_lr ? 1 : 0));
     }
     mbar_init(acc_full, 1);
     mbar_init(drain_bar, 1);
@@ -171,9 +173,9 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
     // ---------------------------------------------------- TMA producer ----
     if (lane == 0) {
       const uint32_t tx = QA_X_BYTES + (has_lr ? 256u * r : 0u) + 256u;
+      int st = 0;
+      uint32_t ph = 0;
       for (int i = 0; i < nchunks; ++i) {
-        const int st = i % ST;
-        const uint32_t ph = (i / ST) & 1;
         if (!mbar_wait(empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) break;
         const uint32_t sb = smem_u32(smem + st * SB);
         const int c = c_begin + i;
@@ -182,15 +184,16 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
         if (has_lr) tma_load_2d(sb + QA_X_BYTES, &tm_l1, c * 64, 0, full0 + 8 * st);
         bulk_load(sb + QA_X_BYTES + 256u * r, p.smooth + c * 64, 256, full0 + 8 * st);
         issued = i + 1;
+        if (++st == ST) { st = 0; ph ^= 1; }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------- down-projection ----
     if (has_lr && lane == 0) {
       const uint32_t idesc = idesc_bf16(QA_BM, 2 * r);
+      int st = 0;
+      uint32_t ph = 0;
       for (int i = 0; i < nchunks; ++i) {
-        const int st = i % ST;
-        const uint32_t ph = (i / ST) & 1;
         if (!mbar_wait(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
         tc_fence_after();
         const uint32_t sb = smem_u32(smem + st * SB);
@@ -198,63 +201,79 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
         for (int kk = 0; kk < 4; ++kk)  // K = 16 bf16 = 32 bytes per MMA
           mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
         tc_commit(empty0 + 8 * st);
+        if (++st == ST) { st = 0; ph ^= 1; }
       }
       tc_commit(acc_full);
     }
   } else {
     // ---------------------------------------------- NVFP4 quantization ----
-    const int t = threadIdx.x - 64;
-    const int row_t = t >> 2;          // 0..63
-    const int grp = t & 3;             // 16-group within the 64-wide chunk
-    const int row = rb * QA_BM + row_t;
+    // warp qw owns ring stage qw: chunks qw, qw + ST, qw + 2 ST, ...
+    const int qw = warp - 2;
     const float gs = p.gs_x;
-    for (int i = 0; i < nchunks; ++i) {
-      const int st = i % ST;
-      const uint32_t ph = (i / ST) & 1;
-      if (!mbar_wait_warp(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) break;
-      const uint8_t* sb = smem + st * SB;
-      const int c = c_begin + i;
-      uint4 xw[2];
+    if (qw < ST) {
+      const uint32_t sb = smem_u32(smem + qw * SB);
+      const uint8_t* sbp = smem + qw * SB;
+      uint32_t ph = 0;
+      for (int i = qw; i < nchunks; i += ST, ph ^= 1) {
+        if (!mbar_wait_warp(full0 + 8 * qw, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) break;
+        const int c = c_begin + i;
+        const float4* sp = reinterpret_cast<const float4*>(sbp + QA_X_BYTES + 256u * r);
 #pragma unroll
-      for (int jj = 0; jj < 2; ++jj) {
-        const int phys = (2 * grp + jj) ^ (row_t & 7);  // 128-byte swizzle
-        xw[jj] = *reinterpret_cast<const uint4*>(sb + row_t * 128 + phys * 16);
+        for (int hr = 0; hr < 2; ++hr) {
+          const int row_t = lane + 32 * hr;
+          const int row = rb * QA_BM + row_t;
+          uint32_t cw[8];
+          uint32_t sfw = 0;
+#pragma unroll
+          for (int g = 0; g < 4; ++g) {
+            const uint4 x0 = *reinterpret_cast<const uint4*>(sbp + row_t * 128 + (((2 * g) ^ (row_t & 7)) << 4));
+            const uint4 x1 = *reinterpret_cast<const uint4*>(sbp + row_t * 128 + (((2 * g + 1) ^ (row_t & 7)) << 4));
+            const float4 s0 = sp[4 * g], s1 = sp[4 * g + 1], s2 = sp[4 * g + 2], s3 = sp[4 * g + 3];
+            float v[16];
+            v[0] = __fmul_rn(bf16_lo_f32(x0.x), s0.x);
+            v[1] = __fmul_rn(bf16_hi_f32(x0.x), s0.y);
+            v[2] = __fmul_rn(bf16_lo_f32(x0.y), s0.z);
+            v[3] = __fmul_rn(bf16_hi_f32(x0.y), s0.w);
+            v[4] = __fmul_rn(bf16_lo_f32(x0.z), s1.x);
+            v[5] = __fmul_rn(bf16_hi_f32(x0.z), s1.y);
+            v[6] = __fmul_rn(bf16_lo_f32(x0.w), s1.z);
+            v[7] = __fmul_rn(bf16_hi_f32(x0.w), s1.w);
+            v[8] = __fmul_rn(bf16_lo_f32(x1.x), s2.x);
+            v[9] = __fmul_rn(bf16_hi_f32(x1.x), s2.y);
+            v[10] = __fmul_rn(bf16_lo_f32(x1.y), s2.z);
+            v[11] = __fmul_rn(bf16_hi_f32(x1.y), s2.w);
+            v[12] = __fmul_rn(bf16_lo_f32(x1.z), s3.x);
+            v[13] = __fmul_rn(bf16_hi_f32(x1.z), s3.y);
+            v[14] = __fmul_rn(bf16_lo_f32(x1.w), s3.z);
+            v[15] = __fmul_rn(bf16_hi_f32(x1.w), s3.w);
+            float m0 = fmaxf(fabsf(v[0]), fabsf(v[1])), m1 = fmaxf(fabsf(v[2]), fabsf(v[3]));
+            float m2 = fmaxf(fabsf(v[4]), fabsf(v[5])), m3 = fmaxf(fabsf(v[6]), fabsf(v[7]));
+            float m4 = fmaxf(fabsf(v[8]), fabsf(v[9])), m5 = fmaxf(fabsf(v[10]), fabsf(v[11]));
+            float m6 = fmaxf(fabsf(v[12]), fabsf(v[13])), m7 = fmaxf(fabsf(v[14]), fabsf(v[15]));
+            const float a = fmaxf(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), fmaxf(fmaxf(m4, m5), fmaxf(m6, m7)));
+            const uint32_t code = cvt_e4m3x2(__fmul_rn(a, gs), 0.0f) & 0xFF;
+            const float q = qlut[code];
+            float t0[8], t1[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              t0[e] = __fmul_rn(v[e], q);
+              t1[e] = __fmul_rn(v[8 + e], q);
+            }
+            cw[2 * g] = cvt_e2m1x8(t0);
+            cw[2 * g + 1] = cvt_e2m1x8(t1);
+            sfw |= code << (8 * g);
+          }
+          if (row < p.M) {
+            uint4* dst = reinterpret_cast<uint4*>(p.codes_x + (size_t)row * (p.K >> 1) + (size_t)c * 32);
+            dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+            dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+          }
+          *reinterpret_cast<uint32_t*>(p.sf_x + sf_tile_off(row, 4 * c, p.K)) = sfw;
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * qw);
       }
-      const float4* sp = reinterpret_cast<const float4*>(sb + QA_X_BYTES + 256u * r) + 4 * grp;
-      const uint32_t w[8] = {xw[0].x, xw[0].y, xw[0].z, xw[0].w, xw[1].x, xw[1].y, xw[1].z, xw[1].w};
-      float v[16];
-      float a = 0.0f;
-#pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        const float4 s4 = sp[q4];
-        v[4 * q4 + 0] = __fmul_rn(bf16_lo_f32(w[2 * q4]), s4.x);
-        v[4 * q4 + 1] = __fmul_rn(bf16_hi_f32(w[2 * q4]), s4.y);
-        v[4 * q4 + 2] = __fmul_rn(bf16_lo_f32(w[2 * q4 + 1]), s4.z);
-        v[4 * q4 + 3] = __fmul_rn(bf16_hi_f32(w[2 * q4 + 1]), s4.w);
-      }
-#pragma unroll
-      for (int e = 0; e < 16; ++e) a = fmaxf(a, fabsf(v[e]));
-      const uint32_t code = cvt_e4m3x2(__fmul_rn(a, gs), 0.0f) & 0xFF;
-      const float q = qlut[code];
-      float t0[8], t1[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        t0[e] = __fmul_rn(v[e], q);
-        t1[e] = __fmul_rn(v[8 + e], q);
-      }
-      const uint32_t c0 = cvt_e2m1x8(t0), c1 = cvt_e2m1x8(t1);
-      // the four scale bytes of this row: lanes 4i..4i+3 hold groups 0..3
-      const uint32_t b1 = __shfl_down_sync(0xffffffff, code, 1);
-      const uint32_t b2 = __shfl_down_sync(0xffffffff, code, 2);
-      const uint32_t b3 = __shfl_down_sync(0xffffffff, code, 3);
-      if (row < p.M)
-        *reinterpret_cast<uint2*>(p.codes_x + (size_t)row * (p.K >> 1) + c * 32 + grp * 8) =
-            make_uint2(c0, c1);
-      if (grp == 0)
-        *reinterpret_cast<uint32_t*>(p.sf_x + sf_tile_off(row, 4 * c, p.K)) =
-            code | (b1 << 8) | (b2 << 16) | (b3 << 24);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8 * st);
+      (void)sb;
     }
 
     // ----------------------------------------- low-rank epilogue (X L1) ----
@@ -264,7 +283,7 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
       // M = 64 accumulator: row m sits in lane (m % 16) + 32 (m / 16).  Warp w
       // reads its lane quarter w % 4; lanes 0..15 hold rows 16 (w % 4) + lane.
       const int quad = warp & 3;
-      const int hc = (warp - 2) >> 2;
+      const int hc = (warp - 2) >> 2;          // 0..1: which chunks of 16 columns
       const int lrow_t = quad * 16 + lane;
       const int lrow = rb * QA_BM + lrow_t;
       const bool own = lane < 16;
@@ -273,7 +292,7 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
       const int pstride = r + 1;
       // every quantize warp is done reading the ring before it is reused
       asm volatile("bar.sync 1, %0;" ::"n"(32 * QA_QWARPS) : "memory");
-      for (int ci = hc; ci < r / 16; ci += 2) {
+      for (int ci = hc; ci < r / 16; ci += QA_QWARPS / 4) {  // QA_QWARPS / 4 warps per quarter
         uint32_t hi[16], lo[16];
         const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16);
         if (ok) {

@@ -64,6 +64,7 @@ struct DeviceInfo {
   // max co-resident clusters of the activation kernel, per rank r/16 (0..8)
   // and cluster size S (1..8); -1 = not queried yet
   int max_clusters[9][9];
+  int gemm_pairs = -1;  // max co-resident CTA pairs of the GEMM kernel
   DeviceInfo() {
     for (auto& a : max_clusters)
       for (int& v : a) v = -1;
@@ -120,15 +121,18 @@ svdq_status device_check(int* sms) {
   return SVDQ_OK;
 }
 
-// 2D tensor map over a row-major [rows][inner] matrix, 128-byte swizzle.
+// 2D tensor map over a row-major [rows][inner] matrix (128-byte swizzle
+// unless `swizzle` is false).
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
-              uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows) {
+              uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+              bool swizzle = true) {
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -261,28 +265,58 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
   return SVDQ_OK;
 }
 
+int gemm_max_pairs(int sms) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int& cached = g_dev[dev].gemm_pairs;
+  if (cached < 0) {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof(cfg));
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(G_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = gemm_smem_bytes();
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, w4a4_gemm_kernel, &cfg) != cudaSuccess || n <= 0) {
+      cudaGetLastError();
+      n = sms / 2;
+    }
+    cached = std::min(n, sms / 2);
+  }
+  return std::max(1, cached);
+}
+
 svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint8_t* sf_x,
                         const uint16_t* xl1, int M, uint16_t* Y, int64_t ldy, cudaStream_t s,
                         int sms) {
   const int N = w->N, K = w->K, r = w->r, klr = klr_of(r);
-  CUtensorMap ta, tb, talr, tblr;
+  CUtensorMap ta, tb, tsa, tsb, talr, tblr;
   std::memset(&talr, 0, sizeof(talr));
   std::memset(&tblr, 0, sizeof(tblr));
+  // scale buffers as rows of 256 bytes (half a 512-byte atom), unswizzled
+  const uint64_t sfa_rows = rup((size_t)M, 128) * (K / 16) / 256;
+  const uint64_t sfb_rows = rup((size_t)N, 256) * (K / 16) / 256;
   if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_x, (uint64_t)K / 2, (uint64_t)M,
                 (uint64_t)K / 2, 128, G_BM) ||
       !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes_w, (uint64_t)K / 2, (uint64_t)N,
-                (uint64_t)K / 2, 128, G_BN))
+                (uint64_t)K / 2, 128, G_BN_CTA) ||
+      !make_map(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT8, sf_x, 256, sfa_rows, 256, 256, 8, false) ||
+      !make_map(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->sf_w, 256, sfb_rows, 256, 256, 8, false))
     return SVDQ_ERR_CUDA;
   if (r > 0) {
     if (!make_map(&talr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xl1, (uint64_t)klr, (uint64_t)M,
                   (uint64_t)klr * 2, 64, G_BM) ||
         !make_map(&tblr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l2_mma, (uint64_t)klr, (uint64_t)N,
-                  (uint64_t)klr * 2, 64, G_BN))
+                  (uint64_t)klr * 2, 64, G_BN_CTA))
       return SVDQ_ERR_CUDA;
   }
   GemmParams p;
-  p.sf_x = sf_x;
-  p.sf_w = w->sf_w;
   p.bias = w->bias;
   p.Y = Y;
   p.ldy = ldy;
@@ -293,19 +327,23 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   p.klr = klr;
   p.alpha = w->alpha;
   p.timeout_ns = kDefaultTimeoutNs;
-  const int tiles = ((M + G_BM - 1) / G_BM) * ((N + G_BN - 1) / G_BN);
-  const int grid = std::max(1, std::min(tiles, sms));
+  const int tiles = ((M + 2 * G_BM - 1) / (2 * G_BM)) * ((N + G_BN - 1) / G_BN);
+  const int pairs = std::max(1, std::min(tiles, gemm_max_pairs(sms)));
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
-  cfg.gridDim = dim3((unsigned)grid, 1, 1);
+  cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
   cfg.blockDim = dim3(G_THREADS, 1, 1);
   cfg.dynamicSmemBytes = gemm_smem_bytes();
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0] = pdl_attr();
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = 2;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, w4a4_gemm_kernel, ta, tb, talr, tblr, p) != cudaSuccess) {
+  cfg.numAttrs = 2;
+  if (cudaLaunchKernelEx(&cfg, w4a4_gemm_kernel, ta, tb, tsa, tsb, talr, tblr, p) != cudaSuccess) {
     cudaGetLastError();
     return SVDQ_ERR_CUDA;
   }

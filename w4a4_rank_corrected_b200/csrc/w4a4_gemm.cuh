@@ -6,50 +6,57 @@
 // (section "SVDQuant and the Nunchaku engine"): the low-rank up projection is
 // merged into the 4-bit compute kernel.  The B200 design:
 //
-//   * persistent CTAs (one per SM) walk 128 x 256 output tiles;
-//   * warp 0 (one lane) streams, per 256-wide K step, the E2M1 code tiles of
-//     X [128 x 128 B] and of R [256 x 128 B] with TMA (128-byte swizzle) and
-//     the matching E4M3 scale atoms (512 B each, already in the MMA layout)
-//     with bulk copies, into a 4-deep shared-memory ring;
-//   * warp 1 (one lane) copies the scale atoms into tensor memory
-//     (tcgen05.cp, 32x128b x4) and issues tcgen05.mma kind::mxf4nvf4 with
-//     block16 UE4M3 scales, K = 64 per instruction, into a 128 x 256 fp32
-//     accumulator in tensor memory; after the K loop it streams the low-rank
-//     operands (xl1 hi|lo [128 x 2r] and L2 [256 x 2r], bf16) through the
-//     same ring and accumulates xl1 . L2 into the SAME accumulator with
-//     kind::f16 MMAs (xl1 was pre-multiplied by g_x g_w = 1/alpha);
-//   * warps 2..9 (two per tensor-memory lane quarter, 128 columns each)
-//     drain the accumulator with four 32-column tcgen05.ld and ONE wait,
-//     release it to the MMA warp at once, and only then compute
-//     Y = bf16(alpha * acc + bias) (bias staged per tile in shared memory)
-//     and store, overlapping the next tile's main loop.
+//   * CTA pairs (thread-block clusters of 2) share one tensor-core MMA
+//     (tcgen05 cta_group::2): a pair computes a 256 x 256 output tile, each
+//     CTA holds its 128 rows of the activation codes and half (128 rows) of
+//     the weight codes in its own shared memory and its 128 rows of the fp32
+//     accumulator in its own tensor memory.  Per unit of MMA work each SM
+//     moves half the weight bytes through shared memory that a single-SM
+//     128 x 256 tile would, which is what keeps the tensor core fed;
+//   * warp 0 of each CTA streams, per 256-deep K step, its A and B code tiles
+//     (TMA, 128-byte swizzle) and the scale atoms (TMA; its own 128 rows of
+//     activation scales, all 256 rows of weight scales) into a 5-deep ring;
+//     every load is counted on the leader CTA's barrier (cta_group::2 form,
+//     no multicast);
+//   * warp 1 of the leader copies the scale atoms into both CTAs' tensor
+//     memory (tcgen05.cp cta_group::2) and issues
+//     tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 (M = 256,
+//     N = 256, K = 64); after the K loop it streams the low-rank operands
+//     (xl1 hi|lo and L2, bf16) through the same ring into the SAME
+//     accumulator with kind::f16 MMAs (xl1 was pre-multiplied by
+//     g_x g_w = 1/alpha); completions are multicast to both CTAs;
+//   * warps 2..9 of each CTA drain its accumulator (four 32-column
+//     tcgen05.ld, one wait), release it to the leader, and only then compute
+//     Y = bf16(alpha * acc + bias) (bias staged per tile in shared memory) and
+//     store, overlapping the next tile's main loop.
 #pragma once
 #include "ptx.cuh"
 
 namespace svdq_dev {
 
-constexpr int G_STAGES = 4;
+constexpr int G_STAGES = 5;
 constexpr int G_EPI_WARPS = 8;
 constexpr int G_THREADS = 32 * (2 + G_EPI_WARPS);
-constexpr int G_BM = 128, G_BN = 256;
+constexpr int G_BM = 128;                    // rows per CTA (pair tile: 256)
+constexpr int G_BN = 256;                    // columns per pair tile (MMA N)
+constexpr int G_BN_CTA = 128;                // weight rows held per CTA
 constexpr uint32_t G_A_BYTES = 128 * 128;    // 128 rows x 128 B
-constexpr uint32_t G_B_BYTES = 256 * 128;    // 256 rows x 128 B
+constexpr uint32_t G_B_BYTES = 128 * 128;    // 128 rows x 128 B
 constexpr uint32_t G_SFA_BYTES = 4 * 512;    // 4 atoms (K = 256)
 constexpr uint32_t G_SFB_BYTES = 8 * 512;    // 2 row blocks x 4 atoms
 constexpr uint32_t G_STAGE_BYTES = G_A_BYTES + G_B_BYTES + G_SFA_BYTES + G_SFB_BYTES;
 constexpr uint32_t G_TMEM_COLS = 512;
 constexpr uint32_t G_SF_TMEM = 256;          // scale buffers after the accumulator
 constexpr uint32_t G_SF_TMEM_STRIDE = 48;    // 16 cols SFA + 32 cols SFB
-
 constexpr uint32_t G_BIAS_BYTES = 2 * G_BN * 4;   // two fp32 bias tiles
+constexpr uint32_t G_FP4_TX = 2 * G_STAGE_BYTES;  // bytes per FP4 stage, both CTAs
+constexpr uint32_t G_LR_TX = 2 * (G_A_BYTES + G_B_BYTES);
 
 __host__ __device__ inline uint32_t gemm_smem_bytes() {
   return 1024u + G_STAGES * G_STAGE_BYTES + G_BIAS_BYTES + 256u;  // + barriers
 }
 
 struct GemmParams {
-  const uint8_t* sf_x;
-  const uint8_t* sf_w;
   const uint16_t* bias;
   uint16_t* Y;
   long long ldy;
@@ -59,8 +66,9 @@ struct GemmParams {
 };
 
 __global__ void __launch_bounds__(G_THREADS, 1)
-    w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,
-                     const __grid_constant__ CUtensorMap tm_b,
+    w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                     const __grid_constant__ CUtensorMap tm_sfa,
+                     const __grid_constant__ CUtensorMap tm_sfb,
                      const __grid_constant__ CUtensorMap tm_alr,
                      const __grid_constant__ CUtensorMap tm_blr, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -78,11 +86,14 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const uint32_t warp = warp_id(), lane = lane_id();
+  const uint32_t rank = cluster_ctarank();      // 0 = leader of the pair
+  const bool leader = rank == 0;
   const int M = p.M, N = p.N, K = p.K, r = p.r;
   const bool has_lr = r > 0;
-  const int num_m = (M + G_BM - 1) / G_BM;
+  const int num_m = (M + 2 * G_BM - 1) / (2 * G_BM);
   const int num_n = (N + G_BN - 1) / G_BN;
   const int num_tiles = num_m * num_n;
+  const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
   const int k64 = K >> 6;
   const int kb_total = (k64 + 3) >> 2;
   const int lr_chunks = has_lr ? (p.klr >> 6) : 0;
@@ -94,7 +105,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       mbar_init(empty0 + 8 * i, 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 32 * G_EPI_WARPS);
+    mbar_init(acc_empty, 2 * G_EPI_WARPS);
     mbar_init(drain_bar, 1);
     mbar_init(bias_bar0, 32 * G_EPI_WARPS);
     mbar_init(bias_bar0 + 8, 32 * G_EPI_WARPS);
@@ -104,19 +115,24 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tm_a);
     prefetch_tensormap(&tm_b);
+    prefetch_tensormap(&tm_sfa);
+    prefetch_tensormap(&tm_sfb);
     if (has_lr) {
       prefetch_tensormap(&tm_alr);
       prefetch_tensormap(&tm_blr);
     }
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), G_TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_holder), G_TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
   __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const uint32_t lead_full0 = map_to_rank(full0, 0);
+  const uint32_t lead_acc_empty = map_to_rank(acc_empty, 0);
   // The prologue above overlaps the previous kernel; the activation codes,
   // scales and low-rank operand it produced are read only after this.
   grid_dependency_wait();
@@ -128,8 +144,11 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     if (lane == 0) {
       int it = 0;
       bool stop = false;
-      for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x) {
+      for (int tile = pair; tile < num_tiles && !stop; tile += num_pairs) {
         const int mb = tile % num_m, nb = tile / num_m;
+        const int row0 = mb * 2 * G_BM + (int)rank * G_BM;     // this CTA's A rows
+        const int brow0 = nb * G_BN + (int)rank * G_BN_CTA;    // this CTA's B rows
+        const int sfa_blk = mb * 2 + (int)rank;                // 128-row scale block
         for (int kb = 0; kb < kb_total; ++kb, ++it) {
           const int st = it % G_STAGES;
           const uint32_t ph = (it / G_STAGES) & 1;
@@ -137,17 +156,17 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             stop = true;
             break;
           }
-          const int nk = min(4, k64 - 4 * kb);
           const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
-          const uint32_t fb = full0 + 8 * st;
-          mbar_arrive_expect_tx(fb, G_A_BYTES + G_B_BYTES + 3u * 512u * nk);
-          tma_load_2d(sb, &tm_a, kb * 128, mb * G_BM, fb);
-          tma_load_2d(sb + G_A_BYTES, &tm_b, kb * 128, nb * G_BN, fb);
-          bulk_load(sb + G_A_BYTES + G_B_BYTES, p.sf_x + ((size_t)mb * k64 + 4 * kb) * 512,
-                    512u * nk, fb);
+          if (leader) mbar_arrive_expect_tx(full0 + 8 * st, G_FP4_TX);
+          const uint32_t fb = lead_full0 + 8 * st;
+          tma_load_2d_pair(sb, &tm_a, kb * 128, row0, fb);
+          tma_load_2d_pair(sb + G_A_BYTES, &tm_b, kb * 128, brow0, fb);
+          // scale atoms: rows of 256 bytes = half atoms; 4 atoms = 8 rows
+          tma_load_2d_pair(sb + G_A_BYTES + G_B_BYTES, &tm_sfa, 0,
+                           (sfa_blk * k64 + 4 * kb) * 2, fb);
           for (int hh = 0; hh < 2; ++hh)
-            bulk_load(sb + G_A_BYTES + G_B_BYTES + G_SFA_BYTES + hh * 2048,
-                      p.sf_w + ((size_t)(2 * nb + hh) * k64 + 4 * kb) * 512, 512u * nk, fb);
+            tma_load_2d_pair(sb + G_A_BYTES + G_B_BYTES + G_SFA_BYTES + hh * 2048, &tm_sfb, 0,
+                             ((2 * nb + hh) * k64 + 4 * kb) * 2, fb);
           issued = it + 1;
         }
         for (int c = 0; c < lr_chunks && !stop; ++c, ++it) {
@@ -158,22 +177,22 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             break;
           }
           const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
-          const uint32_t fb = full0 + 8 * st;
-          mbar_arrive_expect_tx(fb, G_A_BYTES + G_B_BYTES);
-          tma_load_2d(sb, &tm_alr, c * 64, mb * G_BM, fb);
-          tma_load_2d(sb + G_A_BYTES, &tm_blr, c * 64, nb * G_BN, fb);
+          if (leader) mbar_arrive_expect_tx(full0 + 8 * st, G_LR_TX);
+          const uint32_t fb = lead_full0 + 8 * st;
+          tma_load_2d_pair(sb, &tm_alr, c * 64, row0, fb);
+          tma_load_2d_pair(sb + G_A_BYTES, &tm_blr, c * 64, brow0, fb);
           issued = it + 1;
         }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------ MMA issuer ----
-    if (lane == 0) {
-      const uint32_t id_fp4 = idesc_nvfp4(G_BM, G_BN);
-      const uint32_t id_lr = idesc_bf16(G_BM, G_BN);
+    // ------------------------------------------- MMA issuer (leader only) ----
+    if (leader && lane == 0) {
+      const uint32_t id_fp4 = idesc_nvfp4(2 * G_BM, G_BN);
+      const uint32_t id_lr = idesc_bf16(2 * G_BM, G_BN);
       int it = 0, tcount = 0;
       bool stop = false;
-      for (int tile = blockIdx.x; tile < num_tiles && !stop; tile += gridDim.x, ++tcount) {
+      for (int tile = pair; tile < num_tiles && !stop; tile += num_pairs, ++tcount) {
         if (!mbar_wait(acc_empty, (tcount & 1) ^ 1, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
         tc_fence_after();
         uint32_t accumulate = 0;
@@ -192,17 +211,17 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           const uint32_t sfa_t = tmem + G_SF_TMEM + (it & 1) * G_SF_TMEM_STRIDE;
           const uint32_t sfb_t = sfa_t + 16;
           for (int kk = 0; kk < nk; ++kk) {
-            tmem_copy_32x128b_x4(sfa_t + 4 * kk, sdesc_sf_block(sfa_s + 512 * kk));
-            tmem_copy_32x128b_x4(sfb_t + 8 * kk, sdesc_sf_block(sfb_s + 512 * kk));
-            tmem_copy_32x128b_x4(sfb_t + 8 * kk + 4, sdesc_sf_block(sfb_s + 2048 + 512 * kk));
+            tmem_copy_32x128b_x4_pair(sfa_t + 4 * kk, sdesc_sf_block(sfa_s + 512 * kk));
+            tmem_copy_32x128b_x4_pair(sfb_t + 8 * kk, sdesc_sf_block(sfb_s + 512 * kk));
+            tmem_copy_32x128b_x4_pair(sfb_t + 8 * kk + 4, sdesc_sf_block(sfb_s + 2048 + 512 * kk));
           }
           const uint64_t da = sdesc_sw128(sb), db = sdesc_sw128(sb + G_A_BYTES);
           for (int kk = 0; kk < nk; ++kk) {  // K = 64 E2M1 = 32 bytes per MMA
-            mma_nvfp4(tmem, da + 2 * kk, db + 2 * kk, id_fp4, sfa_t + 4 * kk, sfb_t + 8 * kk,
-                      accumulate);
+            mma_nvfp4_pair(tmem, da + 2 * kk, db + 2 * kk, id_fp4, sfa_t + 4 * kk,
+                           sfb_t + 8 * kk, accumulate);
             accumulate = 1;
           }
-          tc_commit(empty0 + 8 * st);
+          tc_commit_pair(empty0 + 8 * st, 0x3);
         }
         for (int c = 0; c < lr_chunks && !stop; ++c, ++it) {
           const int st = it % G_STAGES;
@@ -216,12 +235,12 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           const uint64_t da = sdesc_sw128(sb), db = sdesc_sw128(sb + G_A_BYTES);
           const int nks = min(4, (2 * r - 64 * c) >> 4);  // K = 16 bf16 per MMA
           for (int kk = 0; kk < nks; ++kk) {
-            mma_bf16(tmem, da + 2 * kk, db + 2 * kk, id_lr, accumulate);
+            mma_bf16_pair(tmem, da + 2 * kk, db + 2 * kk, id_lr, accumulate);
             accumulate = 1;
           }
-          tc_commit(empty0 + 8 * st);
+          tc_commit_pair(empty0 + 8 * st, 0x3);
         }
-        tc_commit(acc_full);
+        tc_commit_pair(acc_full, 0x3);
       }
     }
   } else {
@@ -231,7 +250,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int et = threadIdx.x - 64;           // 0..255
     const float alpha = p.alpha;
     int tcount = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tcount) {
+    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++tcount) {
       const int mb = tile % num_m, nb = tile / num_m;
       // stage this tile's bias (fp32) while the main loop runs.  Buffer
       // tcount&1 was last read for tile tcount-2, which every thread had
@@ -254,8 +273,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       tmem_ld32(tbase + 96, acc[3]);
       tmem_wait_ld();
       tc_fence_before();
-      mbar_arrive(acc_empty);                  // the accumulator is free again
-      const int row = mb * G_BM + quad * 32 + lane;
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(lead_acc_empty);   // accumulator free again
+      const int row = mb * 2 * G_BM + (int)rank * G_BM + quad * 32 + lane;
       uint16_t* yrow = p.Y + (size_t)row * p.ldy;
 #pragma unroll
       for (int ch = 0; ch < 4; ++ch) {
@@ -285,19 +305,29 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   if (*abort_flag) {
-    if (warp == 0 && lane == 0) {
+    // the leader's barriers count both CTAs' loads: drain those, then the
+    // tensor-core work in flight
+    if (leader && warp == 0 && lane == 0) {
       for (int i = max(0, issued - G_STAGES); i < issued; ++i)
         mbar_wait_drain(full0 + 8 * (i % G_STAGES), (i / G_STAGES) & 1, p.timeout_ns);
     }
-    if (warp == 1 && lane == 0) {
-      tc_commit(drain_bar);
+    if (leader && warp == 1 && lane == 0) {
+      tc_commit_pair(drain_bar, 0x1);
       mbar_wait_drain(drain_bar, 0, p.timeout_ns);
+    }
+    // the other CTA's loads complete on the leader's barriers; give any that
+    // are still landing in this CTA's shared memory a bounded moment
+    if (threadIdx.x == 0) {
+      const uint64_t t0 = globaltimer_ns();
+      while (globaltimer_ns() - t0 < 100000) {
+      }
     }
     __syncthreads();
   }
+  cluster_sync();  // the pair is done with shared and tensor memory
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, G_TMEM_COLS);
+    tmem_dealloc_pair(tmem, G_TMEM_COLS);
   }
 }
 
