@@ -15,9 +15,11 @@
 //     ring with TMA (128-byte swizzle);
 //   * W quantize warps (W = number of ring stages, up to 8): warp w owns ring
 //     stage w and processes every chunk that lands there, whole.  Lane l
-//     handles rows l and l + 32 (all four 16-groups), so the warps work on
-//     different chunks at the same time instead of in lockstep and each lane
-//     has 8 independent groups in flight.  Per group: multiply by the
+//     handles rows l and l + 32 (all four 16-groups): it copies its rows and
+//     the chunk's smoothing factors into registers and hands the stage back
+//     before quantizing, so the next chunk for that stage is already loading
+//     while this one is processed; the warps work on different chunks at the
+//     same time instead of in lockstep.  Per group: multiply by the
 //     smoothing factors, take the maximum in registers, form the E4M3 block
 //     scale with one multiply and the hardware conversion, look up g/scale in
 //     a 127-entry table (the IEEE quotients, computed once per CTA), form the
@@ -217,7 +219,25 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
       for (int i = qw; i < nchunks; i += ST, ph ^= 1) {
         if (!mbar_wait_warp(full0 + 8 * qw, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) break;
         const int c = c_begin + i;
-        const float4* sp = reinterpret_cast<const float4*>(sbp + QA_X_BYTES + 256u * r);
+        // copy this lane's two rows and the chunk's smoothing factors into
+        // registers, then hand the stage back so the next chunk can land
+        // while this one is quantized
+        uint4 xr[2][8];
+        float4 sv[16];
+#pragma unroll
+        for (int hr = 0; hr < 2; ++hr) {
+          const int row_t = lane + 32 * hr;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            xr[hr][j] = *reinterpret_cast<const uint4*>(sbp + row_t * 128 + ((j ^ (row_t & 7)) << 4));
+        }
+        {
+          const float4* sp = reinterpret_cast<const float4*>(sbp + QA_X_BYTES + 256u * r);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) sv[j] = sp[j];
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * qw);
 #pragma unroll
         for (int hr = 0; hr < 2; ++hr) {
           const int row_t = lane + 32 * hr;
@@ -226,9 +246,8 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
           uint32_t sfw = 0;
 #pragma unroll
           for (int g = 0; g < 4; ++g) {
-            const uint4 x0 = *reinterpret_cast<const uint4*>(sbp + row_t * 128 + (((2 * g) ^ (row_t & 7)) << 4));
-            const uint4 x1 = *reinterpret_cast<const uint4*>(sbp + row_t * 128 + (((2 * g + 1) ^ (row_t & 7)) << 4));
-            const float4 s0 = sp[4 * g], s1 = sp[4 * g + 1], s2 = sp[4 * g + 2], s3 = sp[4 * g + 3];
+            const uint4 x0 = xr[hr][2 * g], x1 = xr[hr][2 * g + 1];
+            const float4 s0 = sv[4 * g], s1 = sv[4 * g + 1], s2 = sv[4 * g + 2], s3 = sv[4 * g + 3];
             float v[16];
             v[0] = __fmul_rn(bf16_lo_f32(x0.x), s0.x);
             v[1] = __fmul_rn(bf16_hi_f32(x0.x), s0.y);
@@ -270,8 +289,6 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
           }
           *reinterpret_cast<uint32_t*>(p.sf_x + sf_tile_off(row, 4 * c, p.K)) = sfw;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + 8 * qw);
       }
       (void)sb;
     }
