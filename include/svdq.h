@@ -194,6 +194,31 @@ svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t* X,
                                 void* workspace, size_t ws_bytes,
                                 void* stream);
 
+/* svdq_linear_forward_static: the same forward as svdq_linear_forward, with
+ * the intermediates in a fixed scratch area that the library holds in device
+ * memory (SVDQ_STATIC_WORKSPACE_BYTES per device, reserved when the library's
+ * module loads).  The paper has no counterpart: it is a convenience for
+ * callers that cannot allocate device memory while a forward runs, such as a
+ * plain C host with no device allocator of its own, or a runtime that plans
+ * all memory ahead and forbids allocation inside its step.
+ *   - Never allocates or frees device memory and calls no allocating library
+ *     routine.  The first call on each device looks the scratch address up
+ *     once (cudaGetSymbolAddress) and caches it; make that first call before
+ *     any stream capture.
+ *   - M is limited by the scratch size: svdq_act_workspace_bytes(M, K, r)
+ *     must be <= SVDQ_STATIC_WORKSPACE_BYTES, else SVDQ_ERR_WORKSPACE and
+ *     nothing is launched (e.g. K = 3072, r = 32 allows M <= 9033).
+ *   - Nothing in the scratch needs to start at zero: the activation kernel
+ *     writes every byte the GEMM reads, padding rows included.
+ *   - One scratch area per device: calls that overlap in time (different
+ *     streams, or threads without ordering) race on it.  Calls in order on
+ *     one stream are safe.
+ * Arguments, layouts and the other errors are those of svdq_linear_forward. */
+#define SVDQ_STATIC_WORKSPACE_BYTES ((size_t)16 << 20)
+svdq_status svdq_linear_forward_static(const svdq_weight* w, const uint16_t* X,
+                                       int M, int64_t ldx, uint16_t* Y,
+                                       int64_t ldy, void* stream);
+
 /* ------------------------------------------------------------- failure --
  * Every wait inside the kernels is bounded (about one second).  A kernel
  * that gives up records a code in a device-side word and exits cleanly

@@ -86,6 +86,7 @@ def _load() -> ctypes.CDLL:
         "svdq_quantize_act": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P, P, P]),
         "svdq_gemm": (I, [ctypes.POINTER(SvdqWeight), P, P, P, I, P, I64, P]),
         "svdq_linear_forward": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P, SZ, P]),
+        "svdq_linear_forward_static": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P]),
         "svdq_device_error": (I, [P, ctypes.POINTER(I)]),
         "svdq_selftest_timeout": (I, [I, P]),
         "svdq_debug_convert": (I, [P, P, P, I64, P]),
@@ -288,6 +289,25 @@ def svdq_linear_forward(w: DeviceWeight, X, Y=None, workspace=None, stream=None)
                                    Y.data_ptr(), Y.stride(0), workspace.data_ptr(),
                                    workspace.numel(), _stream_ptr(stream)),
            "svdq_linear_forward")
+    return Y
+
+
+SVDQ_STATIC_WORKSPACE_BYTES = 16 << 20
+
+
+def svdq_linear_forward_static(w: DeviceWeight, X, Y=None, stream=None):
+    """The forward with the library's own fixed device scratch: the C call
+    allocates nothing (Y is allocated here only when not given).  M is
+    limited to svdq_act_workspace_bytes(M, K, r) <= SVDQ_STATIC_WORKSPACE_BYTES;
+    calls that overlap in time on one device share the scratch and race."""
+    import torch
+    _check_x(X, w.K)
+    M = X.shape[0]
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+    _check(lib.svdq_linear_forward_static(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
+                                          Y.data_ptr(), Y.stride(0), _stream_ptr(stream)),
+           "svdq_linear_forward_static")
     return Y
 
 

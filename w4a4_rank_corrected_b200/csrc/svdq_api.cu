@@ -431,6 +431,53 @@ extern "C" svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t*
   return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, s, sms);
 }
 
+// Scratch of svdq_linear_forward_static: one per device, module-resident, so
+// that the call itself never allocates.  Calls that overlap in time (two
+// streams, two host threads) share it and race.
+__device__ __align__(256) unsigned char g_static_ws[SVDQ_STATIC_WORKSPACE_BYTES];
+
+namespace {
+void* g_static_ws_addr[kMaxDevices];
+
+// Device address of g_static_ws for the current device, looked up once per
+// device (cudaGetSymbolAddress) and cached.
+svdq_status static_ws_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return SVDQ_ERR_UNSUPPORTED_ARCH;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_static_ws_addr[dev]) {
+    void* a = nullptr;
+    if (cudaGetSymbolAddress(&a, g_static_ws) != cudaSuccess || !a) {
+      cudaGetLastError();
+      return SVDQ_ERR_CUDA;
+    }
+    g_static_ws_addr[dev] = a;
+  }
+  *out = g_static_ws_addr[dev];
+  return SVDQ_OK;
+}
+}  // namespace
+
+extern "C" svdq_status svdq_linear_forward_static(const svdq_weight* w, const uint16_t* X,
+                                                  int M, int64_t ldx, uint16_t* Y, int64_t ldy,
+                                                  void* stream) {
+  svdq_status st = check_weight(w);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || ldx < w->K || ldy < w->N) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !Y) return SVDQ_ERR_INVALID_ARG;
+  const size_t need = svdq_act_workspace_bytes(M, w->K, w->r);
+  if (need == 0 || need > SVDQ_STATIC_WORKSPACE_BYTES) return SVDQ_ERR_WORKSPACE;
+  if (!aligned16(X) || !aligned16(Y) || ldx % 8 || ldy % 8) return SVDQ_ERR_MISALIGNED;
+  if ((st = device_check(nullptr)) != SVDQ_OK) return st;
+  void* ws = nullptr;
+  if ((st = static_ws_address(&ws)) != SVDQ_OK) return st;
+  return svdq_linear_forward(w, X, M, ldx, Y, ldy, ws, SVDQ_STATIC_WORKSPACE_BYTES, stream);
+}
+
 extern "C" svdq_status svdq_device_error(void* stream, int* code) {
   if (!code) return SVDQ_ERR_INVALID_ARG;
   *code = 0;
