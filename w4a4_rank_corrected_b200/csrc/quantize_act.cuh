@@ -8,43 +8,99 @@
 // pass over the activations.  The B200 design:
 //
 //   * one CTA owns 64 rows x a contiguous slice of K (64-column chunks).  The
-//     host picks how many CTAs split K (a thread-block cluster of 1, 2, 4 or
-//     8) so that the whole grid is resident in one wave;
-//   * warp 0 streams X chunks [64 x 64] bf16, the matching chunk of the
-//     low-rank operand and 64 smoothing factors into a deep shared-memory
-//     ring with TMA (128-byte swizzle);
-//   * W quantize warps (W = number of ring stages, up to 8): warp w owns ring
-//     stage w and processes every chunk that lands there, whole.  Lane l
-//     handles rows l and l + 32 (all four 16-groups): it copies its rows and
-//     the chunk's smoothing factors into registers and hands the stage back
-//     before quantizing, so the next chunk for that stage is already loading
-//     while this one is processed; the warps work on different chunks at the
-//     same time instead of in lockstep.  Per group: multiply by the
-//     smoothing factors, take the maximum in registers, form the E4M3 block
-//     scale with one multiply and the hardware conversion, look up g/scale in
-//     a 127-entry table (the IEEE quotients, computed once per CTA), form the
-//     E2M1 codes with the hardware conversion; per row: 32 code bytes and one
-//     32-bit word of scales straight into the MMA tile layout;
+//     host picks how many CTAs split K (a thread-block cluster of up to 8)
+//     so that the whole grid is resident in one wave;
+//   * the slice's smoothing factors are loaded once (bulk copy) and stay in
+//     shared memory;
+//   * warp 0 streams X chunks [64 x 64] bf16 into a deep ring (8 or 16
+//     stages, TMA, 128-byte swizzle): the ring holds only X, so up to 128 KB
+//     of activations per SM are in flight, which is what it takes to cover
+//     HBM latency at full bandwidth;
+//   * warp 2 streams the matching chunks of the low-rank operand L1' into a
+//     separate ring of up to 8 stages (they come from L2: every row block
+//     reads the same L1', so each row block starts its K slice at a
+//     different chunk to spread those reads);
+//   * QA_QWARPS quantize warps: unit u = (chunk u / 2, rows 32 (u % 2) ..
+//     + 31) goes to warp u % QA_QWARPS; lane l handles one row.  A warp copies
+//     its row segment (128 bytes per lane) into registers, hands the X stage
+//     back, then quantizes: per 16-group multiply by the smoothing factors,
+//     take the maximum, form the E4M3 block scale with one multiply and the
+//     hardware conversion, look up g/scale in a 127-entry table (the IEEE
+//     quotients, computed once per CTA), form the E2M1 codes with the
+//     hardware conversion; per row 32 code bytes and one 32-bit word of
+//     scales go straight into the MMA tile layout;
 //   * warp 1 issues tcgen05 bf16 MMAs (M = 64) on the SAME shared-memory X
 //     tile: X [64 x 64] times L1' [2r x 64]^T into a 64 x 2r fp32 accumulator
 //     in tensor memory.  L1' holds smooth * L1 split into bf16 hi and lo
 //     halves, so X L1' = X_hat L1 to ~2^-16 relative (X itself is exact);
-//   * at the end the accumulator is read back (tcgen05.ld), hi + lo columns
-//     are summed, the partial sums of a K split are reduced across the
-//     cluster through distributed shared memory in a fixed order
-//     (deterministic), and the result times lr_scale is stored as a bf16
-//     hi/lo pair for the GEMM's up-projection.
+//   * at the end the accumulator is read back (tcgen05.ld) and hi + lo
+//     columns are summed.  In a K split every rank but 0 pushes its partial
+//     sums into rank 0's shared memory with st.async (the bytes are counted
+//     on a barrier there), rank 0 adds them in rank order (deterministic) and
+//     stores the result times lr_scale as a bf16 hi/lo pair for the GEMM's
+//     up-projection.
 #pragma once
 #include "ptx.cuh"
 
 namespace svdq_dev {
 
 constexpr int QA_BM = 64;
-constexpr int QA_MAX_STAGES = 8;
-constexpr int QA_QWARPS = QA_MAX_STAGES;                 // one per ring stage (at most)
-constexpr int QA_THREADS = 32 * (2 + QA_QWARPS);
-constexpr uint32_t QA_X_BYTES = QA_BM * 128;  // 64 rows x 64 bf16
-constexpr uint32_t QA_RING_BUDGET = 180 * 1024;
+constexpr int QA_QWARPS = 16;
+constexpr int QA_QWARP0 = 3;                               // first quantize warp
+constexpr int QA_THREADS = 32 * (QA_QWARP0 + QA_QWARPS);
+constexpr uint32_t QA_X_BYTES = QA_BM * 128;               // 64 rows x 64 bf16
+// X ring depth: a multiple of QA_QWARPS / 2.  Warp w's units cover chunks
+// w / 2, w / 2 + 8, w / 2 + 16, ...; with the depth a multiple of 8, the
+// previous use of the stage a warp is about to wait on was that same warp's
+// own earlier chunk, which it has already seen land, so the stage's barrier
+// is never two phases behind a parity wait (which would pass at once).
+constexpr int QA_XST_STEP = QA_QWARPS / 2;
+constexpr int QA_MAX_XST = 16;
+constexpr int QA_MIN_XST = QA_XST_STEP;
+constexpr int QA_MAX_LST = 8;
+static_assert(QA_MAX_XST % QA_XST_STEP == 0, "ring depth must be a multiple of 8");
+constexpr uint32_t QA_SMEM_BUDGET = 224 * 1024;  // + 1.5 KB: within the 227 KB per CTA
+
+// Shared-memory plan of one CTA (offsets from the 1024-aligned base).
+struct QALayout {
+  int xst, lst;              // ring depths (X, low-rank operand)
+  uint32_t l1_bytes;         // one low-rank stage: 2r rows x 128 bytes
+  uint32_t l1_off, s_off, red_off, lut_off, bar_off;
+  uint32_t total;            // bytes to request (incl. alignment slack)
+};
+
+__host__ __device__ inline QALayout qa_layout(int r, int chunks_per_split, int num_splits) {
+  QALayout L;
+  L.l1_bytes = 256u * (uint32_t)r;
+  const uint32_t s_bytes = 256u * (uint32_t)chunks_per_split;
+  const uint32_t red_bytes =
+      (r > 0 && num_splits > 1) ? (uint32_t)(num_splits - 1) * QA_BM * (uint32_t)r * 4u : 0u;
+  const uint32_t fixed = s_bytes + red_bytes + 512u + 512u;
+  // X ring 16 deep if the low-rank ring still gets 2 stages, else 8; the
+  // low-rank ring takes what is left, up to 8 stages
+  L.xst = 0;
+  L.lst = 0;
+  for (int xst = QA_MAX_XST; xst >= QA_MIN_XST; xst -= QA_XST_STEP) {
+    const uint32_t used = fixed + (uint32_t)xst * QA_X_BYTES;
+    if (used > QA_SMEM_BUDGET) continue;
+    int lst = 0;
+    if (r > 0) {
+      lst = (int)((QA_SMEM_BUDGET - used) / L.l1_bytes);
+      lst = lst > QA_MAX_LST ? QA_MAX_LST : lst;
+      if (lst < 2) continue;
+    }
+    L.xst = xst;
+    L.lst = lst;
+    break;
+  }
+  L.l1_off = (uint32_t)L.xst * QA_X_BYTES;
+  L.s_off = L.l1_off + (uint32_t)L.lst * L.l1_bytes;
+  L.red_off = L.s_off + s_bytes;
+  L.lut_off = L.red_off + red_bytes;
+  L.bar_off = L.lut_off + 512u;
+  L.total = 1024u + L.bar_off + 512u;
+  return L;
+}
 
 struct QAParams {
   const float* smooth;
@@ -54,24 +110,11 @@ struct QAParams {
   int M, K, r, klr;
   int chunks_per_split;
   int num_splits;
-  int stages;
-  uint32_t stage_bytes;
+  QALayout L;
   uint32_t tmem_cols;
   float g_x, gs_x, lr_scale;
   uint64_t timeout_ns;
 };
-
-__host__ __device__ inline uint32_t qa_stage_bytes(int r) {
-  const uint32_t b = QA_X_BYTES + 256u * (uint32_t)r + 256u;
-  return (b + 1023u) & ~1023u;
-}
-__host__ __device__ inline int qa_stages(int r) {
-  int st = (int)(QA_RING_BUDGET / qa_stage_bytes(r));
-  return st > QA_MAX_STAGES ? QA_MAX_STAGES : (st < 2 ? 2 : st);
-}
-__host__ __device__ inline uint32_t qa_smem_bytes(int r) {
-  return 1024u + (uint32_t)qa_stages(r) * qa_stage_bytes(r) + 1024u;
-}
 
 __device__ __forceinline__ int64_t sf_tile_off(int row, int g, int K) {
   return ((int64_t)(row >> 7) * (K >> 6) + (g >> 2)) * 512 + (row & 31) * 16 +
@@ -118,35 +161,54 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
                                              ~uintptr_t(1023));
   const int r = p.r;
   const bool has_lr = r > 0;
-  const int ST = p.stages;
-  const uint32_t SB = p.stage_bytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + ST * SB);
-  const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = full0 + 8 * ST;
-  const uint32_t acc_full = full0 + 16 * ST;
-  const uint32_t drain_bar = acc_full + 8;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * ST + 2);
+  const QALayout& L = p.L;
+  const int XST = L.xst, LST = L.lst;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
+  const uint32_t x_full0 = smem_u32(bars);
+  const uint32_t x_empty0 = x_full0 + 8 * XST;
+  const uint32_t l_full0 = x_empty0 + 8 * XST;
+  const uint32_t l_empty0 = l_full0 + 8 * LST;
+  const uint32_t acc_full = l_empty0 + 8 * LST;
+  const uint32_t s_bar = acc_full + 8;
+  const uint32_t red_bar = acc_full + 16;
+  const uint32_t drain_bar = acc_full + 24;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * XST + 2 * LST + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  float* qlut = reinterpret_cast<float*>(smem + ST * SB + 512);  // 128 floats
+  float* qlut = reinterpret_cast<float*>(smem + L.lut_off);  // 128 floats
+  const float* s_sm = reinterpret_cast<const float*>(smem + L.s_off);
 
   const uint32_t warp = warp_id(), lane = lane_id();
-  const int split = blockIdx.x;
+  const int split = blockIdx.x;  // = rank in the cluster when S > 1
   const int rb = blockIdx.y;
+  const int S = p.num_splits;
+  const bool reduce = has_lr && S > 1;
   const int kchunks = p.K >> 6;
   const int c_begin = split * p.chunks_per_split;
   const int c_end = min(kchunks, c_begin + p.chunks_per_split);
   const int nchunks = max(0, c_end - c_begin);
+  // Row blocks walk their K slice from different starting chunks, so the
+  // CTAs do not all ask L2 for the same low-rank tile at the same moment.
+  const int rot = nchunks > 0 ? rb % nchunks : 0;
   const unsigned int kid = 1;  // kernel id in error codes
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < ST; ++i) {
-      mbar_init(full0 + 8 * i, 1);
-      mbar_init(empty0 + 8 * i, 1 + (has_lr ? 1 : 0));
+    for (int i = 0; i < XST; ++i) {
+      mbar_init(x_full0 + 8 * i, 1);
+      mbar_init(x_empty0 + 8 * i, 2 + (has_lr ? 1 : 0));  // two row halves + the MMA
+    }
+    for (int i = 0; i < LST; ++i) {
+      mbar_init(l_full0 + 8 * i, 1);
+      mbar_init(l_empty0 + 8 * i, 1);
     }
     mbar_init(acc_full, 1);
+    mbar_init(s_bar, 1);
+    mbar_init(red_bar, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     mbar_fence_init();
+    // rank 0 of a K split expects the other ranks' partial sums
+    if (reduce && split == 0)
+      mbar_arrive_expect_tx(red_bar, (uint32_t)(S - 1) * QA_BM * (uint32_t)r * 4u);
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tm_x);
@@ -164,213 +226,213 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  // every rank's barriers exist before any rank stores into another's
+  // shared memory (the matching wait comes before the epilogue)
+  if (reduce) cluster_arrive();
   const uint32_t tmem = has_lr ? *tmem_holder : 0u;
   // Everything above overlaps the tail of the previous kernel in the stream;
   // from here on this kernel reads and writes memory that kernel may touch.
   grid_dependency_wait();
   grid_launch_dependents();
 
-  int issued = 0;  // producer: chunks whose loads were issued
+  int x_issued = 0, l_issued = 0;  // producers: chunks whose loads were issued
   if (warp == 0) {
-    // ---------------------------------------------------- TMA producer ----
+    // -------------------------------------------------- X producer (TMA) ----
     if (lane == 0) {
-      const uint32_t tx = QA_X_BYTES + (has_lr ? 256u * r : 0u) + 256u;
+      if (nchunks > 0) {
+        mbar_arrive_expect_tx(s_bar, 256u * (uint32_t)nchunks);
+        bulk_load(smem_u32(smem + L.s_off), p.smooth + c_begin * 64, 256u * (uint32_t)nchunks,
+                  s_bar);
+      }
       int st = 0;
       uint32_t ph = 0;
       for (int i = 0; i < nchunks; ++i) {
-        if (!mbar_wait(empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) break;
-        const uint32_t sb = smem_u32(smem + st * SB);
-        const int c = c_begin + i;
-        mbar_arrive_expect_tx(full0 + 8 * st, tx);
-        tma_load_2d(sb, &tm_x, c * 64, rb * QA_BM, full0 + 8 * st);
-        if (has_lr) tma_load_2d(sb + QA_X_BYTES, &tm_l1, c * 64, 0, full0 + 8 * st);
-        bulk_load(sb + QA_X_BYTES + 256u * r, p.smooth + c * 64, 256, full0 + 8 * st);
-        issued = i + 1;
-        if (++st == ST) { st = 0; ph ^= 1; }
+        if (!mbar_wait(x_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) break;
+        const int cl = i + rot < nchunks ? i + rot : i + rot - nchunks;  // local chunk
+        mbar_arrive_expect_tx(x_full0 + 8 * st, QA_X_BYTES);
+        tma_load_2d(smem_u32(smem + st * QA_X_BYTES), &tm_x, (c_begin + cl) * 64, rb * QA_BM,
+                    x_full0 + 8 * st);
+        x_issued = i + 1;
+        if (++st == XST) { st = 0; ph ^= 1; }
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------ low-rank operand producer (TMA) ----
+    if (has_lr && lane == 0) {
+      int st = 0;
+      uint32_t ph = 0;
+      for (int i = 0; i < nchunks; ++i) {
+        if (!mbar_wait(l_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (5u << 8) | kid)) break;
+        const int cl = i + rot < nchunks ? i + rot : i + rot - nchunks;
+        mbar_arrive_expect_tx(l_full0 + 8 * st, L.l1_bytes);
+        tma_load_2d(smem_u32(smem + L.l1_off + st * L.l1_bytes), &tm_l1, (c_begin + cl) * 64, 0,
+                    l_full0 + 8 * st);
+        l_issued = i + 1;
+        if (++st == LST) { st = 0; ph ^= 1; }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------- down-projection ----
     if (has_lr && lane == 0) {
       const uint32_t idesc = idesc_bf16(QA_BM, 2 * r);
-      int st = 0;
-      uint32_t ph = 0;
+      int xs = 0, ls = 0;
+      uint32_t xph = 0, lph = 0;
       for (int i = 0; i < nchunks; ++i) {
-        if (!mbar_wait(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
+        if (!mbar_wait(x_full0 + 8 * xs, xph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
+        if (!mbar_wait(l_full0 + 8 * ls, lph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
         tc_fence_after();
-        const uint32_t sb = smem_u32(smem + st * SB);
-        const uint64_t da = sdesc_sw128(sb), db = sdesc_sw128(sb + QA_X_BYTES);
+        const uint64_t da = sdesc_sw128(smem_u32(smem + xs * QA_X_BYTES));
+        const uint64_t db = sdesc_sw128(smem_u32(smem + L.l1_off + ls * L.l1_bytes));
         for (int kk = 0; kk < 4; ++kk)  // K = 16 bf16 = 32 bytes per MMA
           mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
-        tc_commit(empty0 + 8 * st);
-        if (++st == ST) { st = 0; ph ^= 1; }
+        tc_commit(x_empty0 + 8 * xs);
+        tc_commit(l_empty0 + 8 * ls);
+        if (++xs == XST) { xs = 0; xph ^= 1; }
+        if (++ls == LST) { ls = 0; lph ^= 1; }
       }
       tc_commit(acc_full);
     }
   } else {
     // ---------------------------------------------- NVFP4 quantization ----
-    // warp qw owns ring stage qw: chunks qw, qw + ST, qw + 2 ST, ...
-    const int qw = warp - 2;
+    const int qw = warp - QA_QWARP0;
     const float gs = p.gs_x;
-    if (qw < ST) {
-      const uint32_t sb = smem_u32(smem + qw * SB);
-      const uint8_t* sbp = smem + qw * SB;
-      uint32_t ph = 0;
-      for (int i = qw; i < nchunks; i += ST, ph ^= 1) {
-        if (!mbar_wait_warp(full0 + 8 * qw, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) break;
-        const int c = c_begin + i;
-        // copy this lane's two rows and the chunk's smoothing factors into
-        // registers, then hand the stage back so the next chunk can land
-        // while this one is quantized
-        uint4 xr[2][8];
-        float4 sv[16];
+    bool ok = nchunks == 0 || mbar_wait_warp(s_bar, 0, p.timeout_ns, abort_flag, (3u << 8) | kid);
+    for (int u = qw; ok && u < 2 * nchunks; u += QA_QWARPS) {
+      const int i = u >> 1;
+      const int cl = i + rot < nchunks ? i + rot : i + rot - nchunks;  // local chunk
+      const int st = i % XST;
+      const uint32_t ph = (uint32_t)(i / XST) & 1u;
+      if (!mbar_wait_warp(x_full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) break;
+      const int row_t = 32 * (u & 1) + lane;
+      const int row = rb * QA_BM + row_t;
+      const uint8_t* xrow = smem + st * QA_X_BYTES + row_t * 128;
+      // copy this lane's row segment into registers, then hand the stage
+      // back so the next chunk can land while this one is quantized
+      uint4 xr[8];
 #pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const int row_t = lane + 32 * hr;
+      for (int j = 0; j < 8; ++j)
+        xr[j] = *reinterpret_cast<const uint4*>(xrow + ((j ^ (row_t & 7)) << 4));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(x_empty0 + 8 * st);
+      const float4* sp = reinterpret_cast<const float4*>(s_sm + cl * 64);
+      uint32_t cw[8];
+      uint32_t sfw = 0;
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            xr[hr][j] = *reinterpret_cast<const uint4*>(sbp + row_t * 128 + ((j ^ (row_t & 7)) << 4));
+      for (int g = 0; g < 4; ++g) {
+        const uint4 x0 = xr[2 * g], x1 = xr[2 * g + 1];
+        const float4 s0 = sp[4 * g], s1 = sp[4 * g + 1], s2 = sp[4 * g + 2], s3 = sp[4 * g + 3];
+        float v[16];
+        v[0] = __fmul_rn(bf16_lo_f32(x0.x), s0.x);
+        v[1] = __fmul_rn(bf16_hi_f32(x0.x), s0.y);
+        v[2] = __fmul_rn(bf16_lo_f32(x0.y), s0.z);
+        v[3] = __fmul_rn(bf16_hi_f32(x0.y), s0.w);
+        v[4] = __fmul_rn(bf16_lo_f32(x0.z), s1.x);
+        v[5] = __fmul_rn(bf16_hi_f32(x0.z), s1.y);
+        v[6] = __fmul_rn(bf16_lo_f32(x0.w), s1.z);
+        v[7] = __fmul_rn(bf16_hi_f32(x0.w), s1.w);
+        v[8] = __fmul_rn(bf16_lo_f32(x1.x), s2.x);
+        v[9] = __fmul_rn(bf16_hi_f32(x1.x), s2.y);
+        v[10] = __fmul_rn(bf16_lo_f32(x1.y), s2.z);
+        v[11] = __fmul_rn(bf16_hi_f32(x1.y), s2.w);
+        v[12] = __fmul_rn(bf16_lo_f32(x1.z), s3.x);
+        v[13] = __fmul_rn(bf16_hi_f32(x1.z), s3.y);
+        v[14] = __fmul_rn(bf16_lo_f32(x1.w), s3.z);
+        v[15] = __fmul_rn(bf16_hi_f32(x1.w), s3.w);
+        float m0 = fmaxf(fabsf(v[0]), fabsf(v[1])), m1 = fmaxf(fabsf(v[2]), fabsf(v[3]));
+        float m2 = fmaxf(fabsf(v[4]), fabsf(v[5])), m3 = fmaxf(fabsf(v[6]), fabsf(v[7]));
+        float m4 = fmaxf(fabsf(v[8]), fabsf(v[9])), m5 = fmaxf(fabsf(v[10]), fabsf(v[11]));
+        float m6 = fmaxf(fabsf(v[12]), fabsf(v[13])), m7 = fmaxf(fabsf(v[14]), fabsf(v[15]));
+        const float a = fmaxf(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), fmaxf(fmaxf(m4, m5), fmaxf(m6, m7)));
+        const uint32_t code = cvt_e4m3x2(__fmul_rn(a, gs), 0.0f) & 0xFF;
+        const float q = qlut[code];
+        float t0[8], t1[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          t0[e] = __fmul_rn(v[e], q);
+          t1[e] = __fmul_rn(v[8 + e], q);
         }
-        {
-          const float4* sp = reinterpret_cast<const float4*>(sbp + QA_X_BYTES + 256u * r);
-#pragma unroll
-          for (int j = 0; j < 16; ++j) sv[j] = sp[j];
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + 8 * qw);
-#pragma unroll
-        for (int hr = 0; hr < 2; ++hr) {
-          const int row_t = lane + 32 * hr;
-          const int row = rb * QA_BM + row_t;
-          uint32_t cw[8];
-          uint32_t sfw = 0;
-#pragma unroll
-          for (int g = 0; g < 4; ++g) {
-            const uint4 x0 = xr[hr][2 * g], x1 = xr[hr][2 * g + 1];
-            const float4 s0 = sv[4 * g], s1 = sv[4 * g + 1], s2 = sv[4 * g + 2], s3 = sv[4 * g + 3];
-            float v[16];
-            v[0] = __fmul_rn(bf16_lo_f32(x0.x), s0.x);
-            v[1] = __fmul_rn(bf16_hi_f32(x0.x), s0.y);
-            v[2] = __fmul_rn(bf16_lo_f32(x0.y), s0.z);
-            v[3] = __fmul_rn(bf16_hi_f32(x0.y), s0.w);
-            v[4] = __fmul_rn(bf16_lo_f32(x0.z), s1.x);
-            v[5] = __fmul_rn(bf16_hi_f32(x0.z), s1.y);
-            v[6] = __fmul_rn(bf16_lo_f32(x0.w), s1.z);
-            v[7] = __fmul_rn(bf16_hi_f32(x0.w), s1.w);
-            v[8] = __fmul_rn(bf16_lo_f32(x1.x), s2.x);
-            v[9] = __fmul_rn(bf16_hi_f32(x1.x), s2.y);
-            v[10] = __fmul_rn(bf16_lo_f32(x1.y), s2.z);
-            v[11] = __fmul_rn(bf16_hi_f32(x1.y), s2.w);
-            v[12] = __fmul_rn(bf16_lo_f32(x1.z), s3.x);
-            v[13] = __fmul_rn(bf16_hi_f32(x1.z), s3.y);
-            v[14] = __fmul_rn(bf16_lo_f32(x1.w), s3.z);
-            v[15] = __fmul_rn(bf16_hi_f32(x1.w), s3.w);
-            float m0 = fmaxf(fabsf(v[0]), fabsf(v[1])), m1 = fmaxf(fabsf(v[2]), fabsf(v[3]));
-            float m2 = fmaxf(fabsf(v[4]), fabsf(v[5])), m3 = fmaxf(fabsf(v[6]), fabsf(v[7]));
-            float m4 = fmaxf(fabsf(v[8]), fabsf(v[9])), m5 = fmaxf(fabsf(v[10]), fabsf(v[11]));
-            float m6 = fmaxf(fabsf(v[12]), fabsf(v[13])), m7 = fmaxf(fabsf(v[14]), fabsf(v[15]));
-            const float a = fmaxf(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), fmaxf(fmaxf(m4, m5), fmaxf(m6, m7)));
-            const uint32_t code = cvt_e4m3x2(__fmul_rn(a, gs), 0.0f) & 0xFF;
-            const float q = qlut[code];
-            float t0[8], t1[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              t0[e] = __fmul_rn(v[e], q);
-              t1[e] = __fmul_rn(v[8 + e], q);
-            }
-            cw[2 * g] = cvt_e2m1x8(t0);
-            cw[2 * g + 1] = cvt_e2m1x8(t1);
-            sfw |= code << (8 * g);
-          }
-          if (row < p.M) {
-            uint4* dst = reinterpret_cast<uint4*>(p.codes_x + (size_t)row * (p.K >> 1) + (size_t)c * 32);
-            dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-            dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-          }
-          *reinterpret_cast<uint32_t*>(p.sf_x + sf_tile_off(row, 4 * c, p.K)) = sfw;
-        }
+        cw[2 * g] = cvt_e2m1x8(t0);
+        cw[2 * g + 1] = cvt_e2m1x8(t1);
+        sfw |= code << (8 * g);
       }
-      (void)sb;
-    }
-
-    // ----------------------------------------- low-rank epilogue (X L1) ----
-    if (has_lr) {
-      const bool ok = mbar_wait_warp(acc_full, 0, p.timeout_ns, abort_flag, (4u << 8) | kid);
-      tc_fence_after();
-      // M = 64 accumulator: row m sits in lane (m % 16) + 32 (m / 16).  Warp w
-      // reads its lane quarter w % 4; lanes 0..15 hold rows 16 (w % 4) + lane.
-      const int quad = warp & 3;
-      const int hc = (warp - 2) >> 2;          // 0..1: which chunks of 16 columns
-      const int lrow_t = quad * 16 + lane;
-      const int lrow = rb * QA_BM + lrow_t;
-      const bool own = lane < 16;
-      const int S = p.num_splits;
-      float* P = reinterpret_cast<float*>(smem);  // [64][r+1], reuses the ring
-      const int pstride = r + 1;
-      // every quantize warp is done reading the ring before it is reused
-      asm volatile("bar.sync 1, %0;" ::"n"(32 * QA_QWARPS) : "memory");
-      for (int ci = hc; ci < r / 16; ci += QA_QWARPS / 4) {  // QA_QWARPS / 4 warps per quarter
-        uint32_t hi[16], lo[16];
-        const uint32_t base = tmem + ((uint32_t)(quad * 32) << 16);
-        if (ok) {
-          tmem_ld16(base + 16 * ci, hi);
-          tmem_ld16(base + r + 16 * ci, lo);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) hi[j] = lo[j] = 0u;
-        }
-        float part[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) part[j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
-        if (own) {
-          if (S > 1) {
-#pragma unroll
-            for (int j = 0; j < 16; ++j) P[lrow_t * pstride + 16 * ci + j] = part[j];
-          } else if (lrow < p.M) {
-            store_hi_lo16(part, p.lr_scale, p.xl1 + (size_t)lrow * p.klr + 16 * ci,
-                          p.xl1 + (size_t)lrow * p.klr + r + 16 * ci);
-          }
-        }
+      if (row < p.M) {
+        uint4* dst = reinterpret_cast<uint4*>(p.codes_x + (size_t)row * (p.K >> 1) +
+                                              (size_t)(c_begin + cl) * 32);
+        dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+        dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
       }
-      if (S == 1 && hc == 0 && own && lrow < p.M) {
-        for (int cpad = 2 * r; cpad < p.klr; cpad += 8)
-          *reinterpret_cast<uint4*>(p.xl1 + (size_t)lrow * p.klr + cpad) = make_uint4(0, 0, 0, 0);
-      }
+      *reinterpret_cast<uint32_t*>(p.sf_x + sf_tile_off(row, 4 * (c_begin + cl), p.K)) = sfw;
     }
   }
 
-  // ------------------------------------ cross-CTA reduction of X L1 parts ----
-  if (has_lr && p.num_splits > 1) {
-    tc_fence_before();
-    __syncthreads();
-    cluster_sync();  // every rank's partial sums are in its shared memory
-    if (blockIdx.x == 0 && warp >= 2) {
-      const int t = threadIdx.x - 64;           // 0..255
-      const int lrow_t = t >> 2;                // 64 rows x 4 threads
-      const int lrow = rb * QA_BM + lrow_t;
-      const int pstride = r + 1;
-      const uint32_t Pbase = smem_u32(smem);
-      if (lrow < p.M) {
-        for (int ci = (t & 3); ci < r / 16; ci += 4) {
-          float acc[16];
+  // ----------------------------------------- low-rank epilogue (X L1) ----
+  if (reduce) cluster_wait();
+  if (has_lr && warp >= QA_QWARP0) {
+    const bool ok = mbar_wait_warp(acc_full, 0, p.timeout_ns, abort_flag, (4u << 8) | kid);
+    tc_fence_after();
+    // M = 64 accumulator: row m sits in lane (m % 16) + 32 (m / 16).  Warp w
+    // reads its lane quarter w % 4; lanes 0..15 hold rows 16 (w % 4) + lane.
+    const int quad = warp & 3;
+    const int slot = (warp - QA_QWARP0) >> 2;   // 0 .. QA_QWARPS / 4 - 1
+    const int lrow_t = quad * 16 + lane;
+    const int lrow = rb * QA_BM + lrow_t;
+    const bool own = lane < 16;
+    const uint32_t red_base = smem_u32(smem + L.red_off);
+    const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
+    for (int ci = slot; ci < r / 16; ci += QA_QWARPS / 4) {
+      uint32_t hi[16], lo[16];
+      if (ok) {
+        tmem_ld16(tbase + 16 * ci, hi);
+        tmem_ld16(tbase + r + 16 * ci, lo);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
-          for (int s = 0; s < p.num_splits; ++s) {
-            const uint32_t rbase = map_to_rank(Pbase, (uint32_t)s);
+        for (int j = 0; j < 16; ++j) hi[j] = lo[j] = 0u;
+      }
+      float part[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-              acc[j] += ld_cluster_f32(rbase + 4u * (uint32_t)(lrow_t * pstride + 16 * ci + j));
+      for (int j = 0; j < 16; ++j) part[j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
+      if (!reduce) {
+        if (own && lrow < p.M)
+          store_hi_lo16(part, p.lr_scale, p.xl1 + (size_t)lrow * p.klr + 16 * ci,
+                        p.xl1 + (size_t)lrow * p.klr + r + 16 * ci);
+      } else if (split != 0) {
+        // partial sums [row][r] of rank `split` into rank 0's buffer split-1
+        if (own) {
+          const uint32_t dst = map_to_rank(
+              red_base + 4u * (uint32_t)(((split - 1) * QA_BM + lrow_t) * r + 16 * ci), 0);
+          const uint32_t bar = map_to_rank(red_bar, 0);
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            st_async_v4(dst + 4u * j, part[j], part[j + 1], part[j + 2], part[j + 3], bar);
+        }
+      } else {
+        const bool got = mbar_wait_warp(red_bar, 0, p.timeout_ns, abort_flag, (6u << 8) | kid);
+        if (own && lrow < p.M) {
+          if (got) {
+            for (int sr = 1; sr < S; ++sr) {
+              const float4* q4 = reinterpret_cast<const float4*>(
+                  smem + L.red_off + 4u * (uint32_t)(((sr - 1) * QA_BM + lrow_t) * r + 16 * ci));
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const float4 t = q4[j];
+                part[4 * j] += t.x;
+                part[4 * j + 1] += t.y;
+                part[4 * j + 2] += t.z;
+                part[4 * j + 3] += t.w;
+              }
+            }
           }
-          store_hi_lo16(acc, p.lr_scale, p.xl1 + (size_t)lrow * p.klr + 16 * ci,
+          store_hi_lo16(part, p.lr_scale, p.xl1 + (size_t)lrow * p.klr + 16 * ci,
                         p.xl1 + (size_t)lrow * p.klr + r + 16 * ci);
         }
-        if ((t & 3) == 0)
-          for (int cpad = 2 * r; cpad < p.klr; cpad += 8)
-            *reinterpret_cast<uint4*>(p.xl1 + (size_t)lrow * p.klr + cpad) = make_uint4(0, 0, 0, 0);
       }
     }
-    cluster_sync();  // keep every rank's shared memory alive until read
+    // zero columns [2r, klr) of the rows this CTA finishes
+    if (split == 0 && slot == 0 && own && lrow < p.M) {
+      for (int cpad = 2 * r; cpad < p.klr; cpad += 8)
+        *reinterpret_cast<uint4*>(p.xl1 + (size_t)lrow * p.klr + cpad) = make_uint4(0, 0, 0, 0);
+    }
   }
 
   // ------------------------------------------------------------ teardown ----
@@ -379,8 +441,13 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   if (*abort_flag) {
     // drain: loads still in flight, then tensor-core work still in flight
     if (warp == 0 && lane == 0) {
-      for (int i = max(0, issued - ST); i < issued; ++i)
-        mbar_wait_drain(full0 + 8 * (i % ST), (i / ST) & 1, p.timeout_ns);
+      for (int i = max(0, x_issued - XST); i < x_issued; ++i)
+        mbar_wait_drain(x_full0 + 8 * (i % XST), (i / XST) & 1, p.timeout_ns);
+      if (nchunks > 0) mbar_wait_drain(s_bar, 0, p.timeout_ns);
+    }
+    if (warp == 2 && lane == 0) {
+      for (int i = max(0, l_issued - LST); i < l_issued; ++i)
+        mbar_wait_drain(l_full0 + 8 * (i % LST), (i / LST) & 1, p.timeout_ns);
     }
     if (warp == 1 && lane == 0 && has_lr) {
       tc_commit(drain_bar);
@@ -388,6 +455,8 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
     }
     __syncthreads();
   }
+  // no rank leaves while another may still store into its shared memory
+  if (reduce) cluster_sync();
   if (warp == 1 && has_lr) {
     tc_fence_after();
     tmem_dealloc(tmem, p.tmem_cols);

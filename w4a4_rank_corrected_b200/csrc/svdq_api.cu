@@ -95,8 +95,7 @@ svdq_status device_check(int* sms) {
   }
   if (!d.ok) return SVDQ_ERR_UNSUPPORTED_ARCH;
   if (!d.attrs_set) {
-    uint32_t qa_max = 0;
-    for (int rr = 0; rr <= 128; rr += 16) qa_max = std::max(qa_max, qa_smem_bytes(rr));
+    const uint32_t qa_max = 1024u + QA_SMEM_BUDGET + 512u;  // every qa_layout fits
     if (cudaFuncSetAttribute(quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)qa_max) != cudaSuccess ||
         cudaFuncSetAttribute(w4a4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -163,21 +162,25 @@ cudaLaunchAttribute pdl_attr() {
 }
 
 // Largest K split S (cluster size when the low-rank branch needs the
-// cross-CTA reduction) such that the whole grid is resident in one wave.
+// cross-CTA reduction) such that the whole grid is resident in one wave and
+// the split's shared-memory plan keeps a deep enough activation ring.
 int choose_splits(int tiles, int kchunks, int r, int sms) {
   int dev = 0;
   cudaGetDevice(&dev);
   int best = 1;
   for (int S = 2; S <= 8; ++S) {
     if (S > kchunks || tiles * S > sms) break;
+    const int cps = (kchunks + S - 1) / S;
+    const QALayout L = qa_layout(r, cps, S);
+    if (L.xst < QA_MIN_XST) break;
     if (r > 0) {
-      int& cached = g_dev[dev].max_clusters[r / 16][S];
+      int& cached = g_dev[dev].max_clusters[0][S];
       if (cached < 0) {
         cudaLaunchConfig_t cfg;
         std::memset(&cfg, 0, sizeof(cfg));
         cfg.gridDim = dim3((unsigned)S, 1, 1);
         cfg.blockDim = dim3(QA_THREADS, 1, 1);
-        cfg.dynamicSmemBytes = qa_smem_bytes(r);
+        cfg.dynamicSmemBytes = L.total;
         cudaLaunchAttribute attr;
         attr.id = cudaLaunchAttributeClusterDimension;
         attr.val.clusterDim.x = (unsigned)S;
@@ -210,6 +213,8 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
   int S = choose_splits(tiles, KC, r, sms);
   const int cps = (KC + S - 1) / S;
   S = (KC + cps - 1) / cps;
+  const QALayout L = qa_layout(r, cps, S);
+  if (L.xst < QA_MIN_XST) return SVDQ_ERR_INVALID_ARG;  // K too large for one CTA's slice
 
   CUtensorMap tm_x, tm_l1;
   std::memset(&tm_l1, 0, sizeof(tm_l1));
@@ -231,8 +236,7 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
   p.klr = klr_of(r);
   p.chunks_per_split = cps;
   p.num_splits = S;
-  p.stages = qa_stages(r);
-  p.stage_bytes = qa_stage_bytes(r);
+  p.L = L;
   uint32_t cols = 32;
   while (cols < (uint32_t)(2 * r)) cols <<= 1;
   p.tmem_cols = cols;
@@ -245,7 +249,7 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)S, (unsigned)tiles, 1);
   cfg.blockDim = dim3(QA_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = qa_smem_bytes(r);
+  cfg.dynamicSmemBytes = L.total;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0] = pdl_attr();

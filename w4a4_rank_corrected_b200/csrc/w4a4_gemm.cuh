@@ -18,6 +18,12 @@
 //     activation scales, all 256 rows of weight scales) into a 5-deep ring;
 //     every load is counted on the leader CTA's barrier (cta_group::2 form,
 //     no multicast);
+//   * each pair works through a contiguous run of output tiles in M-major
+//     order; for K <= 3072 the activation scales of the current 256-row
+//     block stay in tensor memory (192 columns beside the 256-column
+//     accumulator) and are loaded and copied only when the run enters a new
+//     row block, which takes a third of the scale copies off the MMA
+//     issuer's path (each copy beyond about one per MMA stalls it);
 //   * warp 1 of the leader copies the scale atoms into both CTAs' tensor
 //     memory (tcgen05.cp cta_group::2) and issues
 //     tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 (M = 256,
@@ -48,8 +54,14 @@ constexpr uint32_t G_STAGE_BYTES = G_A_BYTES + G_B_BYTES + G_SFA_BYTES + G_SFB_B
 constexpr uint32_t G_TMEM_COLS = 512;
 constexpr uint32_t G_SF_TMEM = 256;          // scale buffers after the accumulator
 constexpr uint32_t G_SF_TMEM_STRIDE = 48;    // 16 cols SFA + 32 cols SFB
+// Resident activation scales: 4 columns per 64-deep K step, all of K, for
+// K <= 3072 (192 columns); then the weight scales double-buffer after them.
+constexpr int G_SFA_RES_MAX_K64 = 48;
+constexpr uint32_t G_SFB_RES_TMEM = G_SF_TMEM + 4 * G_SFA_RES_MAX_K64;  // 448
+constexpr uint32_t G_SFB_RES_STRIDE = 32;
 constexpr uint32_t G_BIAS_BYTES = 2 * G_BN * 4;   // two fp32 bias tiles
 constexpr uint32_t G_FP4_TX = 2 * G_STAGE_BYTES;  // bytes per FP4 stage, both CTAs
+constexpr uint32_t G_FP4_TX_NOSFA = 2 * (G_STAGE_BYTES - G_SFA_BYTES);
 constexpr uint32_t G_LR_TX = 2 * (G_A_BYTES + G_B_BYTES);
 
 __host__ __device__ inline uint32_t gemm_smem_bytes() {
@@ -94,7 +106,13 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   const int num_n = (N + G_BN - 1) / G_BN;
   const int num_tiles = num_m * num_n;
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+  // Each pair takes a contiguous run of tiles in M-major order (tile t is
+  // M block t / num_n, N block t % num_n), so consecutive tiles mostly share
+  // their activation rows and those rows' scales stay in tensor memory.
+  const int t_begin = (int)(((long long)pair * num_tiles) / num_pairs);
+  const int t_end = (int)(((long long)(pair + 1) * num_tiles) / num_pairs);
   const int k64 = K >> 6;
+  const bool sfa_res = k64 <= G_SFA_RES_MAX_K64;
   const int kb_total = (k64 + 3) >> 2;
   const int lr_chunks = has_lr ? (p.klr >> 6) : 0;
   const unsigned int kid = 2;
@@ -144,8 +162,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     if (lane == 0) {
       int it = 0;
       bool stop = false;
-      for (int tile = pair; tile < num_tiles && !stop; tile += num_pairs) {
-        const int mb = tile % num_m, nb = tile / num_m;
+      for (int tile = t_begin; tile < t_end && !stop; ++tile) {
+        const int mb = tile / num_n, nb = tile % num_n;
+        const bool load_sfa = !sfa_res || tile == t_begin || nb == 0;
         const int row0 = mb * 2 * G_BM + (int)rank * G_BM;     // this CTA's A rows
         const int brow0 = nb * G_BN + (int)rank * G_BN_CTA;    // this CTA's B rows
         const int sfa_blk = mb * 2 + (int)rank;                // 128-row scale block
@@ -157,13 +176,14 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             break;
           }
           const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
-          if (leader) mbar_arrive_expect_tx(full0 + 8 * st, G_FP4_TX);
+          if (leader) mbar_arrive_expect_tx(full0 + 8 * st, load_sfa ? G_FP4_TX : G_FP4_TX_NOSFA);
           const uint32_t fb = lead_full0 + 8 * st;
           tma_load_2d_pair(sb, &tm_a, kb * 128, row0, fb);
           tma_load_2d_pair(sb + G_A_BYTES, &tm_b, kb * 128, brow0, fb);
           // scale atoms: rows of 256 bytes = half atoms; 4 atoms = 8 rows
-          tma_load_2d_pair(sb + G_A_BYTES + G_B_BYTES, &tm_sfa, 0,
-                           (sfa_blk * k64 + 4 * kb) * 2, fb);
+          if (load_sfa)
+            tma_load_2d_pair(sb + G_A_BYTES + G_B_BYTES, &tm_sfa, 0,
+                             (sfa_blk * k64 + 4 * kb) * 2, fb);
           for (int hh = 0; hh < 2; ++hh)
             tma_load_2d_pair(sb + G_A_BYTES + G_B_BYTES + G_SFA_BYTES + hh * 2048, &tm_sfb, 0,
                              ((2 * nb + hh) * k64 + 4 * kb) * 2, fb);
@@ -192,9 +212,12 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       const uint32_t id_lr = idesc_bf16(2 * G_BM, G_BN);
       int it = 0, tcount = 0;
       bool stop = false;
-      for (int tile = pair; tile < num_tiles && !stop; tile += num_pairs, ++tcount) {
+      for (int tile = t_begin; tile < t_end && !stop; ++tile, ++tcount) {
+        // (the accumulator is free only once every MMA of the previous tile
+        // has completed, so resident scales may be overwritten after this)
         if (!mbar_wait(acc_empty, (tcount & 1) ^ 1, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
         tc_fence_after();
+        const bool load_sfa = !sfa_res || tile == t_begin || tile % num_n == 0;
         uint32_t accumulate = 0;
         for (int kb = 0; kb < kb_total; ++kb, ++it) {
           const int st = it % G_STAGES;
@@ -208,10 +231,13 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
           const uint32_t sfa_s = sb + G_A_BYTES + G_B_BYTES;
           const uint32_t sfb_s = sfa_s + G_SFA_BYTES;
-          const uint32_t sfa_t = tmem + G_SF_TMEM + (it & 1) * G_SF_TMEM_STRIDE;
-          const uint32_t sfb_t = sfa_t + 16;
+          const uint32_t sfa_t = sfa_res ? tmem + G_SF_TMEM + 16 * kb
+                                         : tmem + G_SF_TMEM + (it & 1) * G_SF_TMEM_STRIDE;
+          const uint32_t sfb_t = sfa_res ? tmem + G_SFB_RES_TMEM + (it & 1) * G_SFB_RES_STRIDE
+                                         : sfa_t + 16;
           for (int kk = 0; kk < nk; ++kk) {
-            tmem_copy_32x128b_x4_pair(sfa_t + 4 * kk, sdesc_sf_block(sfa_s + 512 * kk));
+            if (load_sfa)
+              tmem_copy_32x128b_x4_pair(sfa_t + 4 * kk, sdesc_sf_block(sfa_s + 512 * kk));
             tmem_copy_32x128b_x4_pair(sfb_t + 8 * kk, sdesc_sf_block(sfb_s + 512 * kk));
             tmem_copy_32x128b_x4_pair(sfb_t + 8 * kk + 4, sdesc_sf_block(sfb_s + 2048 + 512 * kk));
           }
@@ -250,8 +276,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int et = threadIdx.x - 64;           // 0..255
     const float alpha = p.alpha;
     int tcount = 0;
-    for (int tile = pair; tile < num_tiles; tile += num_pairs, ++tcount) {
-      const int mb = tile % num_m, nb = tile / num_m;
+    for (int tile = t_begin; tile < t_end; ++tile, ++tcount) {
+      const int mb = tile / num_n, nb = tile % num_n;
       // stage this tile's bias (fp32) while the main loop runs.  Buffer
       // tcount&1 was last read for tile tcount-2, which every thread had
       // finished before arriving on the other buffer's barrier.
