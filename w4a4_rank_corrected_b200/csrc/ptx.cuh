@@ -24,6 +24,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// One lane of a converged warp (elect.sync).  Roles that issue TMA copies or
+// tcgen05 instructions run as whole warps: every lane waits on the barriers
+// and one elected lane issues, with the warp converged again after each
+// issue block.  A lone lane running the whole loop while the rest of its
+// warp waits elsewhere was measured at about half the issue rate.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

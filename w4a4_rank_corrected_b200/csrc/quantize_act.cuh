@@ -12,7 +12,8 @@
 //     so that the whole grid is resident in one wave;
 //   * the slice's smoothing factors are loaded once (bulk copy) and stay in
 //     shared memory;
-//   * warp 0 streams X chunks [64 x 64] bf16 into a deep ring (8 or 16
+//   * warp 0 (the whole warp waits, an elected lane issues; the same for
+//     warps 1 and 2) streams X chunks [64 x 64] bf16 into a deep ring (8 or 16
 //     stages, TMA, 128-byte swizzle): the ring holds only X, so up to 128 KB
 //     of activations per SM are in flight, which is what it takes to cover
 //     HBM latency at full bandwidth;
@@ -237,60 +238,76 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
 
   int x_issued = 0, l_issued = 0;  // producers: chunks whose loads were issued
   if (warp == 0) {
-    // -------------------------------------------------- X producer (TMA) ----
-    if (lane == 0) {
-      if (nchunks > 0) {
+    // ------------------------------------------- X producer (TMA, warp) ----
+    if (nchunks > 0) {
+      if (elect_one()) {
         mbar_arrive_expect_tx(s_bar, 256u * (uint32_t)nchunks);
         bulk_load(smem_u32(smem + L.s_off), p.smooth + c_begin * 64, 256u * (uint32_t)nchunks,
                   s_bar);
       }
-      int st = 0;
-      uint32_t ph = 0;
-      for (int i = 0; i < nchunks; ++i) {
-        if (!mbar_wait(x_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) break;
+      __syncwarp();
+    }
+    int st = 0;
+    uint32_t ph = 0;
+    for (int i = 0; i < nchunks; ++i) {
+      if (!mbar_wait_warp(x_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) break;
+      if (elect_one()) {
         const int cl = i + rot < nchunks ? i + rot : i + rot - nchunks;  // local chunk
         mbar_arrive_expect_tx(x_full0 + 8 * st, QA_X_BYTES);
         tma_load_2d(smem_u32(smem + st * QA_X_BYTES), &tm_x, (c_begin + cl) * 64, rb * QA_BM,
                     x_full0 + 8 * st);
-        x_issued = i + 1;
-        if (++st == XST) { st = 0; ph ^= 1; }
       }
+      __syncwarp();
+      x_issued = i + 1;
+      if (++st == XST) { st = 0; ph ^= 1; }
     }
   } else if (warp == 2) {
-    // ------------------------------------ low-rank operand producer (TMA) ----
-    if (has_lr && lane == 0) {
+    // ----------------------------- low-rank operand producer (TMA, warp) ----
+    if (has_lr) {
       int st = 0;
       uint32_t ph = 0;
       for (int i = 0; i < nchunks; ++i) {
-        if (!mbar_wait(l_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (5u << 8) | kid)) break;
-        const int cl = i + rot < nchunks ? i + rot : i + rot - nchunks;
-        mbar_arrive_expect_tx(l_full0 + 8 * st, L.l1_bytes);
-        tma_load_2d(smem_u32(smem + L.l1_off + st * L.l1_bytes), &tm_l1, (c_begin + cl) * 64, 0,
-                    l_full0 + 8 * st);
+        if (!mbar_wait_warp(l_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (5u << 8) | kid))
+          break;
+        if (elect_one()) {
+          const int cl = i + rot < nchunks ? i + rot : i + rot - nchunks;
+          mbar_arrive_expect_tx(l_full0 + 8 * st, L.l1_bytes);
+          tma_load_2d(smem_u32(smem + L.l1_off + st * L.l1_bytes), &tm_l1, (c_begin + cl) * 64, 0,
+                      l_full0 + 8 * st);
+        }
+        __syncwarp();
         l_issued = i + 1;
         if (++st == LST) { st = 0; ph ^= 1; }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------- down-projection ----
-    if (has_lr && lane == 0) {
+    // ------------------------------------------ down-projection (warp) ----
+    if (has_lr) {
       const uint32_t idesc = idesc_bf16(QA_BM, 2 * r);
       int xs = 0, ls = 0;
       uint32_t xph = 0, lph = 0;
       for (int i = 0; i < nchunks; ++i) {
-        if (!mbar_wait(x_full0 + 8 * xs, xph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
-        if (!mbar_wait(l_full0 + 8 * ls, lph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
-        tc_fence_after();
+        // both tiles have landed (complete_tx); the MMAs read them through
+        // the async proxy
+        if (!mbar_wait_warp(x_full0 + 8 * xs, xph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
+        if (!mbar_wait_warp(l_full0 + 8 * ls, lph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
         const uint64_t da = sdesc_sw128(smem_u32(smem + xs * QA_X_BYTES));
         const uint64_t db = sdesc_sw128(smem_u32(smem + L.l1_off + ls * L.l1_bytes));
-        for (int kk = 0; kk < 4; ++kk)  // K = 16 bf16 = 32 bytes per MMA
-          mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
-        tc_commit(x_empty0 + 8 * xs);
-        tc_commit(l_empty0 + 8 * ls);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {  // K = 16 bf16 = 32 bytes per MMA
+          if (elect_one()) mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
+          __syncwarp();
+        }
+        if (elect_one()) {
+          tc_commit(x_empty0 + 8 * xs);
+          tc_commit(l_empty0 + 8 * ls);
+        }
+        __syncwarp();
         if (++xs == XST) { xs = 0; xph ^= 1; }
         if (++ls == LST) { ls = 0; lph ^= 1; }
       }
-      tc_commit(acc_full);
+      if (elect_one()) tc_commit(acc_full);
+      __syncwarp();
     }
   } else {
     // ---------------------------------------------- NVFP4 quantization ----
@@ -449,9 +466,13 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
       for (int i = max(0, l_issued - LST); i < l_issued; ++i)
         mbar_wait_drain(l_full0 + 8 * (i % LST), (i / LST) & 1, p.timeout_ns);
     }
-    if (warp == 1 && lane == 0 && has_lr) {
-      tc_commit(drain_bar);
-      mbar_wait_drain(drain_bar, 0, p.timeout_ns);
+    if (warp == 1 && has_lr) {
+      // from the lane that issued the MMAs (elect.sync picks it again)
+      if (elect_one()) {
+        tc_commit(drain_bar);
+        mbar_wait_drain(drain_bar, 0, p.timeout_ns);
+      }
+      __syncwarp();
     }
     __syncthreads();
   }

@@ -13,7 +13,8 @@
 //     accumulator in its own tensor memory.  Per unit of MMA work each SM
 //     moves half the weight bytes through shared memory that a single-SM
 //     128 x 256 tile would, which is what keeps the tensor core fed;
-//   * warp 0 of each CTA streams, per 256-deep K step, its A and B code tiles
+//   * warp 0 of each CTA (the whole warp waits, one elected lane issues)
+//     streams, per 256-deep K step, its A and B code tiles
 //     (TMA, 128-byte swizzle) and the scale atoms (TMA; its own 128 rows of
 //     activation scales, all 256 rows of weight scales) into a 5-deep ring;
 //     every load is counted on the leader CTA's barrier (cta_group::2 form,
@@ -24,7 +25,8 @@
 //     accumulator) and are loaded and copied only when the run enters a new
 //     row block, which takes a third of the scale copies off the MMA
 //     issuer's path (each copy beyond about one per MMA stalls it);
-//   * warp 1 of the leader copies the scale atoms into both CTAs' tensor
+//   * warp 1 of the leader (converged; an elected lane issues each
+//     instruction) copies the scale atoms into both CTAs' tensor
 //     memory (tcgen05.cp cta_group::2) and issues
 //     tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 (M = 256,
 //     N = 256, K = 64); after the K loop it streams the low-rank operands
@@ -158,23 +160,23 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 
   int issued = 0;
   if (warp == 0) {
-    // ---------------------------------------------------- TMA producer ----
-    if (lane == 0) {
-      int it = 0;
-      bool stop = false;
-      for (int tile = t_begin; tile < t_end && !stop; ++tile) {
-        const int mb = tile / num_n, nb = tile % num_n;
-        const bool load_sfa = !sfa_res || tile == t_begin || nb == 0;
-        const int row0 = mb * 2 * G_BM + (int)rank * G_BM;     // this CTA's A rows
-        const int brow0 = nb * G_BN + (int)rank * G_BN_CTA;    // this CTA's B rows
-        const int sfa_blk = mb * 2 + (int)rank;                // 128-row scale block
-        for (int kb = 0; kb < kb_total; ++kb, ++it) {
-          const int st = it % G_STAGES;
-          const uint32_t ph = (it / G_STAGES) & 1;
-          if (!mbar_wait(empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) {
-            stop = true;
-            break;
-          }
+    // ---------------------------------------------- TMA producer (warp) ----
+    int it = 0;
+    bool stop = false;
+    for (int tile = t_begin; tile < t_end && !stop; ++tile) {
+      const int mb = tile / num_n, nb = tile % num_n;
+      const bool load_sfa = !sfa_res || tile == t_begin || nb == 0;
+      const int row0 = mb * 2 * G_BM + (int)rank * G_BM;     // this CTA's A rows
+      const int brow0 = nb * G_BN + (int)rank * G_BN_CTA;    // this CTA's B rows
+      const int sfa_blk = mb * 2 + (int)rank;                // 128-row scale block
+      for (int kb = 0; kb < kb_total; ++kb, ++it) {
+        const int st = it % G_STAGES;
+        const uint32_t ph = (it / G_STAGES) & 1;
+        if (!mbar_wait_warp(empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) {
+          stop = true;
+          break;
+        }
+        if (elect_one()) {
           const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
           if (leader) mbar_arrive_expect_tx(full0 + 8 * st, load_sfa ? G_FP4_TX : G_FP4_TX_NOSFA);
           const uint32_t fb = lead_full0 + 8 * st;
@@ -187,27 +189,31 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           for (int hh = 0; hh < 2; ++hh)
             tma_load_2d_pair(sb + G_A_BYTES + G_B_BYTES + G_SFA_BYTES + hh * 2048, &tm_sfb, 0,
                              ((2 * nb + hh) * k64 + 4 * kb) * 2, fb);
-          issued = it + 1;
         }
-        for (int c = 0; c < lr_chunks && !stop; ++c, ++it) {
-          const int st = it % G_STAGES;
-          const uint32_t ph = (it / G_STAGES) & 1;
-          if (!mbar_wait(empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) {
-            stop = true;
-            break;
-          }
+        __syncwarp();
+        issued = it + 1;
+      }
+      for (int c = 0; c < lr_chunks && !stop; ++c, ++it) {
+        const int st = it % G_STAGES;
+        const uint32_t ph = (it / G_STAGES) & 1;
+        if (!mbar_wait_warp(empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) {
+          stop = true;
+          break;
+        }
+        if (elect_one()) {
           const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
           if (leader) mbar_arrive_expect_tx(full0 + 8 * st, G_LR_TX);
           const uint32_t fb = lead_full0 + 8 * st;
           tma_load_2d_pair(sb, &tm_alr, c * 64, row0, fb);
           tma_load_2d_pair(sb + G_A_BYTES, &tm_blr, c * 64, brow0, fb);
-          issued = it + 1;
         }
+        __syncwarp();
+        issued = it + 1;
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------- MMA issuer (leader only) ----
-    if (leader && lane == 0) {
+    // -------------------------------------- MMA issuer (leader, warp) ----
+    if (leader) {
       const uint32_t id_fp4 = idesc_nvfp4(2 * G_BM, G_BN);
       const uint32_t id_lr = idesc_bf16(2 * G_BM, G_BN);
       int it = 0, tcount = 0;
@@ -215,19 +221,20 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       for (int tile = t_begin; tile < t_end && !stop; ++tile, ++tcount) {
         // (the accumulator is free only once every MMA of the previous tile
         // has completed, so resident scales may be overwritten after this)
-        if (!mbar_wait(acc_empty, (tcount & 1) ^ 1, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
+        if (!mbar_wait_warp(acc_empty, (tcount & 1) ^ 1, p.timeout_ns, abort_flag, (2u << 8) | kid))
+          break;
         tc_fence_after();
         const bool load_sfa = !sfa_res || tile == t_begin || tile % num_n == 0;
         uint32_t accumulate = 0;
         for (int kb = 0; kb < kb_total; ++kb, ++it) {
           const int st = it % G_STAGES;
           const uint32_t ph = (it / G_STAGES) & 1;
-          if (!mbar_wait(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) {
+          // the stage's TMA bytes have landed (complete_tx); the MMAs and
+          // scale copies below read them through the async proxy
+          if (!mbar_wait_warp(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) {
             stop = true;
             break;
           }
-          tc_fence_after();
-          const int nk = min(4, k64 - 4 * kb);
           const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
           const uint32_t sfa_s = sb + G_A_BYTES + G_B_BYTES;
           const uint32_t sfb_s = sfa_s + G_SFA_BYTES;
@@ -235,38 +242,55 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                                          : tmem + G_SF_TMEM + (it & 1) * G_SF_TMEM_STRIDE;
           const uint32_t sfb_t = sfa_res ? tmem + G_SFB_RES_TMEM + (it & 1) * G_SFB_RES_STRIDE
                                          : sfa_t + 16;
-          for (int kk = 0; kk < nk; ++kk) {
-            if (load_sfa)
-              tmem_copy_32x128b_x4_pair(sfa_t + 4 * kk, sdesc_sf_block(sfa_s + 512 * kk));
-            tmem_copy_32x128b_x4_pair(sfb_t + 8 * kk, sdesc_sf_block(sfb_s + 512 * kk));
-            tmem_copy_32x128b_x4_pair(sfb_t + 8 * kk + 4, sdesc_sf_block(sfb_s + 2048 + 512 * kk));
+          // Every stage runs all four 64-deep steps, fixed and fully
+          // unrolled: a loop bounded at run time (or a per-step guard) around
+          // elect.sync here cut the issue rate by up to half.  A short last
+          // stage (K % 256 != 0) reads zero codes past K (TMA fill) against
+          // finite scales, which adds exactly zero.
+          if (elect_one()) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              if (load_sfa)
+                tmem_copy_32x128b_x4_pair(sfa_t + 4 * kk, sdesc_sf_block(sfa_s + 512 * kk));
+              tmem_copy_32x128b_x4_pair(sfb_t + 8 * kk, sdesc_sf_block(sfb_s + 512 * kk));
+              tmem_copy_32x128b_x4_pair(sfb_t + 8 * kk + 4,
+                                        sdesc_sf_block(sfb_s + 2048 + 512 * kk));
+            }
           }
+          __syncwarp();
           const uint64_t da = sdesc_sw128(sb), db = sdesc_sw128(sb + G_A_BYTES);
-          for (int kk = 0; kk < nk; ++kk) {  // K = 64 E2M1 = 32 bytes per MMA
-            mma_nvfp4_pair(tmem, da + 2 * kk, db + 2 * kk, id_fp4, sfa_t + 4 * kk,
-                           sfb_t + 8 * kk, accumulate);
-            accumulate = 1;
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // K = 64 E2M1 = 32 bytes per MMA
+            if (elect_one())
+              mma_nvfp4_pair(tmem, da + 2 * kk, db + 2 * kk, id_fp4, sfa_t + 4 * kk,
+                             sfb_t + 8 * kk, kk > 0 ? 1u : accumulate);
+            __syncwarp();
           }
-          tc_commit_pair(empty0 + 8 * st, 0x3);
+          accumulate = 1;
+          if (elect_one()) tc_commit_pair(empty0 + 8 * st, 0x3);
+          __syncwarp();
         }
         for (int c = 0; c < lr_chunks && !stop; ++c, ++it) {
           const int st = it % G_STAGES;
           const uint32_t ph = (it / G_STAGES) & 1;
-          if (!mbar_wait(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) {
+          if (!mbar_wait_warp(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) {
             stop = true;
             break;
           }
-          tc_fence_after();
           const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
           const uint64_t da = sdesc_sw128(sb), db = sdesc_sw128(sb + G_A_BYTES);
-          const int nks = min(4, (2 * r - 64 * c) >> 4);  // K = 16 bf16 per MMA
-          for (int kk = 0; kk < nks; ++kk) {
-            mma_bf16_pair(tmem, da + 2 * kk, db + 2 * kk, id_lr, accumulate);
-            accumulate = 1;
+          // four 16-deep bf16 steps; columns [2r, klr) of both operands are
+          // zeros, so a partial last chunk adds exactly zero
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            if (elect_one()) mma_bf16_pair(tmem, da + 2 * kk, db + 2 * kk, id_lr, 1u);
+            __syncwarp();
           }
-          tc_commit_pair(empty0 + 8 * st, 0x3);
+          if (elect_one()) tc_commit_pair(empty0 + 8 * st, 0x3);
+          __syncwarp();
         }
-        tc_commit_pair(acc_full, 0x3);
+        if (elect_one()) tc_commit_pair(acc_full, 0x3);
+        __syncwarp();
       }
     }
   } else {
@@ -337,9 +361,14 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       for (int i = max(0, issued - G_STAGES); i < issued; ++i)
         mbar_wait_drain(full0 + 8 * (i % G_STAGES), (i / G_STAGES) & 1, p.timeout_ns);
     }
-    if (leader && warp == 1 && lane == 0) {
-      tc_commit_pair(drain_bar, 0x1);
-      mbar_wait_drain(drain_bar, 0, p.timeout_ns);
+    if (leader && warp == 1) {
+      // the commit must come from the lane that issued the MMAs: elect.sync
+      // over the full warp picks the same lane every time
+      if (elect_one()) {
+        tc_commit_pair(drain_bar, 0x1);
+        mbar_wait_drain(drain_bar, 0, p.timeout_ns);
+      }
+      __syncwarp();
     }
     // the other CTA's loads complete on the leader's barriers; give any that
     // are still landing in this CTA's shared memory a bounded moment
