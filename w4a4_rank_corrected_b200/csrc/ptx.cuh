@@ -103,6 +103,20 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, ui
   return __all_sync(0xffffffff, ok) != 0;
 }
 
+// Non-blocking test of a phase by every lane (each lane gets its own acquire
+// when it succeeds); true only if all lanes saw it complete.
+__device__ __forceinline__ bool mbar_test_warp(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return __all_sync(0xffffffff, ok != 0) != 0;
+}
+
 // Bounded wait used on the error path only: ignores the abort flag, gives
 // up silently after `timeout_ns`.
 __device__ __forceinline__ void mbar_wait_drain(uint32_t bar, uint32_t parity,

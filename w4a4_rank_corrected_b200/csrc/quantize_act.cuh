@@ -12,11 +12,9 @@
 //     so that the whole grid is resident in one wave;
 //   * the slice's smoothing factors are loaded once (bulk copy) and stay in
 //     shared memory;
-//   * warp 0 (the whole warp waits, an elected lane issues; the same for
-//     warps 1 and 2) streams X chunks [64 x 64] bf16 into a deep ring (8 or 16
-//     stages, TMA, 128-byte swizzle): the ring holds only X, so up to 128 KB
-//     of activations per SM are in flight, which is what it takes to cover
-//     HBM latency at full bandwidth;
+//   * warp 0 streams X chunks [64 x 64] bf16 into a deep ring (6 or 12
+//     stages, TMA, 128-byte swizzle): the ring holds only X, so up to 96 KB
+//     of activations per SM are in flight;
 //   * warp 2 streams the matching chunks of the low-rank operand L1' into a
 //     separate ring of up to 8 stages (they come from L2: every row block
 //     reads the same L1', so each row block starts its K slice at a
@@ -30,7 +28,8 @@
 //     quotients, computed once per CTA), form the E2M1 codes with the
 //     hardware conversion; per row 32 code bytes and one 32-bit word of
 //     scales go straight into the MMA tile layout;
-//   * warp 1 issues tcgen05 bf16 MMAs (M = 64) on the SAME shared-memory X
+//   * warp 1 (converged: every lane waits, an elected lane issues) issues
+//     tcgen05 bf16 MMAs (M = 64) on the SAME shared-memory X
 //     tile: X [64 x 64] times L1' [2r x 64]^T into a 64 x 2r fp32 accumulator
 //     in tensor memory.  L1' holds smooth * L1 split into bf16 hi and lo
 //     halves, so X L1' = X_hat L1 to ~2^-16 relative (X itself is exact);
@@ -46,20 +45,20 @@
 namespace svdq_dev {
 
 constexpr int QA_BM = 64;
-constexpr int QA_QWARPS = 16;
+constexpr int QA_QWARPS = 12;
 constexpr int QA_QWARP0 = 3;                               // first quantize warp
 constexpr int QA_THREADS = 32 * (QA_QWARP0 + QA_QWARPS);
 constexpr uint32_t QA_X_BYTES = QA_BM * 128;               // 64 rows x 64 bf16
 // X ring depth: a multiple of QA_QWARPS / 2.  Warp w's units cover chunks
-// w / 2, w / 2 + 8, w / 2 + 16, ...; with the depth a multiple of 8, the
+// w / 2, w / 2 + 6, w / 2 + 12, ...; with the depth a multiple of 6, the
 // previous use of the stage a warp is about to wait on was that same warp's
 // own earlier chunk, which it has already seen land, so the stage's barrier
 // is never two phases behind a parity wait (which would pass at once).
 constexpr int QA_XST_STEP = QA_QWARPS / 2;
-constexpr int QA_MAX_XST = 16;
+constexpr int QA_MAX_XST = 2 * QA_XST_STEP;
 constexpr int QA_MIN_XST = QA_XST_STEP;
 constexpr int QA_MAX_LST = 8;
-static_assert(QA_MAX_XST % QA_XST_STEP == 0, "ring depth must be a multiple of 8");
+static_assert(QA_MAX_XST % QA_XST_STEP == 0, "ring depth must be a multiple of QA_QWARPS / 2");
 constexpr uint32_t QA_SMEM_BUDGET = 224 * 1024;  // + 1.5 KB: within the 227 KB per CTA
 
 // Shared-memory plan of one CTA (offsets from the 1024-aligned base).
@@ -238,48 +237,53 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
 
   int x_issued = 0, l_issued = 0;  // producers: chunks whose loads were issued
   if (warp == 0) {
-    // ------------------------------------------- X producer (TMA, warp) ----
-    if (nchunks > 0) {
-      if (elect_one()) {
+    // ------------------------------------------------ X producer (TMA) ----
+    // One lane runs the loop (its warp shares an SM sub-partition with busy
+    // quantize warps, so the fewer instructions per load the better); the
+    // rest of the warp waits at the __syncwarp below.
+    if (lane == 0) {
+      if (nchunks > 0) {
         mbar_arrive_expect_tx(s_bar, 256u * (uint32_t)nchunks);
         bulk_load(smem_u32(smem + L.s_off), p.smooth + c_begin * 64, 256u * (uint32_t)nchunks,
                   s_bar);
       }
-      __syncwarp();
-    }
-    int st = 0;
-    uint32_t ph = 0;
-    for (int i = 0; i < nchunks; ++i) {
-      if (!mbar_wait_warp(x_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) break;
-      if (elect_one()) {
-        const int cl = i + rot < nchunks ? i + rot : i + rot - nchunks;  // local chunk
+      int st = 0;
+      uint32_t ph = 0;
+      int cl = rot;  // local chunk of load i: (i + rot) mod nchunks
+      for (int i = 0; i < nchunks; ++i) {
+        // every stage starts free: the first XST loads go out back to back
+        // (a satisfied try_wait still costs a round trip per load)
+        if (i >= XST &&
+            !mbar_wait(x_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid))
+          break;
         mbar_arrive_expect_tx(x_full0 + 8 * st, QA_X_BYTES);
         tma_load_2d(smem_u32(smem + st * QA_X_BYTES), &tm_x, (c_begin + cl) * 64, rb * QA_BM,
                     x_full0 + 8 * st);
+        x_issued = i + 1;
+        if (++st == XST) { st = 0; ph ^= 1; }
+        if (++cl == nchunks) cl = 0;
       }
-      __syncwarp();
-      x_issued = i + 1;
-      if (++st == XST) { st = 0; ph ^= 1; }
     }
+    __syncwarp();
   } else if (warp == 2) {
-    // ----------------------------- low-rank operand producer (TMA, warp) ----
-    if (has_lr) {
+    // ---------------------------------- low-rank operand producer (TMA) ----
+    if (has_lr && lane == 0) {
       int st = 0;
       uint32_t ph = 0;
+      int cl = rot;
       for (int i = 0; i < nchunks; ++i) {
-        if (!mbar_wait_warp(l_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (5u << 8) | kid))
+        if (i >= LST &&
+            !mbar_wait(l_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (5u << 8) | kid))
           break;
-        if (elect_one()) {
-          const int cl = i + rot < nchunks ? i + rot : i + rot - nchunks;
-          mbar_arrive_expect_tx(l_full0 + 8 * st, L.l1_bytes);
-          tma_load_2d(smem_u32(smem + L.l1_off + st * L.l1_bytes), &tm_l1, (c_begin + cl) * 64, 0,
-                      l_full0 + 8 * st);
-        }
-        __syncwarp();
+        mbar_arrive_expect_tx(l_full0 + 8 * st, L.l1_bytes);
+        tma_load_2d(smem_u32(smem + L.l1_off + st * L.l1_bytes), &tm_l1, (c_begin + cl) * 64, 0,
+                    l_full0 + 8 * st);
         l_issued = i + 1;
         if (++st == LST) { st = 0; ph ^= 1; }
+        if (++cl == nchunks) cl = 0;
       }
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------ down-projection (warp) ----
     if (has_lr) {

@@ -218,6 +218,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       const uint32_t id_lr = idesc_bf16(2 * G_BM, G_BN);
       int it = 0, tcount = 0;
       bool stop = false;
+      // `ready`: the stage `it` was already seen full by a non-blocking test
+      // made right after the previous stage was issued (its latency then
+      // overlaps the tensor-core work instead of preceding the next issue)
+      bool ready = false;
       for (int tile = t_begin; tile < t_end && !stop; ++tile, ++tcount) {
         // (the accumulator is free only once every MMA of the previous tile
         // has completed, so resident scales may be overwritten after this)
@@ -231,7 +235,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           const uint32_t ph = (it / G_STAGES) & 1;
           // the stage's TMA bytes have landed (complete_tx); the MMAs and
           // scale copies below read them through the async proxy
-          if (!mbar_wait_warp(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) {
+          if (!ready &&
+              !mbar_wait_warp(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) {
             stop = true;
             break;
           }
@@ -267,13 +272,15 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             __syncwarp();
           }
           accumulate = 1;
+          ready = mbar_test_warp(full0 + 8 * ((it + 1) % G_STAGES), ((it + 1) / G_STAGES) & 1);
           if (elect_one()) tc_commit_pair(empty0 + 8 * st, 0x3);
           __syncwarp();
         }
         for (int c = 0; c < lr_chunks && !stop; ++c, ++it) {
           const int st = it % G_STAGES;
           const uint32_t ph = (it / G_STAGES) & 1;
-          if (!mbar_wait_warp(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) {
+          if (!ready &&
+              !mbar_wait_warp(full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) {
             stop = true;
             break;
           }
@@ -286,6 +293,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             if (elect_one()) mma_bf16_pair(tmem, da + 2 * kk, db + 2 * kk, id_lr, 1u);
             __syncwarp();
           }
+          ready = mbar_test_warp(full0 + 8 * ((it + 1) % G_STAGES), ((it + 1) / G_STAGES) & 1);
           if (elect_one()) tc_commit_pair(empty0 + 8 * st, 0x3);
           __syncwarp();
         }
