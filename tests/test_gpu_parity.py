@@ -217,3 +217,26 @@ def test_mlp_pair_parity():
     check_output(from_dev_bf16(Y1)[rows], Y1r)
     Y2r, _, _, _ = O.linear_reference(Hb, op2, fc2.bias_bf16, rows=rows)
     check_output(from_dev_bf16(Y2)[rows], Y2r)
+
+
+def test_host_streamer_matches_forward():
+    """The overlapped host-buffer path (three streams, two buffer sets) gives
+    the device forward's output bit for bit, batch after batch."""
+    S = _S()
+    M, K, N, r = 300, 512, 384, 32
+    X0, W, b = SI.random_layer(91, M, K, N)
+    lp, op, dw = prepare(W, SI.channel_absmax(X0), r, b)
+    hs = S.HostStreamer(dw, M, "cuda")
+    outs, refs = [], []
+    for i in range(4):
+        X, _, _ = SI.random_layer(200 + i, M, K, N)
+        Xh = torch.from_numpy(X.view(np.int16)).view(torch.bfloat16).pin_memory()
+        Yh = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        hs.submit(Xh, Yh)
+        outs.append((Xh, Yh))
+        refs.append(from_dev_bf16(S.svdq_linear_forward(dw, to_dev_bf16(X))))
+    hs.synchronize()
+    torch.cuda.synchronize()
+    for (Xh, Yh), ref in zip(outs, refs):
+        got = Yh.view(torch.int16).numpy().view(np.uint16)
+        assert np.array_equal(got, ref)

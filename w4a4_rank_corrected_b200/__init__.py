@@ -322,6 +322,50 @@ def svdq_linear_forward_host(w: DeviceWeight, X_host, Y_host, X_dev, Y_dev, work
     return Y_host
 
 
+class HostStreamer:
+    """The forward over a sequence of host batches (pinned X in, pinned Y
+    out), with the upload of batch i+1, the two kernels of batch i and the
+    download of batch i-1 overlapped: three streams and two device buffer
+    sets.  submit() only enqueues; synchronize() waits for all of it."""
+
+    def __init__(self, w: DeviceWeight, M: int, device="cuda"):
+        import torch
+        self.w, self.M = w, M
+        self.X = [torch.empty((M, w.K), dtype=torch.bfloat16, device=device) for _ in range(2)]
+        self.Y = [torch.empty((M, w.N), dtype=torch.bfloat16, device=device) for _ in range(2)]
+        self.ws = torch.empty(max(svdq_act_workspace_bytes(M, w.K, w.r), 256), dtype=torch.uint8,
+                              device=device)
+        self.up, self.run, self.down = (torch.cuda.Stream(device=device) for _ in range(3))
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]
+        self.uploaded, self.computed, self.downloaded = ev(), ev(), ev()
+        self.n = 0
+
+    def submit(self, X_host, Y_host):
+        b = self.n & 1
+        if self.n >= 2:                       # buffer set b was used by batch n-2
+            self.up.wait_event(self.computed[b])
+            self.run.wait_event(self.downloaded[b])
+        with torch_stream(self.up):
+            self.X[b].copy_(X_host, non_blocking=True)
+        self.uploaded[b].record(self.up)
+        self.run.wait_event(self.uploaded[b])
+        svdq_linear_forward(self.w, self.X[b], self.Y[b], self.ws, self.run)
+        self.computed[b].record(self.run)
+        self.down.wait_event(self.computed[b])
+        with torch_stream(self.down):
+            Y_host.copy_(self.Y[b], non_blocking=True)
+        self.downloaded[b].record(self.down)
+        self.n += 1
+
+    def synchronize(self):
+        self.down.synchronize()
+
+
+def torch_stream(s):
+    import torch
+    return torch.cuda.stream(s)
+
+
 def svdq_device_error(stream=None) -> int:
     code = ctypes.c_int(0)
     st = lib.svdq_device_error(_stream_ptr(stream), ctypes.byref(code))

@@ -12,15 +12,17 @@
 //     so that the whole grid is resident in one wave;
 //   * the slice's smoothing factors are loaded once (bulk copy) and stay in
 //     shared memory;
-//   * warp 0 streams X chunks [64 x 64] bf16 into a deep ring (6 or 12
-//     stages, TMA, 128-byte swizzle): the ring holds only X, so up to 96 KB
-//     of activations per SM are in flight;
+//   * warp 0 streams X chunks [64 rows x 128 columns] bf16, as two 64 x 64
+//     boxes (TMA, 128-byte swizzle) under one barrier pair, into a ring of 3
+//     or 6 stages: the ring holds only X, so up to 96 KB of activations per
+//     SM are in flight;
 //   * warp 2 streams the matching chunks of the low-rank operand L1' into a
 //     separate ring of up to 8 stages (they come from L2: every row block
 //     reads the same L1', so each row block starts its K slice at a
 //     different chunk to spread those reads);
-//   * QA_QWARPS quantize warps: unit u = (chunk u / 2, rows 32 (u % 2) ..
-//     + 31) goes to warp u % QA_QWARPS; lane l handles one row.  A warp copies
+//   * QA_QWARPS quantize warps: unit u = (chunk u / 4, box (u % 4) / 2,
+//     rows 32 (u % 2) .. + 31) goes to warp u % QA_QWARPS; lane l handles one
+//     row.  A warp copies
 //     its row segment (128 bytes per lane) into registers, hands the X stage
 //     back, then quantizes: per 16-group multiply by the smoothing factors,
 //     take the maximum, form the E4M3 block scale with one multiply and the
@@ -48,36 +50,44 @@ constexpr int QA_BM = 64;
 constexpr int QA_QWARPS = 12;
 constexpr int QA_QWARP0 = 3;                               // first quantize warp
 constexpr int QA_THREADS = 32 * (QA_QWARP0 + QA_QWARPS);
-constexpr uint32_t QA_X_BYTES = QA_BM * 128;               // 64 rows x 64 bf16
-// X ring depth: a multiple of QA_QWARPS / 2.  Warp w's units cover chunks
-// w / 2, w / 2 + 6, w / 2 + 12, ...; with the depth a multiple of 6, the
+// A chunk is 128 columns of the slice: two 64-column TMA boxes (128-byte
+// swizzle rows) that share one barrier pair, so each barrier round trip of
+// the producer moves 16 KB of X.
+constexpr int QA_BOXES = 2;
+constexpr uint32_t QA_BOX_BYTES = QA_BM * 128;             // 64 rows x 64 bf16
+constexpr uint32_t QA_X_BYTES = QA_BOXES * QA_BOX_BYTES;   // one X stage
+// X ring depth: a multiple of QA_QWARPS / 4.  A chunk has 4 units (two row
+// halves x two boxes); warp w's units cover chunks w / 4, w / 4 + 3,
+// w / 4 + 6, ...; with the depth a multiple of 3, the
 // previous use of the stage a warp is about to wait on was that same warp's
 // own earlier chunk, which it has already seen land, so the stage's barrier
 // is never two phases behind a parity wait (which would pass at once).
-constexpr int QA_XST_STEP = QA_QWARPS / 2;
+constexpr int QA_UNITS = 2 * QA_BOXES;                     // units per chunk
+constexpr int QA_XST_STEP = QA_QWARPS / QA_UNITS;
 constexpr int QA_MAX_XST = 2 * QA_XST_STEP;
 constexpr int QA_MIN_XST = QA_XST_STEP;
 constexpr int QA_MAX_LST = 8;
-static_assert(QA_MAX_XST % QA_XST_STEP == 0, "ring depth must be a multiple of QA_QWARPS / 2");
+static_assert(QA_QWARPS % QA_UNITS == 0 && QA_MAX_XST % QA_XST_STEP == 0,
+              "ring depth must be a multiple of the chunk stride of a warp's units");
 constexpr uint32_t QA_SMEM_BUDGET = 224 * 1024;  // + 1.5 KB: within the 227 KB per CTA
 
 // Shared-memory plan of one CTA (offsets from the 1024-aligned base).
 struct QALayout {
   int xst, lst;              // ring depths (X, low-rank operand)
-  uint32_t l1_bytes;         // one low-rank stage: 2r rows x 128 bytes
+  uint32_t l1_bytes;         // one low-rank stage: two boxes of 2r rows x 128 bytes
   uint32_t l1_off, s_off, red_off, lut_off, bar_off;
   uint32_t total;            // bytes to request (incl. alignment slack)
 };
 
 __host__ __device__ inline QALayout qa_layout(int r, int chunks_per_split, int num_splits) {
   QALayout L;
-  L.l1_bytes = 256u * (uint32_t)r;
-  const uint32_t s_bytes = 256u * (uint32_t)chunks_per_split;
+  L.l1_bytes = (uint32_t)QA_BOXES * 256u * (uint32_t)r;
+  const uint32_t s_bytes = (uint32_t)QA_BOXES * 256u * (uint32_t)chunks_per_split;
   const uint32_t red_bytes =
       (r > 0 && num_splits > 1) ? (uint32_t)(num_splits - 1) * QA_BM * (uint32_t)r * 4u : 0u;
   const uint32_t fixed = s_bytes + red_bytes + 512u + 512u;
-  // X ring 16 deep if the low-rank ring still gets 2 stages, else 8; the
-  // low-rank ring takes what is left, up to 8 stages
+  // the deeper X ring if the low-rank ring still gets a stage, else the
+  // shallower one; the low-rank ring takes what is left, up to 8 stages
   L.xst = 0;
   L.lst = 0;
   for (int xst = QA_MAX_XST; xst >= QA_MIN_XST; xst -= QA_XST_STEP) {
@@ -87,7 +97,7 @@ __host__ __device__ inline QALayout qa_layout(int r, int chunks_per_split, int n
     if (r > 0) {
       lst = (int)((QA_SMEM_BUDGET - used) / L.l1_bytes);
       lst = lst > QA_MAX_LST ? QA_MAX_LST : lst;
-      if (lst < 2) continue;
+      if (lst < 1) continue;
     }
     L.xst = xst;
     L.lst = lst;
@@ -182,7 +192,7 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   const int rb = blockIdx.y;
   const int S = p.num_splits;
   const bool reduce = has_lr && S > 1;
-  const int kchunks = p.K >> 6;
+  const int kchunks = ((p.K >> 6) + QA_BOXES - 1) / QA_BOXES;   // 128-column chunks
   const int c_begin = split * p.chunks_per_split;
   const int c_end = min(kchunks, c_begin + p.chunks_per_split);
   const int nchunks = max(0, c_end - c_begin);
@@ -194,7 +204,7 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < XST; ++i) {
       mbar_init(x_full0 + 8 * i, 1);
-      mbar_init(x_empty0 + 8 * i, 2 + (has_lr ? 1 : 0));  // two row halves + the MMA
+      mbar_init(x_empty0 + 8 * i, QA_UNITS + (has_lr ? 1 : 0));  // its 4 units + the MMA
     }
     for (int i = 0; i < LST; ++i) {
       mbar_init(l_full0 + 8 * i, 1);
@@ -243,9 +253,9 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
     // rest of the warp waits at the __syncwarp below.
     if (lane == 0) {
       if (nchunks > 0) {
-        mbar_arrive_expect_tx(s_bar, 256u * (uint32_t)nchunks);
-        bulk_load(smem_u32(smem + L.s_off), p.smooth + c_begin * 64, 256u * (uint32_t)nchunks,
-                  s_bar);
+        const int ncols = min(p.K - c_begin * 128, nchunks * 128);  // a multiple of 64
+        mbar_arrive_expect_tx(s_bar, 4u * (uint32_t)ncols);
+        bulk_load(smem_u32(smem + L.s_off), p.smooth + c_begin * 128, 4u * (uint32_t)ncols, s_bar);
       }
       int st = 0;
       uint32_t ph = 0;
@@ -257,8 +267,10 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
             !mbar_wait(x_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid))
           break;
         mbar_arrive_expect_tx(x_full0 + 8 * st, QA_X_BYTES);
-        tma_load_2d(smem_u32(smem + st * QA_X_BYTES), &tm_x, (c_begin + cl) * 64, rb * QA_BM,
-                    x_full0 + 8 * st);
+        // (a box past K reads zeros: the TMA fill)
+        for (int b = 0; b < QA_BOXES; ++b)
+          tma_load_2d(smem_u32(smem + st * QA_X_BYTES + b * QA_BOX_BYTES), &tm_x,
+                      (c_begin + cl) * 128 + 64 * b, rb * QA_BM, x_full0 + 8 * st);
         x_issued = i + 1;
         if (++st == XST) { st = 0; ph ^= 1; }
         if (++cl == nchunks) cl = 0;
@@ -276,8 +288,9 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
             !mbar_wait(l_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (5u << 8) | kid))
           break;
         mbar_arrive_expect_tx(l_full0 + 8 * st, L.l1_bytes);
-        tma_load_2d(smem_u32(smem + L.l1_off + st * L.l1_bytes), &tm_l1, (c_begin + cl) * 64, 0,
-                    l_full0 + 8 * st);
+        for (int b = 0; b < QA_BOXES; ++b)
+          tma_load_2d(smem_u32(smem + L.l1_off + st * L.l1_bytes + b * (L.l1_bytes / QA_BOXES)),
+                      &tm_l1, (c_begin + cl) * 128 + 64 * b, 0, l_full0 + 8 * st);
         l_issued = i + 1;
         if (++st == LST) { st = 0; ph ^= 1; }
         if (++cl == nchunks) cl = 0;
@@ -295,12 +308,17 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
         // the async proxy
         if (!mbar_wait_warp(x_full0 + 8 * xs, xph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
         if (!mbar_wait_warp(l_full0 + 8 * ls, lph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
-        const uint64_t da = sdesc_sw128(smem_u32(smem + xs * QA_X_BYTES));
-        const uint64_t db = sdesc_sw128(smem_u32(smem + L.l1_off + ls * L.l1_bytes));
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {  // K = 16 bf16 = 32 bytes per MMA
-          if (elect_one()) mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (i | kk) != 0 ? 1u : 0u);
-          __syncwarp();
+        for (int b = 0; b < QA_BOXES; ++b) {
+          const uint64_t da = sdesc_sw128(smem_u32(smem + xs * QA_X_BYTES + b * QA_BOX_BYTES));
+          const uint64_t db =
+              sdesc_sw128(smem_u32(smem + L.l1_off + ls * L.l1_bytes + b * (L.l1_bytes / QA_BOXES)));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {  // K = 16 bf16 = 32 bytes per MMA
+            if (elect_one())
+              mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (i | b | kk) != 0 ? 1u : 0u);
+            __syncwarp();
+          }
         }
         if (elect_one()) {
           tc_commit(x_empty0 + 8 * xs);
@@ -318,15 +336,17 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
     const int qw = warp - QA_QWARP0;
     const float gs = p.gs_x;
     bool ok = nchunks == 0 || mbar_wait_warp(s_bar, 0, p.timeout_ns, abort_flag, (3u << 8) | kid);
-    for (int u = qw; ok && u < 2 * nchunks; u += QA_QWARPS) {
-      const int i = u >> 1;
+    for (int u = qw; ok && u < QA_UNITS * nchunks; u += QA_QWARPS) {
+      const int i = u / QA_UNITS;
+      const int box = (u % QA_UNITS) >> 1;
       const int cl = i + rot < nchunks ? i + rot : i + rot - nchunks;  // local chunk
       const int st = i % XST;
       const uint32_t ph = (uint32_t)(i / XST) & 1u;
       if (!mbar_wait_warp(x_full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) break;
       const int row_t = 32 * (u & 1) + lane;
       const int row = rb * QA_BM + row_t;
-      const uint8_t* xrow = smem + st * QA_X_BYTES + row_t * 128;
+      const int col0 = (c_begin + cl) * 128 + 64 * box;   // first column of the unit
+      const uint8_t* xrow = smem + st * QA_X_BYTES + box * QA_BOX_BYTES + row_t * 128;
       // copy this lane's row segment into registers, then hand the stage
       // back so the next chunk can land while this one is quantized
       uint4 xr[8];
@@ -335,7 +355,8 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
         xr[j] = *reinterpret_cast<const uint4*>(xrow + ((j ^ (row_t & 7)) << 4));
       __syncwarp();
       if (lane == 0) mbar_arrive(x_empty0 + 8 * st);
-      const float4* sp = reinterpret_cast<const float4*>(s_sm + cl * 64);
+      if (col0 >= p.K) continue;  // the zero box past K: nothing to store
+      const float4* sp = reinterpret_cast<const float4*>(s_sm + cl * 128 + 64 * box);
       uint32_t cw[8];
       uint32_t sfw = 0;
 #pragma unroll
@@ -377,12 +398,11 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
         sfw |= code << (8 * g);
       }
       if (row < p.M) {
-        uint4* dst = reinterpret_cast<uint4*>(p.codes_x + (size_t)row * (p.K >> 1) +
-                                              (size_t)(c_begin + cl) * 32);
+        uint4* dst = reinterpret_cast<uint4*>(p.codes_x + (size_t)row * (p.K >> 1) + (col0 >> 1));
         dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
         dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
       }
-      *reinterpret_cast<uint32_t*>(p.sf_x + sf_tile_off(row, 4 * (c_begin + cl), p.K)) = sfw;
+      *reinterpret_cast<uint32_t*>(p.sf_x + sf_tile_off(row, col0 >> 4, p.K)) = sfw;
     }
   }
 

@@ -209,7 +209,7 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
   // 64-row tiles covering whole 128-row scale atoms (padding rows get zero
   // scales)
   const int tiles = 2 * ((M + 127) / 128);
-  const int KC = K / 64;
+  const int KC = (K / 64 + QA_BOXES - 1) / QA_BOXES;  // 128-column chunks
   int S = choose_splits(tiles, KC, r, sms);
   const int cps = (KC + S - 1) / S;
   S = (KC + cps - 1) / cps;
