@@ -169,6 +169,23 @@ def test_forward_is_deterministic():
     assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
 
 
+def test_activation_kernel_repeats_bit_identical():
+    """Twenty launches of the activation kernel at the Flux shape give the same
+    codes, scales and low-rank operand bit for bit: guards the hand-back of
+    ring stages (generic reads, then a TMA refill) against reordering races,
+    which showed up as one unit of wrong codes in a few percent of launches."""
+    S = _S()
+    M, K, N, r = 4608, 3072, 1024, 32
+    X, W, b = SI.random_layer(24, M, K, N)
+    lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
+    Xd = to_dev_bf16(X)
+    c0, s0, x0 = (t.clone() for t in S.svdq_quantize_act(dw, Xd))
+    for _ in range(20):
+        c, sf, xl1 = S.svdq_quantize_act(dw, Xd)
+        assert torch.equal(c, c0) and torch.equal(sf, s0)
+        assert torch.equal(xl1.view(torch.int16), x0.view(torch.int16))
+
+
 # ---------------------------------------------------- full-size workloads ----
 
 def _workload_layer(name, M=None):

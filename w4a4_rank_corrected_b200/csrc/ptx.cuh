@@ -56,6 +56,17 @@ __device__ __forceinline__ void mbar_fence_init() {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
+// Orders this thread's generic-proxy shared-memory accesses before later
+// async-proxy operations (TMA, tcgen05) on the same bytes.
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// mbar_arrive that cannot be issued before `dep` is available (the operand
+// is not used by the instruction: it only orders the arrive after whatever
+// produced it).
+__device__ __forceinline__ void mbar_arrive_after(uint32_t bar, uint32_t dep) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar), "r"(dep) : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
                : "memory");
@@ -412,6 +423,29 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t code) {
   if (e == 0) return (float)m * 0.001953125f;
   return __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
+// Two fp32 lanes in one 64-bit register (element 0 in the low half).
+__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+// Lane-wise IEEE round-to-nearest products of two fp32 pairs (the same
+// result per lane as __fmul_rn).
+__device__ __forceinline__ uint64_t fmul_f32x2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// The bf16 pair in a 32-bit word as an fp32 pair (exact).
+__device__ __forceinline__ uint64_t bf16x2_to_f32x2(uint32_t w) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+  return r;
+}
+
 __device__ __forceinline__ float bf16_lo_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi_f32(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 

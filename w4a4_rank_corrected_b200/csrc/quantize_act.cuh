@@ -353,45 +353,57 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
 #pragma unroll
       for (int j = 0; j < 8; ++j)
         xr[j] = *reinterpret_cast<const uint4*>(xrow + ((j ^ (row_t & 7)) << 4));
+      // Hand the stage back only after the reads are done and ordered before
+      // the next fill.  The fill is a TMA write (async proxy) after these
+      // generic-proxy reads of the same bytes: each lane folds its loaded
+      // words into one value (its loads have landed), the warp reduces those,
+      // every lane fences the generic proxy against the async proxy, and
+      // lane 0 releases.  Without the proxy fence an occasional refill
+      // overwrote a stage while a warp's reads of it were still being served
+      // (a few percent of launches had one unit wrong).
+      uint32_t dep = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) dep ^= xr[j].x ^ xr[j].y ^ xr[j].z ^ xr[j].w;
+      dep = __reduce_or_sync(0xffffffffu, dep);
+      fence_proxy_async_shared();
       __syncwarp();
-      if (lane == 0) mbar_arrive(x_empty0 + 8 * st);
+      if (lane == 0) mbar_arrive_after(x_empty0 + 8 * st, dep);
       if (col0 >= p.K) continue;  // the zero box past K: nothing to store
       const float4* sp = reinterpret_cast<const float4*>(s_sm + cl * 128 + 64 * box);
       uint32_t cw[8];
       uint32_t sfw = 0;
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
+        // 16 products x * s as 8 lane-pairs (one f32x2 multiply each)
         const uint4 x0 = xr[2 * g], x1 = xr[2 * g + 1];
-        const float4 s0 = sp[4 * g], s1 = sp[4 * g + 1], s2 = sp[4 * g + 2], s3 = sp[4 * g + 3];
-        float v[16];
-        v[0] = __fmul_rn(bf16_lo_f32(x0.x), s0.x);
-        v[1] = __fmul_rn(bf16_hi_f32(x0.x), s0.y);
-        v[2] = __fmul_rn(bf16_lo_f32(x0.y), s0.z);
-        v[3] = __fmul_rn(bf16_hi_f32(x0.y), s0.w);
-        v[4] = __fmul_rn(bf16_lo_f32(x0.z), s1.x);
-        v[5] = __fmul_rn(bf16_hi_f32(x0.z), s1.y);
-        v[6] = __fmul_rn(bf16_lo_f32(x0.w), s1.z);
-        v[7] = __fmul_rn(bf16_hi_f32(x0.w), s1.w);
-        v[8] = __fmul_rn(bf16_lo_f32(x1.x), s2.x);
-        v[9] = __fmul_rn(bf16_hi_f32(x1.x), s2.y);
-        v[10] = __fmul_rn(bf16_lo_f32(x1.y), s2.z);
-        v[11] = __fmul_rn(bf16_hi_f32(x1.y), s2.w);
-        v[12] = __fmul_rn(bf16_lo_f32(x1.z), s3.x);
-        v[13] = __fmul_rn(bf16_hi_f32(x1.z), s3.y);
-        v[14] = __fmul_rn(bf16_lo_f32(x1.w), s3.z);
-        v[15] = __fmul_rn(bf16_hi_f32(x1.w), s3.w);
-        float m0 = fmaxf(fabsf(v[0]), fabsf(v[1])), m1 = fmaxf(fabsf(v[2]), fabsf(v[3]));
-        float m2 = fmaxf(fabsf(v[4]), fabsf(v[5])), m3 = fmaxf(fabsf(v[6]), fabsf(v[7]));
-        float m4 = fmaxf(fabsf(v[8]), fabsf(v[9])), m5 = fmaxf(fabsf(v[10]), fabsf(v[11]));
-        float m6 = fmaxf(fabsf(v[12]), fabsf(v[13])), m7 = fmaxf(fabsf(v[14]), fabsf(v[15]));
-        const float a = fmaxf(fmaxf(fmaxf(m0, m1), fmaxf(m2, m3)), fmaxf(fmaxf(m4, m5), fmaxf(m6, m7)));
-        const uint32_t code = cvt_e4m3x2(__fmul_rn(a, gs), 0.0f) & 0xFF;
-        const float q = qlut[code];
-        float t0[8], t1[8];
+        const ulonglong2* sp2 = reinterpret_cast<const ulonglong2*>(sp + 4 * g);
+        const ulonglong2 s0 = sp2[0], s1 = sp2[1], s2 = sp2[2], s3 = sp2[3];
+        uint64_t v[8];
+        v[0] = fmul_f32x2(bf16x2_to_f32x2(x0.x), s0.x);
+        v[1] = fmul_f32x2(bf16x2_to_f32x2(x0.y), s0.y);
+        v[2] = fmul_f32x2(bf16x2_to_f32x2(x0.z), s1.x);
+        v[3] = fmul_f32x2(bf16x2_to_f32x2(x0.w), s1.y);
+        v[4] = fmul_f32x2(bf16x2_to_f32x2(x1.x), s2.x);
+        v[5] = fmul_f32x2(bf16x2_to_f32x2(x1.y), s2.y);
+        v[6] = fmul_f32x2(bf16x2_to_f32x2(x1.z), s3.x);
+        v[7] = fmul_f32x2(bf16x2_to_f32x2(x1.w), s3.y);
+        float m[8];
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          t0[e] = __fmul_rn(v[e], q);
-          t1[e] = __fmul_rn(v[8 + e], q);
+          float lo, hi;
+          unpack_f32x2(v[e], lo, hi);
+          m[e] = fmaxf(fabsf(lo), fabsf(hi));
+        }
+        const float a = fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
+                              fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+        const uint32_t code = cvt_e4m3x2(__fmul_rn(a, gs), 0.0f) & 0xFF;
+        const float q = qlut[code];
+        const uint64_t qq = pack_f32x2(q, q);
+        float t0[8], t1[8];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          unpack_f32x2(fmul_f32x2(v[e], qq), t0[2 * e], t0[2 * e + 1]);
+          unpack_f32x2(fmul_f32x2(v[4 + e], qq), t1[2 * e], t1[2 * e + 1]);
         }
         cw[2 * g] = cvt_e2m1x8(t0);
         cw[2 * g + 1] = cvt_e2m1x8(t1);
