@@ -50,8 +50,11 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="flux_qkv")
+    ap.add_argument("--layer", type=int, default=0, help="which layer of the workload to time")
     ap.add_argument("--sets", type=int, default=4, help="rotating input/weight/output sets")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each step from a CUDA graph (small layers are launch-bound)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
     return ap.parse_args()
@@ -84,6 +87,23 @@ def rank_activations(spec, rank: int, M: int, K: int) -> np.ndarray:
         return SI.make_workload(spec.name, M=M).X_bf16
     rng = np.random.default_rng(spec.seed * 1000003 + rank)
     return SI.draw_activations(rng, M, K, spec.x_dist, spec.x_outliers, spec.x_scale)
+
+
+def layer_setup(spec, layer: int, rank: int = 0):
+    """(layer spec, W, bias, X) of layer `layer` of a workload.  Layer 0 takes
+    the workload's own input draw; a later layer (whose real input is the
+    previous layer's output) takes a seeded draw of its own shape with the
+    same value model, which is what its timing needs."""
+    wl = SI.make_workload(spec.name)
+    lt = wl.layers[layer]
+    ls = lt.spec
+    if layer == 0:
+        X0 = wl.X_bf16 if rank == 0 else rank_activations(spec, rank, ls.M, ls.K)
+    else:
+        rng = np.random.default_rng(spec.seed * 7919 + 100 * layer + rank)
+        X0 = SI.draw_activations(rng, ls.M, ls.K, spec.x_dist, min(spec.x_outliers, ls.K),
+                                 spec.x_scale)
+    return ls, lt.W, lt.bias_bf16, X0
 
 
 def load_peaks():
@@ -196,11 +216,8 @@ def run_ours(args):
     import w4a4_rank_corrected_b200 as S
 
     spec = SI.workload_specs()[args.workload]
-    ls = spec.layers[0]
+    ls, W, bias, X0 = layer_setup(spec, args.layer, rank)
     M, K, N, r = ls.M, ls.K, ls.N, ls.r
-    wl = SI.make_workload(spec.name)
-    W, bias = wl.layers[0].W, wl.layers[0].bias_bf16
-    X0 = wl.X_bf16 if rank == 0 else rank_activations(spec, rank, M, K)
     cx = SI.channel_absmax(X0)
     packed = S.svdq_pack_weight(W, cx, r)
 
@@ -231,23 +248,45 @@ def run_ours(args):
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
 
+    # With --graph each step (activation kernel + GEMM, the two launches of
+    # svdq_linear_forward) is captured once per buffer set into a CUDA graph
+    # and replayed, so the timed loop measures the GPU rather than per-call
+    # host work (TMA descriptor encoding, Python marshalling), which
+    # dominates at small M.  By default the launches are issued one by one
+    # (at large M they overlap through programmatic dependent launch).
+    graphs, qgraphs, ggraphs = None, None, None
+    if args.graph:
+        try:
+            graphs, qgraphs, ggraphs = [], [], []
+            for j in range(nsets):
+                for lst, what in ((graphs, "both"), (qgraphs, "q"), (ggraphs, "g")):
+                    g = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(g):
+                        if what in ("both", "q"):
+                            S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j])
+                        if what in ("both", "g"):
+                            S.svdq_gemm(weights[j], codes[j], sfs[j], xl1s[j], M, Ys[j])
+                    lst.append(g)
+            for j in range(nsets):
+                graphs[j].replay()
+            torch.cuda.synchronize(dev)
+        except Exception as ex:  # capture not available: time the launches directly
+            print(f"graph capture failed ({type(ex).__name__}: {ex}); timing direct launches",
+                  file=sys.stderr)
+            graphs = qgraphs = ggraphs = None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+
     K_steps = args.steps
-    stride = max(1, K_steps // 1000)
     ev_start = torch.cuda.Event(enable_timing=True)
     ev_end = torch.cuda.Event(enable_timing=True)
-    marks = []
     ev_start.record(stream)
-    for i in range(K_steps):
-        if i % stride == 0:
-            e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-            j = i % nsets
-            e0.record(stream)
-            S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j], stream)
-            e1.record(stream)
-            S.svdq_gemm(weights[j], codes[j], sfs[j], xl1s[j], M, Ys[j], stream)
-            e2.record(stream)
-            marks.append((e0, e1, e2))
-        else:
+    if graphs is not None:
+        for i in range(K_steps):
+            graphs[i % nsets].replay()
+    else:
+        for i in range(K_steps):
             step(i)
     ev_end.record(stream)
     torch.cuda.synchronize(dev)
@@ -260,8 +299,27 @@ def run_ours(args):
     if err:
         raise SystemExit(f"device error code {err:#x}")
 
-    q_ms = statistics.mean(a.elapsed_time(b) for a, b, _ in marks)
-    g_ms = statistics.mean(b.elapsed_time(c) for _, b, c in marks)
+    # per-kernel times, after the timed region: each kernel on its own
+    # (graph replays when available), events around a batch of launches
+    def timed_batch(fn, n):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(n):
+            fn(i)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / n
+    n_per = max(8, min(1000, K_steps // 4))
+    if qgraphs is not None:
+        q_ms = timed_batch(lambda i: qgraphs[i % nsets].replay(), n_per)
+        g_ms = timed_batch(lambda i: ggraphs[i % nsets].replay(), n_per)
+    else:
+        q_ms = timed_batch(lambda i: S.svdq_quantize_act(weights[i % nsets], Xs[i % nsets],
+                                                         codes[i % nsets], sfs[i % nsets],
+                                                         xl1s[i % nsets], stream), n_per)
+        g_ms = timed_batch(lambda i: S.svdq_gemm(weights[i % nsets], codes[i % nsets],
+                                                 sfs[i % nsets], xl1s[i % nsets], M,
+                                                 Ys[i % nsets], stream), n_per)
     ms_per_step = elapsed_ms / K_steps
     flops = 2.0 * M * N * K
     value = world * flops * K_steps / (elapsed_ms * 1e-3) / 1e12
@@ -281,8 +339,9 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "nvfp4",
         "data": "synthetic",
         "config": {
-            "workload": f"{spec.name}: {spec.description}", "M": M, "K": K, "N": N, "r": r,
+            "workload": f"{spec.name}: {spec.description}", "layer": ls.name, "M": M, "K": K, "N": N, "r": r,
             "global_batch": M * world, "parallelism": f"dp{world} (independent replicas, no collective)",
+            "launch": "CUDA graph replay per step" if graphs is not None else "direct launches",
             "l2": f"{nsets} rotating input/weight/output sets (~{nsets * (M * K * 2 + M * N * 2 + N * K // 2) / 1e6:.0f} MB > 126 MB L2)",
             "us_per_layer": round(ms_per_step * 1e3, 2),
             "us_quantize_act": round(q_ms * 1e3, 2), "us_gemm": round(g_ms * 1e3, 2),
@@ -404,10 +463,8 @@ def run_reference(args):
     import w4a4_rank_corrected_b200 as S  # host pack only (the oracle takes its factors)
     from oracle import svdq as O
     spec = SI.workload_specs()[args.workload]
-    ls = spec.layers[0]
+    ls, W, bias, X0 = layer_setup(spec, args.layer)
     M, K, N, r = ls.M, ls.K, ls.N, ls.r
-    wl = SI.make_workload(spec.name)
-    W, bias, X0 = wl.layers[0].W, wl.layers[0].bias_bf16, wl.X_bf16
     packed = S.svdq_pack_weight(W, SI.channel_absmax(X0), r)
     op, deq_w = _oracle_setup(W, X0, packed, r)
 
@@ -429,7 +486,7 @@ def run_reference(args):
            "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
            "impl": "reference",
-           "config": {"workload": f"{spec.name}: {spec.description}", "M": M, "K": K, "N": N,
+           "config": {"workload": f"{spec.name}: {spec.description}", "layer": ls.name, "M": M, "K": K, "N": N,
                       "r": r, "rows_per_step": rows},
            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": cores,
                             "kind": "oracle",

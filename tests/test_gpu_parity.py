@@ -236,6 +236,38 @@ def test_mlp_pair_parity():
     check_output(from_dev_bf16(Y2)[rows], Y2r)
 
 
+def test_flux_block_parity():
+    """Config 4 (M = 18432): qkv -> out on the V slice of the qkv output
+    (strided input, ldx = 9216) -> fc1 -> GELU (tanh, bf16, on the GPU) ->
+    fc2 (K = 12288).  Each layer is calibrated on, and compared with the
+    oracle fed, its actual bf16 input; codes and scales bit-exact and the
+    output within tolerance on sampled rows."""
+    S = _S()
+    wl = SI.make_workload("flux_block")
+    X = wl.X_bf16
+    qkv, out, fc1, fc2 = wl.layers
+    M, H = X.shape
+    rows = rows_sample(M, 48, seed=9)
+
+    def layer(lt, Xin_dev, Xin_bits):
+        lp, op, dw = prepare(lt.W, SI.channel_absmax(Xin_bits), lt.spec.r, lt.bias_bf16)
+        codes, sf, xl1 = S.svdq_quantize_act(dw, Xin_dev)
+        Y = S.svdq_linear_forward(dw, Xin_dev)
+        torch.cuda.synchronize()
+        check_activation(codes, sf, xl1, Xin_bits, op, M, lt.spec.K, lt.spec.r, rows=rows)
+        Yr, _, _, _ = O.linear_reference(Xin_bits, op, lt.bias_bf16, rows=rows)
+        check_output(from_dev_bf16(Y)[rows], Yr)
+        return Y
+
+    Yq = layer(qkv, to_dev_bf16(X), X)
+    V = Yq[:, 2 * H:]                       # strided view, ldx = 3 H
+    assert V.stride(0) == 3 * H
+    Yo = layer(out, V, from_dev_bf16(V))
+    Y1 = layer(fc1, Yo, from_dev_bf16(Yo))
+    G = torch.nn.functional.gelu(Y1, approximate="tanh")
+    layer(fc2, G, from_dev_bf16(G))
+
+
 def test_host_streamer_matches_forward():
     """The overlapped host-buffer path (three streams, two buffer sets) gives
     the device forward's output bit for bit, batch after batch."""
