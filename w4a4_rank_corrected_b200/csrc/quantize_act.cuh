@@ -13,8 +13,8 @@
 //   * the slice's smoothing factors are loaded once (bulk copy) and stay in
 //     shared memory;
 //   * warp 0 streams X chunks [64 rows x 128 columns] bf16, as two 64 x 64
-//     boxes (TMA, 128-byte swizzle) under one barrier pair, into a ring of 3
-//     or 6 stages: the ring holds only X, so up to 96 KB of activations per
+//     boxes (TMA, 128-byte swizzle) under one barrier pair, into a ring of 4
+//     or 8 stages: the ring holds only X, so up to 128 KB of activations per
 //     SM are in flight;
 //   * warp 2 streams the matching chunks of the low-rank operand L1' into a
 //     separate ring of up to 8 stages (they come from L2: every row block
@@ -47,7 +47,7 @@
 namespace svdq_dev {
 
 constexpr int QA_BM = 64;
-constexpr int QA_QWARPS = 12;
+constexpr int QA_QWARPS = 16;
 constexpr int QA_QWARP0 = 3;                               // first quantize warp
 constexpr int QA_THREADS = 32 * (QA_QWARP0 + QA_QWARPS);
 // A chunk is 128 columns of the slice: two 64-column TMA boxes (128-byte
