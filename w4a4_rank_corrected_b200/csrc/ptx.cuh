@@ -208,25 +208,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-// D(tmem) (+)= (A . SFA)(B . SFB)^T with E2M1 operands and one UE4M3 scale
-// per 16 elements along K (K = 64 per instruction).
-__device__ __forceinline__ void mma_nvfp4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], "
-      "p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-// Copy one 32-row x 16-byte block from shared memory to tensor memory,
-// replicated into all four 32-lane quarters.
-__device__ __forceinline__ void tmem_copy_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
-               : "memory");
-}
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -292,6 +273,9 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint16_t cta_mask) 
       "h"(cta_mask)
       : "memory");
 }
+// D(tmem) (+)= (A . SFA)(B . SFB)^T over the CTA pair: E2M1 operands (K = 64
+// per instruction) with one UE4M3 scale per 16 elements along K read from
+// tensor memory (block16); `accumulate` = 0 overwrites D.
 __device__ __forceinline__ void mma_nvfp4_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                                uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
                                                uint32_t accumulate) {
@@ -386,11 +370,6 @@ __device__ __forceinline__ void st_async_v4(uint32_t addr_cluster, float a, floa
           "r"(addr_cluster),
       "f"(a), "f"(b), "f"(c), "f"(d), "r"(bar_cluster)
       : "memory");
-}
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
 }
 
 // -------------------------------------------------------- conversions ----
