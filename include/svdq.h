@@ -170,7 +170,9 @@ size_t svdq_act_workspace_bytes(int M, int K, int r);
  *   codes_x  device u8 [M][K/2]
  *   sf_x     device u8, MMA tiles, round_up(M,128) * K/16 bytes (pad rows 0)
  *   xl1      device bf16 [M][klr] (may be NULL if r == 0)
- * Reads X exactly once.
+ * Reads X exactly once.  Returns SVDQ_ERR_INVALID_ARG when one CTA's share
+ * of K does not fit its shared-memory plan (for large M, where K is split at
+ * most two ways: K above roughly 36000 at r <= 32, 24000 at r = 128).
  */
 svdq_status svdq_quantize_act(const svdq_weight* w, const uint16_t* X, int M,
                               int64_t ldx, uint8_t* codes_x, uint8_t* sf_x,
