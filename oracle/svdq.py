@@ -11,7 +11,7 @@ Powers 12B Flux ..."):
      4-bit (W4A4), NVFP4 on Blackwell (hardware-support table);
   4. the forward pass is  Y = Q(X_hat) Q(R)^T + (X_hat L1) L2 (+ bias).
 
-Readings of what the pages leave open (each is also listed in the design doc):
+Readings of what the pages leave open:
   R1 smoothing: lambda_j = (cx_j / wmax_j) ** alpha with alpha = 0.5, where
      cx_j = max_m |X_mj| over the calibration batch and wmax_j =
      max_n |W_nj|; lambda_j = 1 if either maximum is 0.  The stored factor
