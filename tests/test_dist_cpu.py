@@ -59,3 +59,19 @@ def test_two_rank_timing_reduction_and_batches():
 def test_single_rank_is_identity():
     import bench
     assert bench.max_over_ranks(3.25, 1) == 3.25
+
+
+def test_layer_setup_shapes():
+    """bench --layer: every layer of every workload gets an input of its own
+    (M, K) shape, weights of (N, K), seeded (two calls agree)."""
+    import bench
+    import svdq_inputs as SI
+    for name in ("flux_mlp",):
+        spec = SI.workload_specs()[name]
+        for i, ls in enumerate(spec.layers):
+            ls2, W, b, X = bench.layer_setup(spec, i)
+            assert ls2 == ls
+            assert X.shape == (ls.M, ls.K) and X.dtype == np.uint16
+            assert W.shape == (ls.N, ls.K) and b.shape == (ls.N,)
+            _, _, _, X2 = bench.layer_setup(spec, i)
+            assert np.array_equal(X, X2)
