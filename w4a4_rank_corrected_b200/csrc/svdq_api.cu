@@ -300,7 +300,7 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
                         const uint16_t* xl1, int M, uint16_t* Y, int64_t ldy, cudaStream_t s,
                         int sms) {
   const int N = w->N, K = w->K, r = w->r, klr = klr_of(r);
-  CUtensorMap ta, tb, tsa, tsb, talr, tblr;
+  CUtensorMap ta, tb, tsa, tsb, talr, tblr, ty;
   std::memset(&talr, 0, sizeof(talr));
   std::memset(&tblr, 0, sizeof(tblr));
   // scale buffers as rows of 256 bytes (half a 512-byte atom), unswizzled
@@ -311,7 +311,10 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
       !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes_w, (uint64_t)K / 2, (uint64_t)N,
                 (uint64_t)K / 2, 128, G_BN_CTA) ||
       !make_map(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT8, sf_x, 256, sfa_rows, 256, 256, 8, false) ||
-      !make_map(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->sf_w, 256, sfb_rows, 256, 256, 8, false))
+      !make_map(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->sf_w, 256, sfb_rows, 256, 256, 8, false) ||
+      // Y is written in 128-row x 64-column boxes (128-byte swizzle)
+      !make_map(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, (uint64_t)N, (uint64_t)M,
+                (uint64_t)ldy * 2, G_OUT_COLS, G_BM))
     return SVDQ_ERR_CUDA;
   if (r > 0) {
     if (!make_map(&talr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xl1, (uint64_t)klr, (uint64_t)M,
@@ -322,8 +325,6 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   }
   GemmParams p;
   p.bias = w->bias;
-  p.Y = Y;
-  p.ldy = ldy;
   p.M = M;
   p.N = N;
   p.K = K;
@@ -347,7 +348,7 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, w4a4_gemm_kernel, ta, tb, tsa, tsb, talr, tblr, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, w4a4_gemm_kernel, ta, tb, tsa, tsb, talr, tblr, ty, p) != cudaSuccess) {
     cudaGetLastError();
     return SVDQ_ERR_CUDA;
   }

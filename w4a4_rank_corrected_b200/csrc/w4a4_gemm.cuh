@@ -35,8 +35,14 @@
 //     g_x g_w = 1/alpha); completions are multicast to both CTAs;
 //   * warps 2..9 of each CTA drain its accumulator (four 32-column
 //     tcgen05.ld, one wait), release it to the leader, and only then compute
-//     Y = bf16(alpha * acc + bias) (bias staged per tile in shared memory) and
-//     store, overlapping the next tile's main loop.
+//     Y = bf16(alpha * acc + bias) (bias staged per tile in shared memory),
+//     overlapping the next tile's main loop.  Each group of four warps owns
+//     128 columns and writes them as two 128-row x 64-column boxes through a
+//     16 KB shared-memory buffer (128-byte swizzle, so the row-per-thread
+//     writes are free of bank conflicts) that one thread stores with TMA:
+//     one bulk store per box instead of a 16-byte global store per thread
+//     and row, which scattered each warp instruction over 32 rows and held
+//     the MMA issuer back.
 #pragma once
 #include "ptx.cuh"
 
@@ -62,18 +68,22 @@ constexpr int G_SFA_RES_MAX_K64 = 48;
 constexpr uint32_t G_SFB_RES_TMEM = G_SF_TMEM + 4 * G_SFA_RES_MAX_K64;  // 448
 constexpr uint32_t G_SFB_RES_STRIDE = 32;
 constexpr uint32_t G_BIAS_BYTES = 2 * G_BN * 4;   // two fp32 bias tiles
+constexpr int G_OUT_COLS = 64;                    // columns per output box (128 bytes)
+constexpr uint32_t G_OUT_HALF_BYTES = G_BM * 128; // one box: 128 rows x 128 bytes
+constexpr uint32_t G_OUT_BYTES = 2 * G_OUT_HALF_BYTES;
 constexpr uint32_t G_FP4_TX = 2 * G_STAGE_BYTES;  // bytes per FP4 stage, both CTAs
 constexpr uint32_t G_FP4_TX_NOSFA = 2 * (G_STAGE_BYTES - G_SFA_BYTES);
 constexpr uint32_t G_LR_TX = 2 * (G_A_BYTES + G_B_BYTES);
 
 __host__ __device__ inline uint32_t gemm_smem_bytes() {
-  return 1024u + G_STAGES * G_STAGE_BYTES + G_BIAS_BYTES + 256u;  // + barriers
+  return 1024u + G_STAGES * G_STAGE_BYTES + G_OUT_BYTES + G_BIAS_BYTES + 256u;  // + barriers
 }
+static_assert(1024u + G_STAGES * G_STAGE_BYTES + G_OUT_BYTES + G_BIAS_BYTES + 256u <= 232448u,
+              "GEMM shared memory above the 227 KB a CTA may use");
+static_assert((G_STAGES * G_STAGE_BYTES) % 1024 == 0, "output boxes need 1024-byte alignment");
 
 struct GemmParams {
   const uint16_t* bias;
-  uint16_t* Y;
-  long long ldy;
   int M, N, K, r, klr;
   float alpha;
   uint64_t timeout_ns;
@@ -84,12 +94,16 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                      const __grid_constant__ CUtensorMap tm_sfa,
                      const __grid_constant__ CUtensorMap tm_sfb,
                      const __grid_constant__ CUtensorMap tm_alr,
-                     const __grid_constant__ CUtensorMap tm_blr, const GemmParams p) {
+                     const __grid_constant__ CUtensorMap tm_blr,
+                     const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  float* bias_s = reinterpret_cast<float*>(smem + G_STAGES * G_STAGE_BYTES);  // [2][256]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G_STAGES * G_STAGE_BYTES + G_BIAS_BYTES);
+  const uint32_t out_s = smem_u32(smem + G_STAGES * G_STAGE_BYTES);  // [2][128 rows][128 B]
+  float* bias_s =
+      reinterpret_cast<float*>(smem + G_STAGES * G_STAGE_BYTES + G_OUT_BYTES);  // [2][256]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G_STAGES * G_STAGE_BYTES + G_OUT_BYTES +
+                                               G_BIAS_BYTES);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * G_STAGES;
   const uint32_t acc_full = full0 + 16 * G_STAGES;
@@ -98,6 +112,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   const uint32_t bias_bar0 = acc_full + 24;  // two: one per bias buffer
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * G_STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  // per output buffer: "staged" (its 4 warps wrote it) and "free" (the
+  // store issued from it has finished reading it)
+  const uint32_t out_staged0 = smem_u32(bars + 2 * G_STAGES + 6);
+  const uint32_t out_free0 = out_staged0 + 16;
 
   const uint32_t warp = warp_id(), lane = lane_id();
   const uint32_t rank = cluster_ctarank();      // 0 = leader of the pair
@@ -129,6 +147,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     mbar_init(drain_bar, 1);
     mbar_init(bias_bar0, 32 * G_EPI_WARPS);
     mbar_init(bias_bar0 + 8, 32 * G_EPI_WARPS);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(out_staged0 + 8 * h, G_EPI_WARPS / 2);
+      mbar_init(out_free0 + 8 * h, 1);
+    }
     *abort_flag = 0;
     mbar_fence_init();
   }
@@ -137,6 +159,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     prefetch_tensormap(&tm_b);
     prefetch_tensormap(&tm_sfa);
     prefetch_tensormap(&tm_sfb);
+    prefetch_tensormap(&tm_y);
     if (has_lr) {
       prefetch_tensormap(&tm_alr);
       prefetch_tensormap(&tm_blr);
@@ -307,6 +330,12 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int half = (warp - 2) >> 2;          // columns [128 half, 128 half + 128)
     const int et = threadIdx.x - 64;           // 0..255
     const float alpha = p.alpha;
+    const int row_t = quad * 32 + lane;        // this thread's row of the CTA's 128
+    const uint32_t obuf = out_s + half * G_OUT_HALF_BYTES;
+    const uint32_t staged = out_staged0 + 8 * half, freed = out_free0 + 8 * half;
+    // one thread per group of four warps issues the group's bulk stores
+    const bool issuer = ((warp - 2) & 3) == 0 && lane == 0;
+    int use = 0;                               // boxes this group has staged
     int tcount = 0;
     for (int tile = t_begin; tile < t_end; ++tile, ++tcount) {
       const int mb = tile / num_n, nb = tile % num_n;
@@ -333,30 +362,61 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(lead_acc_empty);   // accumulator free again
-      const int row = mb * 2 * G_BM + (int)rank * G_BM + quad * 32 + lane;
-      uint16_t* yrow = p.Y + (size_t)row * p.ldy;
+      const int row0 = mb * 2 * G_BM + (int)rank * G_BM;   // first row of this CTA's box
+      bool ok = true;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        const int c0 = half * 128 + ch * 32;
-        const int n0 = nb * G_BN + c0;
-        if (row < M) {
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {      // 8 columns = one 16-byte store
-            if (n0 + 8 * v < N) {
-              uint32_t out[4];
-#pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const int c = 8 * v + 2 * j;
-                const float y0 = fmaf(alpha, __uint_as_float(acc[ch][c]), bt[c0 + c]);
-                const float y1 = fmaf(alpha, __uint_as_float(acc[ch][c + 1]), bt[c0 + c + 1]);
-                out[j] = pack_bf16x2(y0, y1);
-              }
-              *reinterpret_cast<uint4*>(yrow + n0 + 8 * v) = make_uint4(out[0], out[1], out[2], out[3]);
-            }
+      for (int sb = 0; sb < 2; ++sb, ++use) {
+        // the buffer is free once the store issued from it has read it
+        if (use > 0) {
+          if (issuer) {
+            bulk_wait_read_all();
+            mbar_arrive(freed);
+          }
+          __syncwarp();
+          if (!mbar_wait_warp(freed, (use - 1) & 1, p.timeout_ns, abort_flag, (7u << 8) | kid)) {
+            ok = false;
+            break;
           }
         }
+        // 64 columns of this thread's row: 8 chunks of 16 bytes, chunk j at
+        // slot j ^ (row % 8) of the row's 128 bytes (the 128-byte swizzle)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int ch = 2 * sb + (j >> 2);
+          const int cb = 8 * (j & 3);
+          const int c0 = half * 128 + ch * 32 + cb;
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float y0 = fmaf(alpha, __uint_as_float(acc[ch][cb + 2 * q]), bt[c0 + 2 * q]);
+            const float y1 =
+                fmaf(alpha, __uint_as_float(acc[ch][cb + 2 * q + 1]), bt[c0 + 2 * q + 1]);
+            o[q] = pack_bf16x2(y0, y1);
+          }
+          st_shared_v4(obuf + row_t * 128 + ((j ^ (row_t & 7)) << 4), o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(staged);
+        if (issuer) {
+          const int x = nb * G_BN + half * 128 + sb * G_OUT_COLS;
+          // a box wholly past N or M has nothing to write
+          if (mbar_wait(staged, use & 1, p.timeout_ns, abort_flag, (8u << 8) | kid)) {
+            if (x < N && row0 < M) {
+              tma_store_2d(&tm_y, obuf, x, row0);
+              bulk_commit_group();
+            }
+          } else {
+            ok = false;
+          }
+        }
+        ok = __all_sync(0xffffffffu, ok) != 0;   // the issuer's verdict, warp-wide
+        if (!ok) break;
       }
+      if (!ok) break;
     }
+    // no store may still be reading shared memory (or writing Y) at exit
+    if (issuer) bulk_wait_all();
   }
 
   // ------------------------------------------------------------ teardown ----
