@@ -46,6 +46,11 @@ Readings of what the pages leave open:
      scales).
   R7 packed layouts: codes are two per byte, the even k in the low nibble;
      block scales in the MMA tile layout (see `sf_to_mma_tiles`).
+  R5d dynamic per-token activation scale (an alternative to R5 for inputs
+     outside the calibration range; not the pages' path): each row m of
+     X_hat is its own tensor for R4, with A_m = max_k |x_hat_mk| taken at
+     run time; the output undoes g_x,m = fp32(2688 / A_m) row by row.  A row
+     whose x_hat is all zero has A_m = 0, so g = gs = 1 and all codes 0.
 
 Parity pins: tests/test_oracle_formats.py, tests/test_oracle_svdq.py.
 """
@@ -315,6 +320,50 @@ def linear_reference(X_bf16: np.ndarray, p: OraclePack,
     if bias_bf16 is not None:
         Y = Y + bf16_bits_to_f64(bias_bf16)[None, :]
     return Y, cx, sfx, xl1
+
+
+# --------------------------------- dynamic per-token activation scale ----
+
+def activation_absmax_rows(x_hat: np.ndarray) -> np.ndarray:
+    """Reading R5d: A_m = max_k |x_hat_mk| per row, fp32 (exact)."""
+    xh = np.asarray(x_hat, F32)
+    if xh.shape[1] == 0:
+        return np.zeros(xh.shape[0], F32)
+    return np.abs(xh).max(axis=1).astype(F32)
+
+
+def quantize_activation_dynamic(X_bf16: np.ndarray, s: np.ndarray):
+    """Reading R5d: smoothing, then R4 on each row with that row's own
+    absmax.  Returns (x_hat fp32, codes [M, K], sf [M, K/16], A fp32 [M])."""
+    xh = smooth_activation(X_bf16, s)
+    A = activation_absmax_rows(xh)
+    M, K = xh.shape
+    codes = np.zeros((M, K), np.uint8)
+    sf = np.zeros((M, K // NVFP4_GROUP), np.uint8)
+    for m in range(M):
+        codes[m:m + 1], sf[m:m + 1] = nvfp4_quantize(xh[m:m + 1], A[m])
+    return xh, codes, sf, A
+
+
+def linear_reference_dynamic(X_bf16: np.ndarray, p: OraclePack,
+                             bias_bf16: Optional[np.ndarray] = None,
+                             rows: Optional[np.ndarray] = None,
+                             deq_w: Optional[np.ndarray] = None):
+    """Reading R6 with R5d in place of R5: row m of the 4-bit product is
+    divided by g_x,m g_w.  Returns (Y_ref, codes_x, sf_x, xl1, A_rows)."""
+    X = X_bf16 if rows is None else X_bf16[rows]
+    xh, cx, sfx, A = quantize_activation_dynamic(X, p.s)
+    if deq_w is None:
+        deq_w = nvfp4_dequantize(p.codes_w, p.sf_w)
+    g_rows = np.array([tensor_encode_scale(a) for a in A], np.float64)
+    D = nvfp4_dequantize(cx, sfx) @ deq_w.T
+    Y = D / (g_rows[:, None] * np.float64(p.g_w))
+    xl1 = lowrank_down(xh, p.L1)
+    if p.L1.shape[1]:
+        Y = Y + xl1 @ bf16_bits_to_f64(p.L2)
+    if bias_bf16 is not None:
+        Y = Y + bf16_bits_to_f64(bias_bf16)[None, :]
+    return Y, cx, sfx, xl1, A
 
 
 # ------------------------------------------------------------ tolerance ----

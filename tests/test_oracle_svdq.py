@@ -155,3 +155,88 @@ def test_layer_approximates_exact_linear():
         err[r] = np.linalg.norm(Y - exact) / np.linalg.norm(exact)
     assert err[32] < 0.15
     assert err[32] < 0.8 * err[0]
+
+
+# ------------------------------- dynamic per-token activation scale (R5d) ----
+
+def _rows_with_common_max(seed, M, K):
+    """bf16 X whose column 0 holds the same large value in every row, so
+    every row of x_hat reaches the batch maximum there."""
+    rng = np.random.default_rng(seed)
+    x = rng.uniform(-1.0, 1.0, (M, K)).astype(np.float32)
+    x[:, 0] = 64.0
+    s = rng.uniform(0.5, 2.0, K).astype(np.float32)
+    return SI.f32_to_bf16_bits(x), s
+
+
+def test_dynamic_scale_reduces_to_static_when_row_max_is_batch_max():
+    """If every row's absmax equals the static (calibration) absmax, R5d and
+    R5 quantize identically."""
+    X, s = _rows_with_common_max(11, 12, 128)
+    xh = O.smooth_activation(X, s)
+    A_static = O.activation_absmax(SI.channel_absmax(X), s)
+    assert np.all(O.activation_absmax_rows(xh) == A_static)
+    _, c_st, sf_st = O.quantize_activation(X, s, A_static)
+    _, c_dy, sf_dy, _ = O.quantize_activation_dynamic(X, s)
+    assert np.array_equal(c_st, c_dy) and np.array_equal(sf_st, sf_dy)
+
+
+def test_dynamic_scale_is_per_row_and_power_of_two_invariant():
+    """Scaling one row by 2^k (exact in bf16 and fp32) leaves its codes and
+    scales unchanged, scales its A_m by 2^k, leaves every other row alone, and
+    scales that row of Y - bias by exactly 2^k."""
+    X, W, b = SI.random_layer(12, 16, 128, 32)
+    p = O.pack(W, SI.channel_absmax(X), 16)
+    Y0, c0, s0, _, A0 = O.linear_reference_dynamic(X, p, b)
+    bias = F.bf16_bits_to_f64(b)[None, :]
+    for m, k in ((3, 5), (7, -3)):
+        x = SI.bf16_bits_to_f32(X).copy()
+        x[m] *= np.float32(2.0 ** k)
+        X2 = SI.f32_to_bf16_bits(x)
+        Y2, c2, s2, _, A2 = O.linear_reference_dynamic(X2, p, b)
+        assert np.array_equal(c2, c0) and np.array_equal(s2, s0)
+        assert A2[m] == A0[m] * np.float32(2.0 ** k)
+        others = np.arange(16) != m
+        assert np.array_equal(A2[others], A0[others])
+        assert np.array_equal(Y2[others], Y0[others])
+        np.testing.assert_allclose(Y2[m] - bias[0], (2.0 ** k) * (Y0[m] - bias[0]),
+                                   rtol=1e-12, atol=1e-12 * np.abs(Y0[m]).max())
+
+
+def test_dynamic_scale_row_max_takes_the_top_code():
+    """The element at a row's maximum lands on E2M1 +-6 with block scale
+    E4M3 448: the per-row scale uses the whole 4-bit range."""
+    X, W, _ = SI.random_layer(13, 24, 256, 16)
+    s = O.smoothing_factors(SI.channel_absmax(X), W)
+    xh, codes, sf, A = O.quantize_activation_dynamic(X, s)
+    for m in range(xh.shape[0]):
+        k = int(np.argmax(np.abs(xh[m])))
+        assert abs(float(F.e2m1_decode(codes[m, k]))) == 6.0
+        assert float(F.e4m3_decode(sf[m, k // 16])) == 448.0
+        assert A[m] == np.abs(xh[m, k])
+
+
+def test_dynamic_scale_zero_row():
+    X, W, b = SI.random_layer(14, 6, 64, 16)
+    X = X.copy()
+    X[2] = 0
+    p = O.pack(W, SI.channel_absmax(X), 16)
+    Y, cx, sfx, xl1, A = O.linear_reference_dynamic(X, p, b)
+    assert A[2] == 0 and np.all(cx[2] == 0) and np.all(sfx[2] == 0) and np.all(xl1[2] == 0)
+    assert np.array_equal(Y[2], F.bf16_bits_to_f64(b))
+
+
+def test_dynamic_scale_beats_static_outside_calibration():
+    """Inputs 16x beyond the calibration range saturate the static scale;
+    the per-row scale tracks them."""
+    wl = SI.make_workload("single_256", M=64)
+    X, lt = wl.X_bf16, wl.layers[0]
+    W, b = lt.W, lt.bias_bf16
+    p = O.pack(W, SI.channel_absmax(X), 32)
+    Xbig = SI.f32_to_bf16_bits(SI.bf16_bits_to_f32(X) * np.float32(16.0))
+    exact = F.bf16_bits_to_f64(Xbig) @ W.astype(np.float64).T + F.bf16_bits_to_f64(b)[None, :]
+    Ys, _, _, _ = O.linear_reference(Xbig, p, b)
+    Yd, _, _, _, _ = O.linear_reference_dynamic(Xbig, p, b)
+    es = np.linalg.norm(Ys - exact) / np.linalg.norm(exact)
+    ed = np.linalg.norm(Yd - exact) / np.linalg.norm(exact)
+    assert ed < 0.15 and ed < 0.5 * es
