@@ -102,6 +102,32 @@ def test_quantize_act_strided_input():
 
 # ------------------------------------------------------------ full layer ----
 
+def test_linear_strided_output_writes_only_its_window():
+    """Y as a window of a wider, taller buffer (ldy > N, 8 columns in, rows
+    below M): the layer writes exactly rows [0, M) x columns [0, N) of the
+    window, bit-identical to a contiguous Y, and leaves the rest alone.  The
+    shape has a partial last column box (N = 272) and a partial row box
+    (M = 200)."""
+    S = _S()
+    M, K, N, r = 200, 256, 272, 16
+    X, W, b = SI.random_layer(31, M, K, N)
+    lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
+    Xd = to_dev_bf16(X)
+    Y0 = S.svdq_linear_forward(dw, Xd)
+    ld = N + 72                       # a multiple of 8 elements
+    sentinel = -3.0
+    big = torch.full((M + 130, ld), sentinel, dtype=torch.bfloat16, device="cuda")
+    Yv = big[:M, 8:8 + N]
+    assert Yv.stride(0) == ld and Yv.data_ptr() % 16 == 0
+    S.svdq_linear_forward(dw, Xd, Y=Yv)
+    torch.cuda.synchronize()
+    assert np.array_equal(from_dev_bf16(Yv), from_dev_bf16(Y0))
+    mask = torch.ones_like(big, dtype=torch.bool)
+    mask[:M, 8:8 + N] = False
+    assert bool((big[mask] == sentinel).all()), "the layer wrote outside its output window"
+    assert S.svdq_device_error() == 0
+
+
 LAYER_CASES = [  # M, K, N, r
     (1, 64, 16, 16), (100, 192, 48, 16), (129, 320, 272, 32), (200, 1024, 512, 0),
     (64, 512, 256, 128), (300, 768, 784, 48), (257, 3072, 3072, 32),
