@@ -46,6 +46,13 @@ Readings of what the pages leave open:
      scales).
   R7 packed layouts: codes are two per byte, the even k in the low nibble;
      block scales in the MMA tile layout (see `sf_to_mma_tiles`).
+  R11f GELU between the MLP pair's layers, in a form a fused kernel and this
+     oracle evaluate bit-identically: the tanh form of GELU,
+       0.5 y (1 + tanh(u)),  u = sqrt(2/pi) (y + 0.044715 y^3),
+     rewritten through 1 + tanh(u) = 2 / (1 + e^(-2u)) as
+       h = y / (1 + e^(-2u))      (no cancellation for any y),
+     every step one float32 operation in the order written in `gelu_tanh_f32`,
+     e^x from `exp_f32` (basic float32 operations only), h rounded to bf16.
   R5d dynamic per-token activation scale (an alternative to R5 for inputs
      outside the calibration range; not the pages' path): each row m of
      X_hat is its own tensor for R4, with A_m = max_k |x_hat_mk| taken at
@@ -364,6 +371,65 @@ def linear_reference_dynamic(X_bf16: np.ndarray, p: OraclePack,
     if bias_bf16 is not None:
         Y = Y + bf16_bits_to_f64(bias_bf16)[None, :]
     return Y, cx, sfx, xl1, A
+
+
+# ------------------------------------------- GELU of the MLP pair (R11f) ----
+
+_LOG2E = F32(1.4426950408889634)          # log2(e), rounded to float32
+_EXP2_TAYLOR = [F32(np.log(2.0) ** k / np.prod(np.arange(1, k + 1, dtype=np.float64)))
+                for k in range(8)]        # (ln 2)^k / k!, k = 0..7, float32
+_SQRT_2_OVER_PI = F32(np.sqrt(2.0 / np.pi))
+_GELU_CUBIC = F32(0.044715)
+
+
+def exp_f32(x: np.ndarray) -> np.ndarray:
+    """e^x in float32 from basic float32 operations (reading R11f):
+    t = fp32(x log2 e), clamped to [-126, 128]; n = t rounded to the nearest
+    integer (ties to even); f = t - n (exact, |f| <= 1/2); 2^f from the
+    degree-7 Taylor series of e^(f ln 2) in Horner form (each multiply and
+    add rounded to float32); the result is 2^f scaled by 2^n (exact; 2^128
+    overflows to inf).  Relative error a few 1e-6 at |x| ~ 80, from the
+    rounding of t; far below a bf16 ulp."""
+    x = np.asarray(x, F32)
+    t = (x * _LOG2E).astype(F32)
+    t = np.clip(t, F32(-126.0), F32(128.0)).astype(F32)
+    n = np.rint(t).astype(F32)
+    f = (t - n).astype(F32)
+    p = np.full(x.shape, _EXP2_TAYLOR[7], F32)
+    for k in range(6, -1, -1):
+        p = (p * f).astype(F32)
+        p = (p + _EXP2_TAYLOR[k]).astype(F32)
+    with np.errstate(over="ignore"):
+        return np.ldexp(p, n.astype(np.int32)).astype(F32)
+
+
+def gelu_tanh_f32(y: np.ndarray) -> np.ndarray:
+    """GELU, tanh form, reading R11f: h = y / (1 + e^(-2u)) with
+    u = sqrt(2/pi) (y + 0.044715 y^3), each step one float32 rounding:
+    y2 = y y, y3 = y2 y, v = 0.044715 y3, w = y + v, u = c w, E = exp(-2u),
+    d = 1 + E, h = y / d.  For finite y: h = y exactly for large y (E
+    underflows to 2^-126), and h = -0 once e^(-2u) passes 2^128 (true
+    values below 2^-120 in magnitude, which a bf16 result flushes anyway)."""
+    y = np.asarray(y, F32)
+    with np.errstate(over="ignore", divide="ignore", invalid="ignore"):
+        return _gelu_steps(y)
+
+
+def _gelu_steps(y: np.ndarray) -> np.ndarray:
+    y2 = (y * y).astype(F32)
+    y3 = (y2 * y).astype(F32)
+    v = (_GELU_CUBIC * y3).astype(F32)
+    w = (y + v).astype(F32)
+    u = (_SQRT_2_OVER_PI * w).astype(F32)
+    E = exp_f32((F32(-2.0) * u).astype(F32))
+    d = (F32(1.0) + E).astype(F32)
+    return (y / d).astype(F32)
+
+
+def gelu_bf16(Y_bf16: np.ndarray) -> np.ndarray:
+    """The MLP pair's glue on bf16 bits: bf16(gelu_tanh_f32(y))."""
+    y = bf16_bits_to_f64(Y_bf16).astype(F32)
+    return f64_to_bf16_bits(gelu_tanh_f32(y).astype(np.float64))
 
 
 # ------------------------------------------------------------ tolerance ----
