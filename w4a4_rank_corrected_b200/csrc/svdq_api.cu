@@ -61,13 +61,13 @@ struct DeviceInfo {
   bool ok = false;
   int num_sms = 0;
   bool attrs_set = false;
-  // max co-resident clusters of the activation kernel, per rank r/16 (0..8)
-  // and cluster size S (1..8); -1 = not queried yet
-  int max_clusters[9][9];
+  // max co-resident clusters of the activation kernel per cluster size S
+  // (1..8; every shared-memory plan holds one CTA per SM, so r does not
+  // matter); -1 = not queried yet
+  int max_clusters[9];
   int gemm_pairs = -1;  // max co-resident CTA pairs of the GEMM kernel
   DeviceInfo() {
-    for (auto& a : max_clusters)
-      for (int& v : a) v = -1;
+    for (int& v : max_clusters) v = -1;
   }
 };
 constexpr int kMaxDevices = 64;
@@ -174,7 +174,8 @@ int choose_splits(int tiles, int kchunks, int r, int sms) {
     const QALayout L = qa_layout(r, cps, S);
     if (L.xst < QA_MIN_XST) break;
     if (r > 0) {
-      int& cached = g_dev[dev].max_clusters[0][S];
+      std::lock_guard<std::mutex> lk(g_mu);   // the caches are shared by host threads
+      int& cached = g_dev[dev].max_clusters[S];
       if (cached < 0) {
         cudaLaunchConfig_t cfg;
         std::memset(&cfg, 0, sizeof(cfg));
@@ -272,6 +273,7 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
 int gemm_max_pairs(int sms) {
   int dev = 0;
   cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lk(g_mu);   // the caches are shared by host threads
   int& cached = g_dev[dev].gemm_pairs;
   if (cached < 0) {
     cudaLaunchConfig_t cfg;
