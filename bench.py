@@ -57,6 +57,11 @@ def parse_args():
                     help="replay each step from a CUDA graph (small layers are launch-bound)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--kernel-seconds", type=float, default=1.0,
+                    help="device time of the per-kernel timing batches (each kernel alone)")
+    ap.add_argument("--kernel-launches", type=int, default=1000,
+                    help="minimum launches of the per-kernel timing batches; 0 with "
+                         "--kernel-seconds 0 leaves them out (profiler runs)")
     return ap.parse_args()
 
 
@@ -161,9 +166,19 @@ class ClockSampler:
             self.out = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "50", "-i", str(self.gpu)], stdout=self.out, stderr=subprocess.DEVNULL)
+                 "-lms", "10", "-i", str(self.gpu)], stdout=self.out, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+            return
+        # nvidia-smi needs a moment to start: wait (bounded) for its first line
+        t0 = time.time()
+        while time.time() - t0 < 5.0:
+            try:
+                if os.path.getsize(self.path) > 0:
+                    break
+            except OSError:
+                pass
+            time.sleep(0.02)
 
     def stop(self):
         if self.proc is None:
@@ -254,26 +269,23 @@ def run_ours(args):
     # host work (TMA descriptor encoding, Python marshalling), which
     # dominates at small M.  By default the launches are issued one by one
     # (at large M they overlap through programmatic dependent launch).
-    graphs, qgraphs, ggraphs = None, None, None
+    graphs = None
     if args.graph:
         try:
-            graphs, qgraphs, ggraphs = [], [], []
+            graphs = []
             for j in range(nsets):
-                for lst, what in ((graphs, "both"), (qgraphs, "q"), (ggraphs, "g")):
-                    g = torch.cuda.CUDAGraph()
-                    with torch.cuda.graph(g):
-                        if what in ("both", "q"):
-                            S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j])
-                        if what in ("both", "g"):
-                            S.svdq_gemm(weights[j], codes[j], sfs[j], xl1s[j], M, Ys[j])
-                    lst.append(g)
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j])
+                    S.svdq_gemm(weights[j], codes[j], sfs[j], xl1s[j], M, Ys[j])
+                graphs.append(g)
             for j in range(nsets):
                 graphs[j].replay()
             torch.cuda.synchronize(dev)
         except Exception as ex:  # capture not available: time the launches directly
             print(f"graph capture failed ({type(ex).__name__}: {ex}); timing direct launches",
                   file=sys.stderr)
-            graphs = qgraphs = ggraphs = None
+            graphs = None
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
@@ -293,33 +305,52 @@ def run_ours(args):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
-    clocks = sampler.stop()
     elapsed_ms = max_over_ranks(ev_start.elapsed_time(ev_end), world, dev)
+
+    # Per-kernel times, right after the timed region and under the same clock
+    # sampling: each kernel alone, launched back to back from a CUDA graph of
+    # `per_graph` launches over the rotating buffer sets (so host launch cost
+    # does not hide the kernel), replayed until at least `min_launches`
+    # launches and `min_seconds` of device time; CUDA events on the
+    # launching stream around all replays.
+    def kernel_time_ms(launch, min_launches=1000, min_seconds=1.0, per_graph=200):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for i in range(per_graph):
+                launch(i)
+        g.replay()
+        torch.cuda.synchronize(dev)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        est = a.elapsed_time(b) / per_graph
+        reps = max(-(-min_launches // per_graph), int(min_seconds * 1e3 / (est * per_graph)) + 1)
+        cur = torch.cuda.current_stream(dev)
+        a.record(cur)
+        for _ in range(reps):
+            g.replay()
+        b.record(cur)
+        torch.cuda.synchronize(dev)
+        del g
+        return a.elapsed_time(b) / (reps * per_graph), reps * per_graph
+
+    if args.kernel_seconds > 0 or args.kernel_launches > 0:
+        kt = dict(min_launches=max(1, args.kernel_launches), min_seconds=args.kernel_seconds)
+        q_ms, q_n = kernel_time_ms(lambda i: S.svdq_quantize_act(
+            weights[i % nsets], Xs[i % nsets], codes[i % nsets], sfs[i % nsets], xl1s[i % nsets]),
+            **kt)
+        g_ms, g_n = kernel_time_ms(lambda i: S.svdq_gemm(
+            weights[i % nsets], codes[i % nsets], sfs[i % nsets], xl1s[i % nsets], M,
+            Ys[i % nsets]), **kt)
+    else:                      # profiler runs: per-kernel times come from the profiler
+        q_ms = g_ms = float("nan")
+        q_n = g_n = 0
+    clocks = sampler.stop()
     err = S.svdq_device_error(stream)
     if err:
         raise SystemExit(f"device error code {err:#x}")
-
-    # per-kernel times, after the timed region: each kernel on its own
-    # (graph replays when available), events around a batch of launches
-    def timed_batch(fn, n):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for i in range(n):
-            fn(i)
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        return a.elapsed_time(b) / n
-    n_per = max(8, min(1000, K_steps // 4))
-    if qgraphs is not None:
-        q_ms = timed_batch(lambda i: qgraphs[i % nsets].replay(), n_per)
-        g_ms = timed_batch(lambda i: ggraphs[i % nsets].replay(), n_per)
-    else:
-        q_ms = timed_batch(lambda i: S.svdq_quantize_act(weights[i % nsets], Xs[i % nsets],
-                                                         codes[i % nsets], sfs[i % nsets],
-                                                         xl1s[i % nsets], stream), n_per)
-        g_ms = timed_batch(lambda i: S.svdq_gemm(weights[i % nsets], codes[i % nsets],
-                                                 sfs[i % nsets], xl1s[i % nsets], M,
-                                                 Ys[i % nsets], stream), n_per)
     ms_per_step = elapsed_ms / K_steps
     flops = 2.0 * M * N * K
     value = world * flops * K_steps / (elapsed_ms * 1e-3) / 1e12
@@ -350,12 +381,22 @@ def run_ours(args):
             "pct_fp4_peak_burst": round(100 * gemm_tflops / fp4_burst, 1),
             "pct_fp4_datasheet_9pf": round(100 * gemm_tflops / 9000.0, 1),
             "quantize_act_gbs": round(q_gbs, 1), "quantize_act_pct_hbm": round(100 * q_gbs / hbm, 1),
+            "per_kernel_timing": "each kernel alone after the timed region, >= 1000 launches and >= 1 s from CUDA graphs",
             "layer_roofline_frac": round(max(flops / (fp4_sust * 1e12), (q_bytes + M * N * 2) / (hbm * 1e9)) / (ms_per_step * 1e-3), 3),
         },
-        "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_sust, 1),
-                     "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_sust, 4), "traffic": traffic,
+        "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(fp4_burst, 1),
+                     "unit": "TFLOP/s", "frac": round(gemm_tflops / fp4_burst, 4), "traffic": traffic,
                      "kernel": "w4a4_gemm_kernel",
-                     "peak_source": f"{peak_src} bf16_tflops_sustained x {FP4_OVER_BF16:g} (nominal FP4/BF16 dense ratio)"},
+                     "peak_source": f"{peak_src} bf16_tflops (burst) x {FP4_OVER_BF16:g} (nominal FP4/BF16 dense ratio); the kernel is timed alone",
+                     "frac_sustained": round(gemm_tflops / fp4_sust, 4),
+                     "peak_sustained": round(fp4_sust, 1),
+                     "timing": f"{g_n} back-to-back launches from a CUDA graph, CUDA events on the launching stream"},
+        "roofline_quantize_act": {"bound": "hbm", "achieved": round(q_gbs, 1), "peak": round(hbm, 1),
+                                  "unit": "GB/s", "frac": round(q_gbs / hbm, 4),
+                                  "traffic": profiled_traffic("quantize_act", args.workload),
+                                  "kernel": "quantize_act_kernel",
+                                  "algorithmic_bytes": int(q_bytes),
+                                  "timing": f"{q_n} back-to-back launches from a CUDA graph"},
         "gpu_launches": 2 * K_steps,
         "clocks": clocks,
     }
@@ -372,10 +413,11 @@ def run_ours(args):
 
 
 def e2e_leg(S, w, X0, M, K, N, r, dev, stream, steps, world):
-    """The same metric through the public host-buffer API (HostStreamer):
-    every step uploads X from pinned host memory, runs the layer and
-    downloads Y into pinned host memory; consecutive steps overlap (upload,
-    compute and download on three streams, two device buffer sets)."""
+    """The same metric through the public host-buffer call
+    (svdq_linear_forward_host, via HostStreamer): every step uploads X from
+    pinned host memory, runs the layer and downloads Y into pinned host
+    memory, one C call on one stream; consecutive steps alternate between
+    two streams, so one step's download overlaps the next step's upload."""
     import torch
     Xh = torch.from_numpy(X0.view(np.int16)).view(torch.bfloat16).pin_memory()
     Yh = [torch.empty((M, N), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
@@ -384,17 +426,23 @@ def e2e_leg(S, w, X0, M, K, N, r, dev, stream, steps, world):
         hs.submit(Xh, Yh[i & 1])
     hs.synchronize()
     torch.cuda.synchronize(dev)
+    cur = torch.cuda.current_stream(dev)
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(hs.up)
+    a.record(cur)
+    for st in hs.streams:
+        st.wait_stream(cur)
     for i in range(steps):
         hs.submit(Xh, Yh[i & 1])
-    b.record(hs.down)
+    for st in hs.streams:
+        cur.wait_stream(st)
+    b.record(cur)
     torch.cuda.synchronize(dev)
     ms = max_over_ranks(a.elapsed_time(b), world, dev) / steps
     return {"value": round(world * 2.0 * M * N * K / (ms * 1e-3) / 1e12, 3), "unit": "TFLOPS",
             "ms_per_step": round(ms, 4), "h2d_bytes_per_step": M * K * 2,
-            "d2h_bytes_per_step": M * N * 2, "overlap": "upload / compute / download of "
-            "consecutive steps on three streams"}
+            "d2h_bytes_per_step": M * N * 2,
+            "path": "svdq_linear_forward_host (C ABI): H2D copy, both kernels, D2H copy per step; "
+                    "steps alternate between two streams"}
 
 
 def _oracle_threads():
@@ -457,16 +505,20 @@ def cpu_baseline(spec, W, bias, X0, packed, r, budget_s=15.0):
 # ---------------------------------------------------------- reference ----
 
 def run_reference(args):
+    """The oracle alone, on the host cores (the reference implementation of
+    this path): its own pack (LAPACK SVD, untimed setup), then per step the
+    activation NVFP4, the float64 dequantized GEMM, the low-rank branch and
+    the bias on a bounded sample of rows.  Nothing of the CUDA library is
+    loaded."""
     rank, world, local = dist_env()
     if rank != 0:
         return
-    import w4a4_rank_corrected_b200 as S  # host pack only (the oracle takes its factors)
     from oracle import svdq as O
     spec = SI.workload_specs()[args.workload]
     ls, W, bias, X0 = layer_setup(spec, args.layer)
     M, K, N, r = ls.M, ls.K, ls.N, ls.r
-    packed = S.svdq_pack_weight(W, SI.channel_absmax(X0), r)
-    op, deq_w = _oracle_setup(W, X0, packed, r)
+    op = O.pack(W, SI.channel_absmax(X0), r)
+    deq_w = O.nvfp4_dequantize(op.codes_w, op.sf_w)
 
     def run(idx):
         O.linear_reference(X0, op, bias, rows=idx, deq_w=deq_w)
@@ -490,7 +542,7 @@ def run_reference(args):
                       "r": r, "rows_per_step": rows},
            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOPS", "cores": cores,
                             "kind": "oracle",
-                            "sample": f"{rows} rows of {M} per step (activation NVFP4 + float64 dequantized GEMM + low-rank branch + bias; weight dequantized once, untimed)"},
+                            "sample": f"{rows} rows of {M} per step (activation NVFP4 + float64 dequantized GEMM + low-rank branch + bias; the oracle's own pack and weight dequantization, untimed)"},
            "e2e": {"value": round(value, 6), "unit": "TFLOPS", "h2d_bytes_per_step": 0,
                    "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)

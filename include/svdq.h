@@ -84,8 +84,14 @@ svdq_status svdq_query_sizes(int N, int K, int r, svdq_sizes* out);
 
 /* ------------------------------------------------------------------ pack --
  * svdq_pack_weight: the offline quantization of one linear (host only,
- * synchronous, re-entrant; OpenMP threads).  Steps, in the article's order
- * ("Background: SVDQuant and Nunchaku"):
+ * synchronous, re-entrant; OpenMP threads).
+ * Source: "Bringing Nunchaku 4-bit diffusion inference to Diffusers",
+ * section "Background: SVDQuant and Nunchaku" (and its Korean rendering,
+ * "SVDQuant and the Nunchaku engine"): outliers are moved from the
+ * activations into the weight, the hardest part of each weight becomes a
+ * small 16-bit low-rank branch, the residual is quantized to 4 bit.  The
+ * formula of each step is a reading of that prose (the page prints none).
+ * Steps, in that order:
  *   1. smoothing: lambda_j = (x_absmax_j / max_n |W_nj|)^alpha (lambda = 1
  *      where either maximum is 0); stored as smooth_j = fp32(1/lambda_j), the
  *      activation multiplier (x_hat = fp32(x * smooth_j)); W~ = W / smooth
@@ -104,15 +110,22 @@ svdq_status svdq_query_sizes(int N, int K, int r, svdq_sizes* out);
  *      bf16 lo part of smooth_k * L1[k][i] (exact product in float64, hi =
  *      bf16(p), lo = bf16(p - hi)); l2_mma[n][i] = l2_mma[n][r+i] = L2[i][n],
  *      zero beyond 2r.
+ *   8. bias: carried through unchanged as bf16 (it enters only the GEMM
+ *      epilogue, Y = bf16(alpha * acc + bias), and takes no part in the
+ *      smoothing, the SVD or the quantization).
  * Arguments:
  *   W         host fp32 [N][K] (out x in, the PyTorch Linear layout)
  *   x_absmax  host fp32 [K], per-input-channel max |x| of calibration data
+ *   bias_bf16 host bf16 [N] or NULL (no bias)
  *   smooth_alpha  smoothing exponent (0.5 in the workloads here)
  *   seed      seed of the SVD's random start (the result is deterministic
  *             for a given seed and build)
  *   out       host buffers sized by svdq_query_sizes; every pointer field
- *             except bias must be non-NULL; the scalars are written.
- * Errors: INVALID_ARG for shapes/NULLs, NUMERIC for non-finite input.
+ *             except bias must be non-NULL (l1, l2, l1_mma, l2_mma may be
+ *             NULL when r == 0); the scalars are written.  out->bias, when
+ *             non-NULL, receives bias_bf16 (zeros when bias_bf16 is NULL).
+ * Errors: INVALID_ARG for shapes/NULLs (also bias_bf16 given with
+ * out->bias NULL), NUMERIC for non-finite input.
  */
 typedef struct svdq_packed_host {
   float*    smooth;      /* [K]        */
@@ -122,12 +135,14 @@ typedef struct svdq_packed_host {
   uint16_t* l2_mma;      /* [N][klr]   */
   uint8_t*  codes_w;     /* [N][K/2], even k in the low nibble             */
   uint8_t*  sf_w;        /* MMA tile layout (svdq_sf_tile_offset)          */
+  uint16_t* bias;        /* [N] bf16, or NULL                              */
   float amax_x, amax_w;  /* static activation absmax A_x, residual absmax A_w */
   float g_x, gs_x, g_w, alpha, lr_scale;
 } svdq_packed_host;
 
-svdq_status svdq_pack_weight(const float* W, const float* x_absmax, int N,
-                             int K, int r, float smooth_alpha, uint64_t seed,
+svdq_status svdq_pack_weight(const float* W, const float* x_absmax,
+                             const uint16_t* bias_bf16, int N, int K, int r,
+                             float smooth_alpha, uint64_t seed,
                              svdq_packed_host* out);
 
 /* ---------------------------------------------------------------- layout --
@@ -135,9 +150,20 @@ svdq_status svdq_pack_weight(const float* W, const float* x_absmax, int N,
  * layout used for sf_w and sf_x: atoms of 128 rows x 4 scales (512 bytes),
  * atom (row/128, g/4) at ((row/128) * (K/64) + g/4) * 512, and inside the
  * atom byte (row%32)*16 + ((row%128)/32)*4 + g%4.  Returns -1 on bad args.
- * This is the scale arrangement the block-scaled tensor-core MMA reads.
+ * This is the scale arrangement the block-scaled tensor-core MMA reads; the
+ * pages fix only "one E4M3 scale per 16 elements" (NVFP4, hardware-support
+ * table of "Bringing Nunchaku 4-bit diffusion inference to Diffusers").
  */
 int64_t svdq_sf_tile_offset(int row, int g, int K);
+
+/* svdq_unswizzle_scales: host permutation from the MMA tile layout back to
+ * plain row-major scales, sf_rowmajor[row][g] = sf_mma[svdq_sf_tile_offset(
+ * row, g, K)] for row < rows, g < K/16.  Used to compare device scales with
+ * a row-major reference.  Host pointers; sf_mma holds at least
+ * round_up(rows, 128) * K/16 bytes, sf_rowmajor rows * K/16 bytes.
+ * Errors: INVALID_ARG for NULLs, rows < 0, K not a multiple of 64. */
+svdq_status svdq_unswizzle_scales(const uint8_t* sf_mma, int rows, int K,
+                                  uint8_t* sf_rowmajor);
 
 /* -------------------------------------------------------------- forward --
  * Device-side weight: a plain struct of device pointers (filled by the
@@ -159,7 +185,12 @@ typedef struct svdq_weight {
  * 256-byte aligned.  0 on bad arguments. */
 size_t svdq_act_workspace_bytes(int M, int K, int r);
 
-/* svdq_quantize_act: activation kernel (one launch).  For every row of X:
+/* svdq_quantize_act: activation kernel (one launch).
+ * Source: the Korean rendering of "Bringing Nunchaku 4-bit diffusion
+ * inference to Diffusers", section "SVDQuant and the Nunchaku engine": the
+ * low-rank down projection is fused with the quantization kernel, which
+ * removes the 16-bit branch's extra memory traffic; NVFP4 per the
+ * hardware-support table of the same article.  For every row of X:
  * x_hat = fp32(x * smooth); NVFP4 with the static tensor scales g_x, gs_x
  * (per 16-group max, sf = E4M3(a * gs_x), codes = E2M1(x_hat * g_x / sf),
  * two per byte); and, fused, the
@@ -178,7 +209,11 @@ svdq_status svdq_quantize_act(const svdq_weight* w, const uint16_t* X, int M,
                               int64_t ldx, uint8_t* codes_x, uint8_t* sf_x,
                               uint16_t* xl1, void* stream);
 
-/* svdq_gemm: the 4-bit GEMM kernel (one launch): block-scaled FP4 x FP4
+/* svdq_gemm: the 4-bit GEMM kernel (one launch).
+ * Source: the Korean rendering of "Bringing Nunchaku 4-bit diffusion
+ * inference to Diffusers", section "SVDQuant and the Nunchaku engine": the
+ * low-rank up projection is fused with the 4-bit compute kernel; W4A4 (both
+ * operands 4-bit) per "Background: SVDQuant and Nunchaku".  Block-scaled FP4 x FP4
  * tensor-core MMA into an fp32 accumulator in tensor memory, the low-rank
  * up-projection xl1 * L2 accumulated into the same accumulator, epilogue
  * Y = bf16(alpha * acc + bias).
@@ -188,13 +223,35 @@ svdq_status svdq_gemm(const svdq_weight* w, const uint8_t* codes_x,
                       const uint8_t* sf_x, const uint16_t* xl1, int M,
                       uint16_t* Y, int64_t ldy, void* stream);
 
-/* svdq_linear_forward: svdq_quantize_act then svdq_gemm on one stream, with
- * the intermediates in `workspace` (device, >= svdq_act_workspace_bytes,
- * 256-byte aligned). */
+/* svdq_linear_forward: the whole layer, Y = Q(X_hat) Q(R)^T + (X_hat L1) L2
+ * + bias ("Background: SVDQuant and Nunchaku"; the runtime SVDQW4A4Linear
+ * layer that replaces nn.Linear in "Loading natively in Diffusers"):
+ * svdq_quantize_act then svdq_gemm on one stream, with the intermediates in
+ * `workspace` (device, >= svdq_act_workspace_bytes, 256-byte aligned). */
 svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t* X,
                                 int M, int64_t ldx, uint16_t* Y, int64_t ldy,
                                 void* workspace, size_t ws_bytes,
                                 void* stream);
+
+/* svdq_linear_forward_host: svdq_linear_forward for activations and outputs
+ * that live in host memory (the drop-in layer's view of a host batch):
+ * copies X_host to X_dev, runs the layer, copies Y_dev back to Y_host, all
+ * enqueued on `stream` in that order (one cudaMemcpy2DAsync per copy; no
+ * synchronization; the host buffers must stay valid until the stream
+ * reaches the end of the call, and should be pinned for the copies to be
+ * asynchronous).
+ *   X_host  host bf16 [M][ldx_host], ldx_host >= K
+ *   Y_host  host bf16 [M][ldy_host], ldy_host >= N
+ *   X_dev   device bf16 [M][K] (contiguous, 16-byte aligned)
+ *   Y_dev   device bf16 [M][N] (contiguous, 16-byte aligned)
+ *   workspace, ws_bytes, stream: as svdq_linear_forward.
+ * Errors: those of svdq_linear_forward; SVDQ_ERR_CUDA if a copy cannot be
+ * enqueued (nothing after it is enqueued). */
+svdq_status svdq_linear_forward_host(const svdq_weight* w, const uint16_t* X_host,
+                                     int M, int64_t ldx_host, uint16_t* Y_host,
+                                     int64_t ldy_host, uint16_t* X_dev,
+                                     uint16_t* Y_dev, void* workspace,
+                                     size_t ws_bytes, void* stream);
 
 /* svdq_linear_forward_static: the same forward as svdq_linear_forward, with
  * the intermediates in a fixed scratch area that the library holds in device
@@ -204,9 +261,10 @@ svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t* X,
  * plain C host with no device allocator of its own, or a runtime that plans
  * all memory ahead and forbids allocation inside its step.
  *   - Never allocates or frees device memory and calls no allocating library
- *     routine.  The first call on each device looks the scratch address up
- *     once (cudaGetSymbolAddress) and caches it; make that first call before
- *     any stream capture.
+ *     routine.  Each call looks the scratch address up on the current device
+ *     (cudaGetSymbolAddress, which reserves nothing); make the first call on
+ *     a device before any stream capture, since that lookup may load the
+ *     library's device code on the device.
  *   - M is limited by the scratch size: svdq_act_workspace_bytes(M, K, r)
  *     must be <= SVDQ_STATIC_WORKSPACE_BYTES, else SVDQ_ERR_WORKSPACE and
  *     nothing is launched (e.g. K = 3072, r = 32 allows M <= 9033).

@@ -50,30 +50,59 @@ def check_output(Y_bits: np.ndarray, Y_ref: np.ndarray, tol_fro: float = TOL_FRO
     return fro, maxabs
 
 
-def check_activation(codes_dev, sf_dev, xl1_dev, X_bits, op, M, K, r, rows=None):
-    """Bit-exact codes and scales; xl1 hi+lo against lr_scale * X_hat L1."""
+def check_activation(codes_dev, sf_dev, xl1_dev, X_bits, op, M, K, r, rows=None,
+                     chunk_rows=2048):
+    """Bit-exact codes and scales; xl1 hi+lo against lr_scale * X_hat L1.
+    With rows=None every row is compared (in chunks of rows, to bound the
+    oracle's memory), and the whole scale-tile buffer, padding rows
+    included, must equal the oracle's tiles."""
     torch = torch_mod()
-    idx = np.arange(M) if rows is None else np.asarray(rows)
-    xh, codes, sf = O.quantize_activation(X_bits[idx], op.s, op.A_x)
-    got_codes = codes_dev.cpu().numpy()[idx]
-    assert np.array_equal(got_codes, O.pack_nibbles(codes)), "activation codes differ"
+    codes_all = codes_dev.cpu().numpy()
     tiles = sf_dev.cpu().numpy()
-    got_sf = O.sf_from_mma_tiles(tiles, M, K)[idx]
-    assert np.array_equal(got_sf, sf), "activation scales differ"
-    if rows is None:  # the whole tile buffer, padding rows (zero scales) included
-        exp = O.sf_to_mma_tiles(sf)
+    got_sf_all = O.sf_from_mma_tiles(tiles, M, K)
+    xl_all = from_dev_bf16(xl1_dev) if r else None
+    lr_scale = np.float64(np.float32(op.g_x) * np.float32(op.g_w))
+    L1 = F.bf16_bits_to_f64(op.L1) if r else None
+    if rows is None:
+        blocks = [np.arange(a, min(M, a + chunk_rows)) for a in range(0, M, chunk_rows)]
+        sf_full = np.zeros((M, K // 16), np.uint8)
+    else:
+        blocks = [np.asarray(rows)]
+        sf_full = None
+    for idx in blocks:
+        xh, codes, sf = O.quantize_activation(X_bits[idx], op.s, op.A_x)
+        assert np.array_equal(codes_all[idx], O.pack_nibbles(codes)), \
+            f"activation codes differ in rows {idx[0]}..{idx[-1]}"
+        assert np.array_equal(got_sf_all[idx], sf), \
+            f"activation scales differ in rows {idx[0]}..{idx[-1]}"
+        if sf_full is not None:
+            sf_full[idx] = sf
+        if r:
+            want = O.lowrank_down(xh, op.L1) * lr_scale
+            xl = xl_all[idx]
+            hi = F.bf16_bits_to_f64(xl[:, :r])
+            lo = F.bf16_bits_to_f64(xl[:, r:2 * r])
+            scale = (np.abs(xh.astype(np.float64)) @ np.abs(L1)) * lr_scale
+            err = np.abs(hi + lo - want)
+            assert np.all(err <= 2e-5 * scale + 1e-30), float((err / (scale + 1e-30)).max())
+            assert np.all(xl[:, 2 * r:] == 0)
+    if sf_full is not None:  # the whole tile buffer, padding rows (zero scales) included
+        exp = O.sf_to_mma_tiles(sf_full)
         assert tiles.size >= exp.size
         assert np.array_equal(tiles[:exp.size], exp), "scale tiles differ"
-    if r:
-        lr_scale = np.float64(np.float32(op.g_x) * np.float32(op.g_w))
-        want = O.lowrank_down(xh, op.L1) * lr_scale
-        xl = from_dev_bf16(xl1_dev)[idx]
-        hi = F.bf16_bits_to_f64(xl[:, :r])
-        lo = F.bf16_bits_to_f64(xl[:, r:2 * r])
-        scale = (np.abs(xh.astype(np.float64)) @ np.abs(F.bf16_bits_to_f64(op.L1))) * lr_scale
-        err = np.abs(hi + lo - want)
-        assert np.all(err <= 2e-5 * scale + 1e-30), float((err / (scale + 1e-30)).max())
-        assert np.all(xl[:, 2 * r:] == 0)
+
+
+def rows_every_block(M, per_block=1, extra=64, seed=0, block=128):
+    """Row indices with at least `per_block` rows in every `block`-row block
+    (so every GEMM row tile and activation row block is looked at), plus
+    `extra` random rows and the first and last row."""
+    rng = np.random.default_rng(seed)
+    pick = [0, M - 1]
+    for b0 in range(0, M, block):
+        n = min(block, M - b0)
+        pick.extend((b0 + rng.choice(n, size=min(per_block, n), replace=False)).tolist())
+    pick.extend(rng.choice(M, size=min(extra, M), replace=False).tolist())
+    return np.unique(np.array(pick))
 
 
 def rows_sample(M, n=64, seed=0):

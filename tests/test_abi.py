@@ -127,12 +127,55 @@ def test_gpu_entry_points_refuse_without_b200():
     assert L.svdq_device_error(None, ctypes.byref(code)) == 2
 
 
+def test_unswizzle_scales_matches_oracle_layout():
+    rng = np.random.default_rng(3)
+    rows, K = 300, 512
+    sf = rng.integers(0, 127, (rows, K // 16)).astype(np.uint8)
+    tiled = O.sf_to_mma_tiles(sf)
+    assert np.array_equal(S.svdq_unswizzle_scales(tiled, rows, K), sf)
+    L = S.lib
+    out = np.empty((rows, K // 16), np.uint8)
+    assert L.svdq_unswizzle_scales(tiled.ctypes.data, rows, 100, out.ctypes.data) == 1
+    assert L.svdq_unswizzle_scales(None, rows, K, out.ctypes.data) == 1
+    assert L.svdq_unswizzle_scales(tiled.ctypes.data, -1, K, out.ctypes.data) == 1
+    assert L.svdq_unswizzle_scales(None, 0, K, None) == 0
+
+
+def test_host_forward_argument_validation():
+    L = S.lib
+    w = _fake_weight()
+    Xh, Yh, Xd, Yd, WS = 0x20000000, 0x30000000, 0x40000000, 0x50000000, 0x70000000
+    need = S.svdq_act_workspace_bytes(16, 256, 32)
+    f = L.svdq_linear_forward_host
+    assert f(None, Xh, 16, 256, Yh, 256, Xd, Yd, WS, need, None) == 1
+    assert f(ctypes.byref(w), None, 16, 256, Yh, 256, Xd, Yd, WS, need, None) == 1
+    assert f(ctypes.byref(w), Xh, 16, 255, Yh, 256, Xd, Yd, WS, need, None) == 1   # ldx < K
+    assert f(ctypes.byref(w), Xh, 16, 256, Yh, 200, Xd, Yd, WS, need, None) == 1   # ldy < N
+    assert f(ctypes.byref(w), Xh, 16, 256, Yh, 256, None, Yd, WS, need, None) == 1
+    assert f(ctypes.byref(w), Xh, 16, 256, Yh, 256, Xd, Yd, WS, need - 1, None) == 4
+    assert f(ctypes.byref(w), Xh, 16, 256, Yh, 256, Xd + 8, Yd, WS, need, None) == 3
+    assert f(ctypes.byref(w), Xh, 16, 256, Yh, 256, Xd, Yd, WS + 16, need, None) == 3
+    assert f(ctypes.byref(w), Xh, 0, 256, Yh, 256, Xd, Yd, WS, need, None) == 0
+    # host rows may be strided and unaligned: only the device side is checked
+    if not _has_gpu():
+        assert f(ctypes.byref(w), Xh + 2, 16, 300, Yh + 2, 260, Xd, Yd, WS, need, None) == 2
+
+
 def test_pack_rejects_bad_input():
     W = np.zeros((32, 64), np.float32)
     cx = np.ones(64, np.float32)
     with pytest.raises(S.SvdqError) as e:
         S.svdq_pack_weight(W, cx, 48)
     assert e.value.status == 1
+    # a bias given without an output buffer for it
+    out = S.SvdqPackedHost()
+    sm = np.empty(64, np.float32)
+    cw = np.empty((32, 32), np.uint8)
+    sfw = np.empty(256 * 4, np.uint8)
+    out.smooth, out.codes_w, out.sf_w, out.bias = sm.ctypes.data, cw.ctypes.data, sfw.ctypes.data, None
+    bias = np.zeros(32, np.uint16)
+    assert S.lib.svdq_pack_weight(W.ctypes.data, cx.ctypes.data, bias.ctypes.data, 32, 64, 0,
+                                  0.5, 0, ctypes.byref(out)) == 1
     W[3, 5] = np.nan
     with pytest.raises(S.SvdqError) as e:
         S.svdq_pack_weight(W, cx, 16)

@@ -4,7 +4,8 @@ Bar: bit-exact E2M1 codes and E4M3 scales (activation and weight); bf16
 output with relative Frobenius error <= 2e-3 against the float64 oracle and
 every element within 1e-2 rms(Y_ref) plus half a bf16 ulp.  Shapes span
 several tiles with ragged tails; the full-size workloads run in the launch
-configuration that bench.py times and are compared on sampled rows."""
+configuration that bench.py times, with codes and scales compared on every
+row and the output on at least one row of every 128-row block."""
 import numpy as np
 import pytest
 
@@ -12,8 +13,8 @@ import svdq_inputs as SI
 from oracle import formats as F
 from oracle import svdq as O
 
-from gpu_common import (check_activation, check_output, from_dev_bf16, prepare, rows_sample,
-                         to_dev_bf16)
+from gpu_common import (check_activation, check_output, from_dev_bf16, prepare, rows_every_block,
+                        rows_sample, to_dev_bf16)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,23 +38,41 @@ def _S():
 
 # ---------------------------------------------------------- conversions ----
 
-def _sweep():
-    vals = [0.0, -0.0, 6.0, 7.0, 448.0, 449.0, 464.0, 1e30, 2.0 ** -10, 2.0 ** -9, 3 * 2.0 ** -10]
-    for e in range(-12, 10):
-        m = np.arange(0, 1 << 11) / (1 << 11)
-        vals.extend(((1 + m) * 2.0 ** e).tolist())
-    v = np.array(vals, np.float32)
-    rng = np.random.default_rng(0)
-    v = np.concatenate([v, -v, (rng.standard_normal(200000) * 10).astype(np.float32)])
-    return v
+def _binade(e: int) -> np.ndarray:
+    """Every float32 in [2^e, 2^(e+1))."""
+    bits = ((e + 127) << 23) | np.arange(1 << 23, dtype=np.uint32)
+    return bits.astype(np.uint32).view(np.float32)
 
 
-def test_hardware_conversions_match_oracle():
+def test_hardware_conversions_match_oracle_exhaustive():
+    """The device conversions the activation kernel uses against the
+    oracle's encoders on EVERY float32 of the binades that reach a non-zero
+    code: E2M1 on [2^-3, 2^4) with both signs (below 2^-2 everything rounds
+    to a signed zero; from 6 on everything saturates), E4M3 on [2^-11, 2^10)
+    (non-negative: block scales; the smallest subnormal is 2^-9, the
+    largest finite 448).  Plus zeros, the sub-binade tails and saturation."""
     S = _S()
-    v = _sweep()
-    e2, e4 = S.svdq_debug_convert(torch.from_numpy(v).cuda())
-    assert np.array_equal(e2.cpu().numpy(), F.e2m1_encode(v))
-    assert np.array_equal(e4.cpu().numpy(), F.e4m3_encode_nonneg(np.abs(v)))
+    for e in range(-3, 4):
+        for sign in (1.0, -1.0):
+            v = _binade(e) * np.float32(sign)
+            e2, _ = S.svdq_debug_convert(torch.from_numpy(v).cuda())
+            got = e2.cpu().numpy()
+            want = F.e2m1_encode(v)
+            bad = np.nonzero(got != want)[0]
+            assert bad.size == 0, (e, sign, v[bad[:4]], got[bad[:4]], want[bad[:4]])
+    for e in range(-11, 10):
+        v = _binade(e)
+        _, e4 = S.svdq_debug_convert(torch.from_numpy(v).cuda())
+        got = e4.cpu().numpy()
+        want = F.e4m3_encode_nonneg(v)
+        bad = np.nonzero(got != want)[0]
+        assert bad.size == 0, (e, v[bad[:4]], got[bad[:4]], want[bad[:4]])
+    edge = np.array([0.0, -0.0, 2.0 ** -40, 2.0 ** -12, 1e-30, 6.0, 7.0, 448.0, 464.0, 1e30,
+                     3.0e38], np.float32)
+    edge = np.concatenate([edge, -edge])
+    e2, e4 = S.svdq_debug_convert(torch.from_numpy(edge).cuda())
+    assert np.array_equal(e2.cpu().numpy(), F.e2m1_encode(edge))
+    assert np.array_equal(e4.cpu().numpy(), F.e4m3_encode_nonneg(np.abs(edge)))
 
 
 def test_bounded_wait_reports_and_recovers():
@@ -223,8 +242,9 @@ def _workload_layer(name, M=None):
 @pytest.mark.parametrize("name", ["single_256", "flux_qkv", "sweep_r16", "sweep_r32", "sweep_r64",
                                   "sweep_r128", "sweep_m64", "sweep_m512"])
 def test_workload_parity(name):
-    """Each workload at full size: activation codes/scales bit-exact on every
-    row (or sampled rows for M > 1024), output on sampled rows."""
+    """Each workload at full size: activation codes and scales bit-exact on
+    every row, the output on every row for M <= 1024 and otherwise on at
+    least one row of every 128-row block."""
     S = _S()
     X, W, b, r = _workload_layer(name)
     M, K = X.shape
@@ -234,69 +254,61 @@ def test_workload_parity(name):
     ws = torch.empty(S.svdq_act_workspace_bytes(M, K, r), dtype=torch.uint8, device="cuda")
     Y = S.svdq_linear_forward(dw, Xd, workspace=ws)
     torch.cuda.synchronize()
-    rows = None if M <= 1024 else rows_sample(M, 128, seed=len(name))
-    check_activation(codes, sf, xl1, X, op, M, K, r, rows=rows)
-    idx = np.arange(M) if rows is None else rows
+    check_activation(codes, sf, xl1, X, op, M, K, r)
+    idx = np.arange(M) if M <= 1024 else rows_every_block(M, seed=len(name))
     Y_ref, _, _, _ = O.linear_reference(X, op, b, rows=idx)
     check_output(from_dev_bf16(Y)[idx], Y_ref)
 
 
+def _layer_check(S, lt, Xin_dev, Xin_bits, seed):
+    """One layer of a chain, calibrated on and compared with the oracle fed
+    its actual bf16 input: codes and scales on every row, the output on at
+    least one row of every 128-row block."""
+    M, K, r = Xin_bits.shape[0], lt.spec.K, lt.spec.r
+    lp, op, dw = prepare(lt.W, SI.channel_absmax(Xin_bits), r, lt.bias_bf16)
+    codes, sf, xl1 = S.svdq_quantize_act(dw, Xin_dev)
+    Y = S.svdq_linear_forward(dw, Xin_dev)
+    torch.cuda.synchronize()
+    check_activation(codes, sf, xl1, Xin_bits, op, M, K, r)
+    rows = rows_every_block(M, seed=seed)
+    Yr, _, _, _ = O.linear_reference(Xin_bits, op, lt.bias_bf16, rows=rows)
+    check_output(from_dev_bf16(Y)[rows], Yr)
+    return Y
+
+
 def test_mlp_pair_parity():
-    """fc1 -> GELU (tanh, bf16, on the GPU) -> fc2 (K = 12288).  Each layer is
-    compared with the oracle fed that layer's actual bf16 input."""
+    """fc1 -> GELU (tanh, bf16, on the GPU) -> fc2 (K = 12288)."""
     S = _S()
     wl = SI.make_workload("flux_mlp")
     X = wl.X_bf16
     fc1, fc2 = wl.layers
-    lp1, op1, dw1 = prepare(fc1.W, SI.channel_absmax(X), 32, fc1.bias_bf16)
-    Y1 = S.svdq_linear_forward(dw1, to_dev_bf16(X))
+    Y1 = _layer_check(S, fc1, to_dev_bf16(X), X, seed=5)
     H = torch.nn.functional.gelu(Y1, approximate="tanh")
-    Hb = from_dev_bf16(H)
-    lp2, op2, dw2 = prepare(fc2.W, SI.channel_absmax(Hb), 32, fc2.bias_bf16)
-    Y2 = S.svdq_linear_forward(dw2, H)
-    torch.cuda.synchronize()
-    rows = rows_sample(X.shape[0], 64, seed=5)
-    Y1r, _, _, _ = O.linear_reference(X, op1, fc1.bias_bf16, rows=rows)
-    check_output(from_dev_bf16(Y1)[rows], Y1r)
-    Y2r, _, _, _ = O.linear_reference(Hb, op2, fc2.bias_bf16, rows=rows)
-    check_output(from_dev_bf16(Y2)[rows], Y2r)
+    _layer_check(S, fc2, H, from_dev_bf16(H), seed=6)
 
 
 def test_flux_block_parity():
     """Config 4 (M = 18432): qkv -> out on the V slice of the qkv output
     (strided input, ldx = 9216) -> fc1 -> GELU (tanh, bf16, on the GPU) ->
-    fc2 (K = 12288).  Each layer is calibrated on, and compared with the
-    oracle fed, its actual bf16 input; codes and scales bit-exact and the
-    output within tolerance on sampled rows."""
+    fc2 (K = 12288)."""
     S = _S()
     wl = SI.make_workload("flux_block")
     X = wl.X_bf16
     qkv, out, fc1, fc2 = wl.layers
     M, H = X.shape
-    rows = rows_sample(M, 48, seed=9)
-
-    def layer(lt, Xin_dev, Xin_bits):
-        lp, op, dw = prepare(lt.W, SI.channel_absmax(Xin_bits), lt.spec.r, lt.bias_bf16)
-        codes, sf, xl1 = S.svdq_quantize_act(dw, Xin_dev)
-        Y = S.svdq_linear_forward(dw, Xin_dev)
-        torch.cuda.synchronize()
-        check_activation(codes, sf, xl1, Xin_bits, op, M, lt.spec.K, lt.spec.r, rows=rows)
-        Yr, _, _, _ = O.linear_reference(Xin_bits, op, lt.bias_bf16, rows=rows)
-        check_output(from_dev_bf16(Y)[rows], Yr)
-        return Y
-
-    Yq = layer(qkv, to_dev_bf16(X), X)
+    Yq = _layer_check(S, qkv, to_dev_bf16(X), X, seed=9)
     V = Yq[:, 2 * H:]                       # strided view, ldx = 3 H
     assert V.stride(0) == 3 * H
-    Yo = layer(out, V, from_dev_bf16(V))
-    Y1 = layer(fc1, Yo, from_dev_bf16(Yo))
+    Yo = _layer_check(S, out, V, from_dev_bf16(V), seed=10)
+    Y1 = _layer_check(S, fc1, Yo, from_dev_bf16(Yo), seed=11)
     G = torch.nn.functional.gelu(Y1, approximate="tanh")
-    layer(fc2, G, from_dev_bf16(G))
+    _layer_check(S, fc2, G, from_dev_bf16(G), seed=12)
 
 
 def test_host_streamer_matches_forward():
-    """The overlapped host-buffer path (three streams, two buffer sets) gives
-    the device forward's output bit for bit, batch after batch."""
+    """The host-buffer path (C ABI svdq_linear_forward_host, two streams,
+    two buffer sets) gives the device forward's output bit for bit, batch
+    after batch."""
     S = _S()
     M, K, N, r = 300, 512, 384, 32
     X0, W, b = SI.random_layer(91, M, K, N)
@@ -315,3 +327,53 @@ def test_host_streamer_matches_forward():
     for (Xh, Yh), ref in zip(outs, refs):
         got = Yh.view(torch.int16).numpy().view(np.uint16)
         assert np.array_equal(got, ref)
+
+
+def test_host_forward_strided_host_buffers():
+    """svdq_linear_forward_host with host rows wider than the tensor (ldx_host
+    > K, ldy_host > N): the device forward's output bit for bit, written into
+    exactly the [M, N] window of the host buffer."""
+    S = _S()
+    M, K, N, r = 257, 320, 272, 16
+    X, W, b = SI.random_layer(93, M, K, N)
+    lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
+    Xwide = np.zeros((M, K + 24), np.uint16)
+    Xwide[:, :K] = X
+    Xh = torch.from_numpy(Xwide.view(np.int16)).view(torch.bfloat16).pin_memory()[:, :K]
+    Yh_full = torch.full((M, N + 40), -2.0, dtype=torch.bfloat16).pin_memory()
+    Yh = Yh_full[:, :N]
+    Xd = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    Yd = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(S.svdq_act_workspace_bytes(M, K, r), dtype=torch.uint8, device="cuda")
+    S.svdq_linear_forward_host(dw, Xh, Yh, Xd, Yd, ws)
+    torch.cuda.synchronize()
+    ref = from_dev_bf16(S.svdq_linear_forward(dw, to_dev_bf16(X)))
+    got = Yh_full.view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got[:, :N], ref)
+    assert np.all(got[:, N:] == np.uint16(0xC000))     # bf16(-2.0): untouched
+
+
+def test_forward_on_side_stream_without_workspace():
+    """A forward on a non-current stream whose workspace and output the
+    binding allocates: the binding ties them to that stream, so work queued
+    meanwhile on the current stream cannot reuse their memory."""
+    S = _S()
+    M, K, N, r = 1024, 1024, 768, 32
+    X, W, b = SI.random_layer(95, M, K, N)
+    lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
+    Xd = to_dev_bf16(X)
+    ref = from_dev_bf16(S.svdq_linear_forward(dw, Xd))
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    outs = []
+    for _ in range(3):
+        Y = S.svdq_linear_forward(dw, Xd, stream=side)
+        outs.append(Y)
+        # churn the allocator on the current stream while the side stream runs
+        junk = [torch.full((M * K,), 7, dtype=torch.uint8, device="cuda") for _ in range(4)]
+        del junk
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    for Y in outs:
+        assert np.array_equal(from_dev_bf16(Y), ref)
+    assert S.svdq_device_error() == 0

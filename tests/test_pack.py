@@ -82,3 +82,41 @@ def test_pack_is_deterministic():
     b = S.svdq_pack_weight(W, cx, 32, seed=3)
     for f in ("smooth", "l1", "l2", "codes_w", "sf_w", "l1_mma", "l2_mma"):
         assert np.array_equal(getattr(a, f), getattr(b, f)), f
+
+
+def test_pack_balanced_sqrt_sigma_split():
+    """Reading R2: L1 = V sqrt(S), L2 = sqrt(S) U^T.  So the i-th column of L1
+    and the i-th row of L2 both have norm sqrt(sigma_i) (V, U orthonormal),
+    and L1^T L1 = L2 L2^T = diag(sigma), up to the bf16 rounding of the
+    factors and the randomized SVD's accuracy.  A pack that put all of S into
+    one factor (column norms 1 on the other) fails."""
+    X, W, _ = SI.random_layer(12, 64, 512, 384)
+    cx = SI.channel_absmax(X)
+    r = 32
+    p = S.svdq_pack_weight(W, cx, r)
+    L1 = F.bf16_bits_to_f64(p.l1)
+    L2 = F.bf16_bits_to_f64(p.l2)
+    sig = np.linalg.svd(O.smooth_weight(W, p.smooth), compute_uv=False)[:r]
+    c1 = np.linalg.norm(L1, axis=0)
+    r2 = np.linalg.norm(L2, axis=1)
+    assert np.allclose(c1, r2, rtol=2.0 ** -7), np.max(np.abs(c1 / r2 - 1))
+    # (the randomized SVD resolves the near-degenerate tail of the spectrum
+    # to about 1 %, so each sigma_i gets 2 % and their sum 1 %)
+    assert np.allclose(c1 ** 2, sig, rtol=2e-2)
+    assert abs((c1 ** 2).sum() / sig.sum() - 1) <= 1e-2
+    G1, G2 = L1.T @ L1, L2 @ L2.T
+    off = ~np.eye(r, dtype=bool)
+    assert np.max(np.abs(G1[off])) <= 2e-2 * sig[0]
+    assert np.max(np.abs(G2[off])) <= 2e-2 * sig[0]
+
+
+def test_pack_carries_bias():
+    X, W, b = SI.random_layer(13, 16, 128, 64)
+    cx = SI.channel_absmax(X)
+    p = S.svdq_pack_weight(W, cx, 16, bias_bf16=b)
+    assert np.array_equal(p.bias, b)
+    q = S.svdq_pack_weight(W, cx, 16)
+    assert q.bias is None
+    # the rest of the pack does not depend on the bias
+    for f in ("smooth", "l1", "l2", "codes_w", "sf_w"):
+        assert np.array_equal(getattr(p, f), getattr(q, f)), f

@@ -25,6 +25,7 @@ from . import build as _build
 __all__ = [
     "SvdqError", "PackedWeight", "DeviceWeight", "svdq_query_sizes", "svdq_pack_weight",
     "svdq_quantize_act", "svdq_gemm", "svdq_linear_forward", "svdq_act_workspace_bytes",
+    "svdq_linear_forward_host", "svdq_linear_forward_static", "svdq_unswizzle_scales",
     "svdq_device_error", "svdq_selftest_timeout", "svdq_debug_convert", "svdq_sf_tile_offset",
     "svdq_status_string", "SVDQW4A4Linear", "lib", "STATUS",
 ]
@@ -55,7 +56,7 @@ class SvdqPackedHost(ctypes.Structure):
     _fields_ = [("smooth", ctypes.c_void_p), ("l1", ctypes.c_void_p), ("l2", ctypes.c_void_p),
                 ("l1_mma", ctypes.c_void_p), ("l2_mma", ctypes.c_void_p),
                 ("codes_w", ctypes.c_void_p), ("sf_w", ctypes.c_void_p),
-                ("amax_x", ctypes.c_float), ("amax_w", ctypes.c_float),
+                ("bias", ctypes.c_void_p), ("amax_x", ctypes.c_float), ("amax_w", ctypes.c_float),
                 ("g_x", ctypes.c_float), ("gs_x", ctypes.c_float), ("g_w", ctypes.c_float),
                 ("alpha", ctypes.c_float), ("lr_scale", ctypes.c_float)]
 
@@ -80,7 +81,10 @@ def _load() -> ctypes.CDLL:
         "svdq_status_string": (ctypes.c_char_p, [I]),
         "svdq_version": (ctypes.c_char_p, []),
         "svdq_query_sizes": (I, [I, I, I, ctypes.POINTER(SvdqSizes)]),
-        "svdq_pack_weight": (I, [P, P, I, I, I, F, U64, ctypes.POINTER(SvdqPackedHost)]),
+        "svdq_pack_weight": (I, [P, P, P, I, I, I, F, U64, ctypes.POINTER(SvdqPackedHost)]),
+        "svdq_unswizzle_scales": (I, [P, I, I, P]),
+        "svdq_linear_forward_host": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P, P, P,
+                                         SZ, P]),
         "svdq_sf_tile_offset": (I64, [I, I, I]),
         "svdq_act_workspace_bytes": (SZ, [I, I, I]),
         "svdq_quantize_act": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P, P, P]),
@@ -140,6 +144,7 @@ class PackedWeight:
     l2_mma: np.ndarray       # bf16 [N, klr]
     codes_w: np.ndarray      # u8 [N, K/2]
     sf_w: np.ndarray         # u8, MMA tiles
+    bias: Optional[np.ndarray]  # bf16 [N] or None
     amax_x: float
     amax_w: float
     g_x: float
@@ -149,6 +154,8 @@ class PackedWeight:
     lr_scale: float
 
     def to_device(self, device="cuda", bias_bf16: Optional[np.ndarray] = None) -> "DeviceWeight":
+        """Device copies of the packed buffers.  The bias is the packed one
+        unless `bias_bf16` is given."""
         import torch
 
         def up(a):
@@ -158,6 +165,8 @@ class PackedWeight:
         if self.r > 0:
             t["l1_mma"] = up(self.l1_mma.view(np.int16))
             t["l2_mma"] = up(self.l2_mma.view(np.int16))
+        if bias_bf16 is None:
+            bias_bf16 = self.bias
         if bias_bf16 is not None:
             t["bias"] = up(np.asarray(bias_bf16, np.uint16).view(np.int16))
         return DeviceWeight(self, t)
@@ -192,7 +201,7 @@ class DeviceWeight:
 
 
 def svdq_pack_weight(W: np.ndarray, x_absmax: np.ndarray, r: int, smooth_alpha: float = 0.5,
-                     seed: int = 0) -> PackedWeight:
+                     seed: int = 0, bias_bf16: Optional[np.ndarray] = None) -> PackedWeight:
     W = np.ascontiguousarray(W, dtype=np.float32)
     x_absmax = np.ascontiguousarray(x_absmax, dtype=np.float32)
     N, K = W.shape
@@ -206,6 +215,13 @@ def svdq_pack_weight(W: np.ndarray, x_absmax: np.ndarray, r: int, smooth_alpha: 
     l2m = np.empty((N, sz.klr), np.uint16)
     codes = np.empty((N, K // 2), np.uint8)
     sf = np.empty(sz.sf_w_bytes, np.uint8)
+    bias_in = None
+    bias = None
+    if bias_bf16 is not None:
+        bias_in = np.ascontiguousarray(bias_bf16, dtype=np.uint16)
+        if bias_in.shape != (N,):
+            raise ValueError("bias must have shape [N]")
+        bias = np.empty(N, np.uint16)
     out = SvdqPackedHost()
     out.smooth = smooth.ctypes.data
     out.l1 = l1.ctypes.data if r else None
@@ -214,12 +230,26 @@ def svdq_pack_weight(W: np.ndarray, x_absmax: np.ndarray, r: int, smooth_alpha: 
     out.l2_mma = l2m.ctypes.data if r else None
     out.codes_w = codes.ctypes.data
     out.sf_w = sf.ctypes.data
-    _check(lib.svdq_pack_weight(W.ctypes.data, x_absmax.ctypes.data, N, K, r,
+    out.bias = bias.ctypes.data if bias is not None else None
+    _check(lib.svdq_pack_weight(W.ctypes.data, x_absmax.ctypes.data,
+                                bias_in.ctypes.data if bias_in is not None else None, N, K, r,
                                 float(smooth_alpha), int(seed), ctypes.byref(out)),
            "svdq_pack_weight")
-    return PackedWeight(N, K, r, sz.klr, smooth, l1, l2, l1m, l2m, codes, sf,
+    return PackedWeight(N, K, r, sz.klr, smooth, l1, l2, l1m, l2m, codes, sf, bias,
                         float(out.amax_x), float(out.amax_w), float(out.g_x), float(out.gs_x),
                         float(out.g_w), float(out.alpha), float(out.lr_scale))
+
+
+def svdq_unswizzle_scales(sf_mma: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """MMA tile layout -> row-major [rows, K/16] scales (host permutation)."""
+    sf_mma = np.ascontiguousarray(sf_mma, dtype=np.uint8)
+    need = ((rows + 127) // 128) * 128 * (K // 16)
+    if sf_mma.size < need:
+        raise ValueError("sf_mma smaller than round_up(rows, 128) * K/16 bytes")
+    out = np.empty((rows, K // 16), np.uint8)
+    _check(lib.svdq_unswizzle_scales(sf_mma.ctypes.data, rows, K, out.ctypes.data),
+           "svdq_unswizzle_scales")
+    return out
 
 
 # ------------------------------------------------------------- forward ----
@@ -247,6 +277,18 @@ def _check_x(X, K):
         raise ValueError("X must be a bf16 [M, K] tensor with unit column stride")
 
 
+def _keep_alive_on(stream, *tensors):
+    """Tensors made here on torch's current stream but used by kernels on
+    another stream: tell the caching allocator, so their memory is not
+    handed to other work before that stream is done with it."""
+    import torch
+    if stream is None or stream == torch.cuda.current_stream():
+        return
+    for t in tensors:
+        if t is not None:
+            t.record_stream(stream)
+
+
 def svdq_quantize_act(w: DeviceWeight, X, codes_x=None, sf_x=None, xl1=None, stream=None):
     """Returns (codes_x u8 [M, K/2], sf_x u8 tiles, xl1 bf16 [M, klr] or None)."""
     import torch
@@ -254,25 +296,33 @@ def svdq_quantize_act(w: DeviceWeight, X, codes_x=None, sf_x=None, xl1=None, str
     M = X.shape[0]
     klr, sf_bytes = _act_shapes(M, w.K, w.r)
     dev = X.device
+    made = []
     if codes_x is None:
         codes_x = torch.empty((M, w.K // 2), dtype=torch.uint8, device=dev)
+        made.append(codes_x)
     if sf_x is None:
         sf_x = torch.empty(sf_bytes, dtype=torch.uint8, device=dev)
+        made.append(sf_x)
     if xl1 is None and w.r > 0:
         xl1 = torch.empty((M, klr), dtype=torch.bfloat16, device=dev)
+        made.append(xl1)
     _check(lib.svdq_quantize_act(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
                                  codes_x.data_ptr(), sf_x.data_ptr(), _ptr(xl1),
                                  _stream_ptr(stream)), "svdq_quantize_act")
+    _keep_alive_on(stream, *made)
     return codes_x, sf_x, xl1
 
 
 def svdq_gemm(w: DeviceWeight, codes_x, sf_x, xl1, M: int, Y=None, stream=None):
     import torch
+    made = []
     if Y is None:
         Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=codes_x.device)
+        made.append(Y)
     _check(lib.svdq_gemm(ctypes.byref(w.struct), codes_x.data_ptr(), sf_x.data_ptr(),
                          _ptr(xl1), M, Y.data_ptr(), Y.stride(0), _stream_ptr(stream)),
            "svdq_gemm")
+    _keep_alive_on(stream, *made)
     return Y
 
 
@@ -280,15 +330,19 @@ def svdq_linear_forward(w: DeviceWeight, X, Y=None, workspace=None, stream=None)
     import torch
     _check_x(X, w.K)
     M = X.shape[0]
+    made = []
     if Y is None:
         Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+        made.append(Y)
     need = svdq_act_workspace_bytes(M, w.K, w.r)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+        made.append(workspace)
     _check(lib.svdq_linear_forward(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
                                    Y.data_ptr(), Y.stride(0), workspace.data_ptr(),
                                    workspace.numel(), _stream_ptr(stream)),
            "svdq_linear_forward")
+    _keep_alive_on(stream, *made)
     return Y
 
 
@@ -303,67 +357,64 @@ def svdq_linear_forward_static(w: DeviceWeight, X, Y=None, stream=None):
     import torch
     _check_x(X, w.K)
     M = X.shape[0]
+    made = []
     if Y is None:
         Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+        made.append(Y)
     _check(lib.svdq_linear_forward_static(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
                                           Y.data_ptr(), Y.stride(0), _stream_ptr(stream)),
            "svdq_linear_forward_static")
+    _keep_alive_on(stream, *made)
     return Y
 
 
 def svdq_linear_forward_host(w: DeviceWeight, X_host, Y_host, X_dev, Y_dev, workspace,
                              stream=None):
-    """The host-buffer form of the forward: copy X (pinned host) to the
-    device, run the layer, copy Y back into pinned host memory, all on
-    `stream` (asynchronous)."""
-    X_dev.copy_(X_host, non_blocking=True)
-    svdq_linear_forward(w, X_dev, Y_dev, workspace, stream)
-    Y_host.copy_(Y_dev, non_blocking=True)
+    """The host-buffer forward (C ABI svdq_linear_forward_host): X from host
+    memory (pinned, for an asynchronous copy) to the device, the layer, Y
+    back to host memory, all enqueued on `stream`.  X_dev [M, K], Y_dev
+    [M, N] and the workspace are caller-owned device buffers."""
+    _check_x(X_host, w.K)
+    M = X_host.shape[0]
+    if tuple(X_dev.shape) != (M, w.K) or tuple(Y_dev.shape) != (M, w.N) or \
+            tuple(Y_host.shape) != (M, w.N) or not X_dev.is_contiguous() or \
+            not Y_dev.is_contiguous() or Y_host.stride(1) != 1:
+        raise ValueError("X_dev [M, K], Y_dev [M, N] contiguous; Y_host [M, N] row-major")
+    _check(lib.svdq_linear_forward_host(ctypes.byref(w.struct), X_host.data_ptr(), M,
+                                        X_host.stride(0), Y_host.data_ptr(), Y_host.stride(0),
+                                        X_dev.data_ptr(), Y_dev.data_ptr(), workspace.data_ptr(),
+                                        workspace.numel(), _stream_ptr(stream)),
+           "svdq_linear_forward_host")
     return Y_host
 
 
 class HostStreamer:
-    """The forward over a sequence of host batches (pinned X in, pinned Y
-    out), with the upload of batch i+1, the two kernels of batch i and the
-    download of batch i-1 overlapped: three streams and two device buffer
-    sets.  submit() only enqueues; synchronize() waits for all of it."""
+    """The host-buffer forward over a sequence of host batches (pinned X in,
+    pinned Y out): each batch is one svdq_linear_forward_host call (upload,
+    both kernels, download, in order on one stream); consecutive batches
+    alternate between two streams with a device buffer set each, so the
+    download of one batch overlaps the upload and kernels of the next.
+    submit() only enqueues; synchronize() waits for all of it."""
 
     def __init__(self, w: DeviceWeight, M: int, device="cuda"):
         import torch
         self.w, self.M = w, M
         self.X = [torch.empty((M, w.K), dtype=torch.bfloat16, device=device) for _ in range(2)]
         self.Y = [torch.empty((M, w.N), dtype=torch.bfloat16, device=device) for _ in range(2)]
-        self.ws = torch.empty(max(svdq_act_workspace_bytes(M, w.K, w.r), 256), dtype=torch.uint8,
-                              device=device)
-        self.up, self.run, self.down = (torch.cuda.Stream(device=device) for _ in range(3))
-        ev = lambda: [torch.cuda.Event() for _ in range(2)]
-        self.uploaded, self.computed, self.downloaded = ev(), ev(), ev()
+        need = max(svdq_act_workspace_bytes(M, w.K, w.r), 256)
+        self.ws = [torch.empty(need, dtype=torch.uint8, device=device) for _ in range(2)]
+        self.streams = [torch.cuda.Stream(device=device) for _ in range(2)]
         self.n = 0
 
     def submit(self, X_host, Y_host):
-        b = self.n & 1
-        if self.n >= 2:                       # buffer set b was used by batch n-2
-            self.up.wait_event(self.computed[b])
-            self.run.wait_event(self.downloaded[b])
-        with torch_stream(self.up):
-            self.X[b].copy_(X_host, non_blocking=True)
-        self.uploaded[b].record(self.up)
-        self.run.wait_event(self.uploaded[b])
-        svdq_linear_forward(self.w, self.X[b], self.Y[b], self.ws, self.run)
-        self.computed[b].record(self.run)
-        self.down.wait_event(self.computed[b])
-        with torch_stream(self.down):
-            Y_host.copy_(self.Y[b], non_blocking=True)
-        self.downloaded[b].record(self.down)
+        b = self.n & 1                 # buffer set b is only ever used on stream b
+        svdq_linear_forward_host(self.w, X_host, Y_host, self.X[b], self.Y[b], self.ws[b],
+                                 self.streams[b])
         self.n += 1
 
     def synchronize(self):
-        self.down.synchronize()
-
-
-def torch_stream(s):
-    import torch
-    return torch.cuda.stream(s)
+        for s in self.streams:
+            s.synchronize()
 
 
 def svdq_device_error(stream=None) -> int:
@@ -404,8 +455,8 @@ class SVDQW4A4Linear(_linear_module_base()):
     def __init__(self, weight: np.ndarray, bias_bf16: Optional[np.ndarray], x_absmax: np.ndarray,
                  rank: int = 32, smooth_alpha: float = 0.5, seed: int = 0, device="cuda"):
         super().__init__()
-        self.packed = svdq_pack_weight(weight, x_absmax, rank, smooth_alpha, seed)
-        self.dev = self.packed.to_device(device, bias_bf16)
+        self.packed = svdq_pack_weight(weight, x_absmax, rank, smooth_alpha, seed, bias_bf16)
+        self.dev = self.packed.to_device(device)
         self.in_features = self.packed.K
         self.out_features = self.packed.N
         self._ws = None

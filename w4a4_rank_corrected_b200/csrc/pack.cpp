@@ -346,9 +346,21 @@ extern "C" int64_t svdq_sf_tile_offset(int row, int g, int K) {
   return sf_tile_offset(row, g, K);
 }
 
+extern "C" svdq_status svdq_unswizzle_scales(const uint8_t* sf_mma, int rows, int K,
+                                             uint8_t* sf_rowmajor) {
+  if (rows < 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
+  if (rows == 0) return SVDQ_OK;
+  if (!sf_mma || !sf_rowmajor) return SVDQ_ERR_INVALID_ARG;
+  const int G = K / 16;
+  for (int m = 0; m < rows; ++m)
+    for (int g = 0; g < G; ++g) sf_rowmajor[(size_t)m * G + g] = sf_mma[sf_tile_offset(m, g, K)];
+  return SVDQ_OK;
+}
+
 extern "C" svdq_status svdq_pack_weight(const float* W, const float* x_absmax,
-                                        int N, int K, int r, float smooth_alpha,
-                                        uint64_t seed, svdq_packed_host* out) {
+                                        const uint16_t* bias_bf16, int N, int K, int r,
+                                        float smooth_alpha, uint64_t seed,
+                                        svdq_packed_host* out) {
   svdq_sizes sz;
   svdq_status st = svdq_query_sizes(N, K, r, &sz);
   if (st != SVDQ_OK) return st;
@@ -356,6 +368,7 @@ extern "C" svdq_status svdq_pack_weight(const float* W, const float* x_absmax,
     return SVDQ_ERR_INVALID_ARG;
   if (r > 0 && (!out->l1 || !out->l2 || !out->l1_mma || !out->l2_mma))
     return SVDQ_ERR_INVALID_ARG;
+  if (bias_bf16 && !out->bias) return SVDQ_ERR_INVALID_ARG;
   if (!(smooth_alpha >= 0.0f) || !std::isfinite(smooth_alpha)) return SVDQ_ERR_INVALID_ARG;
   for (int k = 0; k < K; ++k)
     if (!std::isfinite(x_absmax[k]) || x_absmax[k] < 0) return SVDQ_ERR_NUMERIC;
@@ -452,6 +465,14 @@ extern "C" svdq_status svdq_pack_weight(const float* W, const float* x_absmax,
         out->l2_mma[(size_t)n * sz.klr + i] = v;
         out->l2_mma[(size_t)n * sz.klr + r + i] = v;
       }
+  }
+
+  // 8. bias: carried through as bf16 for the GEMM epilogue
+  if (out->bias) {
+    if (bias_bf16)
+      std::memcpy(out->bias, bias_bf16, (size_t)N * 2);
+    else
+      std::memset(out->bias, 0, (size_t)N * 2);
   }
   return SVDQ_OK;
 }

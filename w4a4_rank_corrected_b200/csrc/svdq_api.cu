@@ -438,32 +438,54 @@ extern "C" svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t*
   return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, s, sms);
 }
 
+extern "C" svdq_status svdq_linear_forward_host(const svdq_weight* w, const uint16_t* X_host,
+                                                int M, int64_t ldx_host, uint16_t* Y_host,
+                                                int64_t ldy_host, uint16_t* X_dev,
+                                                uint16_t* Y_dev, void* workspace,
+                                                size_t ws_bytes, void* stream) {
+  svdq_status st = check_weight(w);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || ldx_host < w->K || ldy_host < w->N) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!X_host || !Y_host || !X_dev || !Y_dev || !workspace) return SVDQ_ERR_INVALID_ARG;
+  if (ws_bytes < svdq_act_workspace_bytes(M, w->K, w->r)) return SVDQ_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return SVDQ_ERR_MISALIGNED;
+  if (!aligned16(X_dev) || !aligned16(Y_dev) || w->K % 8 || w->N % 8) return SVDQ_ERR_MISALIGNED;
+  if ((st = device_check(nullptr)) != SVDQ_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  const size_t xrow = (size_t)w->K * 2, yrow = (size_t)w->N * 2;
+  if (cudaMemcpy2DAsync(X_dev, xrow, X_host, (size_t)ldx_host * 2, xrow, (size_t)M,
+                        cudaMemcpyHostToDevice, s) != cudaSuccess) {
+    cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  st = svdq_linear_forward(w, X_dev, M, w->K, Y_dev, w->N, workspace, ws_bytes, stream);
+  if (st != SVDQ_OK) return st;
+  if (cudaMemcpy2DAsync(Y_host, (size_t)ldy_host * 2, Y_dev, yrow, yrow, (size_t)M,
+                        cudaMemcpyDeviceToHost, s) != cudaSuccess) {
+    cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
+}
+
 // Scratch of svdq_linear_forward_static: one per device, module-resident, so
 // that the call itself never allocates.  Calls that overlap in time (two
 // streams, two host threads) share it and race.
 __device__ __align__(256) unsigned char g_static_ws[SVDQ_STATIC_WORKSPACE_BYTES];
 
 namespace {
-void* g_static_ws_addr[kMaxDevices];
-
-// Device address of g_static_ws for the current device, looked up once per
-// device (cudaGetSymbolAddress) and cached.
+// Device address of g_static_ws on the current device.  Looked up on every
+// call (cudaGetSymbolAddress reserves nothing and costs a table lookup), so
+// no address outlives the module it belongs to, for instance across a
+// device reset that reloads the library's device code.
 svdq_status static_ws_address(void** out) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  void* a = nullptr;
+  if (cudaGetSymbolAddress(&a, g_static_ws) != cudaSuccess || !a) {
     cudaGetLastError();
-    return SVDQ_ERR_UNSUPPORTED_ARCH;
+    return SVDQ_ERR_CUDA;
   }
-  std::lock_guard<std::mutex> lk(g_mu);
-  if (!g_static_ws_addr[dev]) {
-    void* a = nullptr;
-    if (cudaGetSymbolAddress(&a, g_static_ws) != cudaSuccess || !a) {
-      cudaGetLastError();
-      return SVDQ_ERR_CUDA;
-    }
-    g_static_ws_addr[dev] = a;
-  }
-  *out = g_static_ws_addr[dev];
+  *out = a;
   return SVDQ_OK;
 }
 }  // namespace
