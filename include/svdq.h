@@ -76,7 +76,7 @@ typedef struct svdq_sizes {
   size_t l1_mma_bytes;   /* bf16 [2r][K]      kernel operand, see pack     */
   size_t l2_mma_bytes;   /* bf16 [N][klr]     kernel operand, see pack     */
   size_t codes_w_bytes;  /* u8   [N][K/2]     E2M1 codes of R              */
-  size_t sf_w_bytes;     /* u8   MMA tiles    E4M3 scales of R (rows padded to 256) */
+  size_t sf_w_bytes;     /* u8   MMA tiles    E4M3 scales of R, ceil(N/192) * 256 rows */
   size_t bias_bytes;     /* bf16 [N]                                       */
 } svdq_sizes;
 
@@ -134,7 +134,8 @@ typedef struct svdq_packed_host {
   uint16_t* l1_mma;      /* [2r][K]    */
   uint16_t* l2_mma;      /* [N][klr]   */
   uint8_t*  codes_w;     /* [N][K/2], even k in the low nibble             */
-  uint8_t*  sf_w;        /* MMA tile layout (svdq_sf_tile_offset)          */
+  uint8_t*  sf_w;        /* MMA tile layout, weight row n at atom-layout
+                            row svdq_weight_sf_row(n)                      */
   uint16_t* bias;        /* [N] bf16, or NULL                              */
   float amax_x, amax_w;  /* static activation absmax A_x, residual absmax A_w */
   float g_x, gs_x, g_w, alpha, lr_scale;
@@ -155,6 +156,13 @@ svdq_status svdq_pack_weight(const float* W, const float* x_absmax,
  * table of "Bringing Nunchaku 4-bit diffusion inference to Diffusers").
  */
 int64_t svdq_sf_tile_offset(int row, int g, int K);
+
+/* Row of that atom layout that holds the scales of weight row n: the GEMM
+ * reads the weight in tiles of 192 rows, each with two atom rows of its own
+ * (rows 0-127 and 128-191 of the tile, the second padded with 64 zero rows),
+ * so weight row n sits at (n / 192) * 256 + n % 192.  sf_w holds
+ * ceil(N / 192) * 256 rows.  -1 for n < 0. */
+int svdq_weight_sf_row(int n);
 
 /* svdq_unswizzle_scales: host permutation from the MMA tile layout back to
  * plain row-major scales, sf_rowmajor[row][g] = sf_mma[svdq_sf_tile_offset(
@@ -177,7 +185,7 @@ typedef struct svdq_weight {
   const uint16_t* l2_mma;   /* device bf16 [N][klr]       (NULL if r == 0) */
   const uint16_t* bias;     /* device bf16 [N] or NULL                     */
   const uint8_t*  codes_w;  /* device u8 [N][K/2]                          */
-  const uint8_t*  sf_w;     /* device u8, MMA tiles, rows padded to 256    */
+  const uint8_t*  sf_w;     /* device u8, MMA tiles, ceil(N/192)*256 rows  */
 } svdq_weight;
 
 /* Bytes of the activation workspace for M tokens: codes_x [M][K/2],

@@ -40,7 +40,7 @@ def test_query_sizes():
     sz = S.svdq_query_sizes(9216, 3072, 32)
     assert (sz.N, sz.K, sz.r, sz.klr) == (9216, 3072, 32, 64)
     assert sz.codes_w_bytes == 9216 * 1536
-    assert sz.sf_w_bytes == 9216 * 192
+    assert sz.sf_w_bytes == 48 * 256 * 192       # 48 tiles of 192 rows, 256 rows each
     sz = S.svdq_query_sizes(48, 192, 16)
     assert sz.klr == 64 and sz.sf_w_bytes == 256 * 12
     for bad in [(9216, 3000, 32), (9210, 3072, 32), (9216, 3072, 40), (9216, 3072, 144),
@@ -60,6 +60,18 @@ def test_sf_tile_offset_matches_oracle_layout():
         assert tiled[S.svdq_sf_tile_offset(r_, g, K)] == sf[r_, g]
     assert S.svdq_sf_tile_offset(0, K // 16, K) == -1
     assert S.svdq_sf_tile_offset(0, 0, 100) == -1
+
+
+def test_weight_sf_row_matches_oracle_layout():
+    rng = np.random.default_rng(1)
+    N, K = 496, 256
+    sf = rng.integers(0, 127, (N, K // 16)).astype(np.uint8)
+    tiled = O.sf_to_weight_tiles(sf)
+    assert tiled.size == S.svdq_query_sizes(N, K, 16).sf_w_bytes
+    for _ in range(1000):
+        n, g = int(rng.integers(N)), int(rng.integers(K // 16))
+        assert tiled[S.svdq_sf_tile_offset(S.lib.svdq_weight_sf_row(n), g, K)] == sf[n, g]
+    assert S.lib.svdq_weight_sf_row(-1) == -1
 
 
 def test_workspace_bytes():

@@ -86,6 +86,7 @@ def _load() -> ctypes.CDLL:
         "svdq_linear_forward_host": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P, P, P,
                                          SZ, P]),
         "svdq_sf_tile_offset": (I64, [I, I, I]),
+        "svdq_weight_sf_row": (I, [I]),
         "svdq_act_workspace_bytes": (SZ, [I, I, I]),
         "svdq_quantize_act": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P, P, P]),
         "svdq_gemm": (I, [ctypes.POINTER(SvdqWeight), P, P, P, I, P, I64, P]),

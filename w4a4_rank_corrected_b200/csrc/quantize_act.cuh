@@ -7,104 +7,136 @@
 // is merged into the quantization kernel so the 16-bit branch costs no extra
 // pass over the activations.  The B200 design:
 //
-//   * one CTA owns 64 rows x a contiguous slice of K (64-column chunks).  The
-//     host picks how many CTAs split K (a thread-block cluster of up to 8)
-//     so that the whole grid is resident in one wave;
+//   * one CTA owns 128 rows x a contiguous slice of K, walked in chunks of
+//     128 columns.  The host picks how many CTAs split K (S = 1, 2, 4 or 8,
+//     a thread-block cluster when S > 1) so that the whole grid is resident
+//     in one wave.  128 rows per CTA (one full scale-factor atom row) means
+//     every byte of the low-rank operand that reaches an SM serves 128 rows
+//     of X;
 //   * the slice's smoothing factors are loaded once (bulk copy) and stay in
 //     shared memory;
-//   * warp 0 streams X chunks [64 rows x 128 columns] bf16, as two 64 x 64
-//     boxes (TMA, 128-byte swizzle) under one barrier pair, into a ring of 4
-//     or 8 stages: the ring holds only X, so up to 128 KB of activations per
-//     SM are in flight;
-//   * warp 2 streams the matching chunks of the low-rank operand L1' into a
-//     separate ring of up to 8 stages (they come from L2: every row block
-//     reads the same L1', so each row block starts its K slice at a
-//     different chunk to spread those reads);
-//   * QA_QWARPS quantize warps: unit u = (chunk u / 4, box (u % 4) / 2,
-//     rows 32 (u % 2) .. + 31) goes to warp u % QA_QWARPS; lane l handles one
-//     row.  A warp copies
-//     its row segment (128 bytes per lane) into registers, hands the X stage
-//     back, then quantizes: per 16-group multiply by the smoothing factors,
-//     take the maximum, form the E4M3 block scale with one multiply and the
-//     hardware conversion, look up g/scale in a 127-entry table (the IEEE
-//     quotients, computed once per CTA), form the E2M1 codes with the
-//     hardware conversion; per row 32 code bytes and one 32-bit word of
-//     scales go straight into the MMA tile layout;
+//   * warp 0 streams X chunks [128 rows x 128 columns] bf16, as two
+//     128 x 64 boxes (TMA, 128-byte swizzle) under one barrier pair, into a
+//     ring of 2 or 4 stages; warp 2 streams the matching chunks of the
+//     low-rank operand L1' into a separate ring (they come from L2: every
+//     row block reads the same L1', so each row block starts its K slice at
+//     a different chunk to spread those reads);
+//   * QA_QWARPS quantize warps: unit u = (chunk u / 8, box (u % 8) / 4,
+//     rows 32 (u % 4) .. + 31) goes to warp u % QA_QWARPS; lane l handles one
+//     row.  A warp copies its row segment (128 bytes per lane) into
+//     registers, hands the X stage back, then quantizes: per 16-group
+//     multiply by the smoothing factors, take the maximum, form the E4M3
+//     block scale with one multiply and the hardware conversion, look up
+//     g/scale in a 127-entry table (the IEEE quotients, computed once per
+//     CTA), form the E2M1 codes with the hardware conversion.  The 32 code
+//     bytes and the 32-bit scale word of each row go into a shared-memory
+//     staging slot laid out exactly as the global tiles (codes with the
+//     64-byte swizzle of their TMA box, scales in the MMA atom layout);
+//   * warp 3 (one lane) writes each finished chunk out: one TMA tile store
+//     of the 128 x 64-byte code box and one bulk copy of the chunk's two
+//     512-byte scale atoms -- coalesced, asynchronous stores instead of one
+//     scattered 16-byte store per lane and row;
 //   * warp 1 (converged: every lane waits, an elected lane issues) issues
-//     tcgen05 bf16 MMAs (M = 64) on the SAME shared-memory X
-//     tile: X [64 x 64] times L1' [2r x 64]^T into a 64 x 2r fp32 accumulator
-//     in tensor memory.  L1' holds smooth * L1 split into bf16 hi and lo
+//     tcgen05 bf16 MMAs (M = 128) on the SAME shared-memory X tile: X
+//     [128 x 64] times L1' [2r x 64]^T into a 128 x 2r fp32 accumulator in
+//     tensor memory.  L1' holds smooth * L1 split into bf16 hi and lo
 //     halves, so X L1' = X_hat L1 to ~2^-16 relative (X itself is exact);
 //   * at the end the accumulator is read back (tcgen05.ld) and hi + lo
-//     columns are summed.  In a K split every rank but 0 pushes its partial
-//     sums into rank 0's shared memory with st.async (the bytes are counted
-//     on a barrier there), rank 0 adds them in rank order (deterministic) and
-//     stores the result times lr_scale as a bf16 hi/lo pair for the GEMM's
-//     up-projection.
+//     columns are summed.  In a K split the r output columns are shared out
+//     among the S ranks (rank o owns columns [o r/S, (o+1) r/S)): every rank
+//     pushes its partial sums of the columns it does not own into the
+//     owner's shared memory with st.async (the bytes are counted on a
+//     barrier there), and each owner adds the S partials of its columns in
+//     rank order (deterministic) and stores them times lr_scale as a bf16
+//     hi/lo pair for the GEMM's up-projection.
 #pragma once
 #include "ptx.cuh"
 
 namespace svdq_dev {
 
-constexpr int QA_BM = 64;
+constexpr int QA_BM = 128;                                 // rows per CTA
 constexpr int QA_QWARPS = 16;
-constexpr int QA_QWARP0 = 3;                               // first quantize warp
+constexpr int QA_QWARP0 = 4;                               // first quantize warp
 constexpr int QA_THREADS = 32 * (QA_QWARP0 + QA_QWARPS);
 // A chunk is 128 columns of the slice: two 64-column TMA boxes (128-byte
 // swizzle rows) that share one barrier pair, so each barrier round trip of
-// the producer moves 16 KB of X.
+// the producer moves 32 KB of X.
 constexpr int QA_BOXES = 2;
-constexpr uint32_t QA_BOX_BYTES = QA_BM * 128;             // 64 rows x 64 bf16
+constexpr uint32_t QA_BOX_BYTES = QA_BM * 128;             // 128 rows x 64 bf16
 constexpr uint32_t QA_X_BYTES = QA_BOXES * QA_BOX_BYTES;   // one X stage
-// X ring depth: a multiple of QA_QWARPS / 4.  A chunk has 4 units (two row
-// halves x two boxes); warp w's units cover chunks w / 4, w / 4 + 3,
-// w / 4 + 6, ...; with the depth a multiple of 3, the
-// previous use of the stage a warp is about to wait on was that same warp's
-// own earlier chunk, which it has already seen land, so the stage's barrier
-// is never two phases behind a parity wait (which would pass at once).
-constexpr int QA_UNITS = 2 * QA_BOXES;                     // units per chunk
+constexpr int QA_UNITS = QA_BOXES * (QA_BM / 32);          // units per chunk (8)
+// Ring depths (X, staging) are multiples of the chunk stride of a warp's
+// units, QA_QWARPS / QA_UNITS = 2: warp w's units cover chunks w / 8,
+// w / 8 + 2, w / 8 + 4, ...  So the previous use of any stage a warp is about
+// to wait on was that same warp's own earlier chunk, which it has already
+// seen complete, and no stage barrier is ever two phases behind a parity
+// wait (which would pass at once).
 constexpr int QA_XST_STEP = QA_QWARPS / QA_UNITS;
 constexpr int QA_MAX_XST = 2 * QA_XST_STEP;
 constexpr int QA_MIN_XST = QA_XST_STEP;
 constexpr int QA_MAX_LST = 8;
-static_assert(QA_QWARPS % QA_UNITS == 0 && QA_MAX_XST % QA_XST_STEP == 0,
-              "ring depth must be a multiple of the chunk stride of a warp's units");
+constexpr int QA_MAX_NSTG = 2 * QA_XST_STEP;
+constexpr int QA_MIN_NSTG = QA_XST_STEP;
+static_assert(QA_QWARPS % QA_UNITS == 0 && QA_MAX_XST % QA_XST_STEP == 0 &&
+                  QA_MAX_NSTG % QA_XST_STEP == 0,
+              "ring depths must be multiples of the chunk stride of a warp's units");
+constexpr uint32_t QA_CODES_STG = QA_BM * 64;              // 128 rows x 64 code bytes
+constexpr uint32_t QA_SF_STG = QA_BOXES * 512;             // two scale atoms
+constexpr uint32_t QA_STG_BYTES = QA_CODES_STG + QA_SF_STG;  // 9 KB, 1024-aligned slots
+static_assert(QA_STG_BYTES % 1024 == 0, "staging slots keep 1024-byte alignment");
 constexpr uint32_t QA_SMEM_BUDGET = 224 * 1024;  // + 1.5 KB: within the 227 KB per CTA
 
 // Shared-memory plan of one CTA (offsets from the 1024-aligned base).
 struct QALayout {
-  int xst, lst;              // ring depths (X, low-rank operand)
+  int xst, lst, nstg;        // ring depths (X, low-rank operand, output staging)
   uint32_t l1_bytes;         // one low-rank stage: two boxes of 2r rows x 128 bytes
-  uint32_t l1_off, s_off, red_off, lut_off, bar_off;
+  uint32_t l1_off, stg_off, s_off, red_off, lut_off, bar_off;
   uint32_t total;            // bytes to request (incl. alignment slack)
 };
+
+// Bytes of one rank's reduction buffer: the (S - 1) other ranks' partial
+// sums of the r / S columns it owns, 128 rows each, fp32.
+__host__ __device__ inline uint32_t qa_red_bytes(int r, int num_splits) {
+  if (r <= 0 || num_splits <= 1) return 0u;
+  return (uint32_t)(num_splits - 1) * QA_BM * (uint32_t)(r / num_splits) * 4u;
+}
 
 __host__ __device__ inline QALayout qa_layout(int r, int chunks_per_split, int num_splits) {
   QALayout L;
   L.l1_bytes = (uint32_t)QA_BOXES * 256u * (uint32_t)r;
   const uint32_t s_bytes = (uint32_t)QA_BOXES * 256u * (uint32_t)chunks_per_split;
-  const uint32_t red_bytes =
-      (r > 0 && num_splits > 1) ? (uint32_t)(num_splits - 1) * QA_BM * (uint32_t)r * 4u : 0u;
+  const uint32_t red_bytes = qa_red_bytes(r, num_splits);
   const uint32_t fixed = s_bytes + red_bytes + 512u + 512u;
-  // the deeper X ring if the low-rank ring still gets a stage, else the
-  // shallower one; the low-rank ring takes what is left, up to 8 stages
+  const int lmax = chunks_per_split < QA_MAX_LST ? (chunks_per_split > 0 ? chunks_per_split : 1)
+                                                 : QA_MAX_LST;
+  // Preference: the deeper X ring, then two staging slots and two low-rank
+  // stages, then as many low-rank stages as fit (up to the chunk count),
+  // then deeper staging; a shallower plan only when nothing deeper fits.
   L.xst = 0;
   L.lst = 0;
-  for (int xst = QA_MAX_XST; xst >= QA_MIN_XST; xst -= QA_XST_STEP) {
-    const uint32_t used = fixed + (uint32_t)xst * QA_X_BYTES;
-    if (used > QA_SMEM_BUDGET) continue;
-    int lst = 0;
-    if (r > 0) {
-      lst = (int)((QA_SMEM_BUDGET - used) / L.l1_bytes);
-      lst = lst > QA_MAX_LST ? QA_MAX_LST : lst;
-      if (lst < 1) continue;
+  L.nstg = 0;
+  for (int pass = 0; pass < 2 && L.xst == 0; ++pass) {
+    const int lmin = (r > 0) ? (pass == 0 ? (lmax < 2 ? lmax : 2) : 1) : 0;
+    for (int xst = QA_MAX_XST; xst >= QA_MIN_XST && L.xst == 0; xst -= QA_XST_STEP) {
+      const uint32_t used = fixed + (uint32_t)xst * QA_X_BYTES + QA_MIN_NSTG * QA_STG_BYTES;
+      if (used + (uint32_t)lmin * L.l1_bytes > QA_SMEM_BUDGET) continue;
+      int lst = 0;
+      if (r > 0) {
+        lst = (int)((QA_SMEM_BUDGET - used) / L.l1_bytes);
+        lst = lst > lmax ? lmax : lst;
+      }
+      int nstg = QA_MIN_NSTG;
+      if (used + (uint32_t)lst * L.l1_bytes + (QA_MAX_NSTG - QA_MIN_NSTG) * QA_STG_BYTES <=
+          QA_SMEM_BUDGET)
+        nstg = QA_MAX_NSTG;
+      L.xst = xst;
+      L.lst = lst;
+      L.nstg = nstg;
     }
-    L.xst = xst;
-    L.lst = lst;
-    break;
   }
   L.l1_off = (uint32_t)L.xst * QA_X_BYTES;
-  L.s_off = L.l1_off + (uint32_t)L.lst * L.l1_bytes;
+  L.stg_off = L.l1_off + (uint32_t)L.lst * L.l1_bytes;      // multiple of 1024
+  L.s_off = L.stg_off + (uint32_t)L.nstg * QA_STG_BYTES;
   L.red_off = L.s_off + s_bytes;
   L.lut_off = L.red_off + red_bytes;
   L.bar_off = L.lut_off + 512u;
@@ -114,7 +146,6 @@ __host__ __device__ inline QALayout qa_layout(int r, int chunks_per_split, int n
 
 struct QAParams {
   const float* smooth;
-  uint8_t* codes_x;
   uint8_t* sf_x;
   uint16_t* xl1;
   int M, K, r, klr;
@@ -125,11 +156,6 @@ struct QAParams {
   float g_x, gs_x, lr_scale;
   uint64_t timeout_ns;
 };
-
-__device__ __forceinline__ int64_t sf_tile_off(int row, int g, int K) {
-  return ((int64_t)(row >> 7) * (K >> 6) + (g >> 2)) * 512 + (row & 31) * 16 +
-         ((row & 127) >> 5) * 4 + (g & 3);
-}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -142,47 +168,41 @@ __device__ __forceinline__ void split_hi_lo(float v, float& hi, float& lo) {
   lo = __fsub_rn(v, hi);
 }
 
-// Store 16 consecutive fp32 values (times lr_scale) as a bf16 hi part at
-// dst_hi and a bf16 lo part at dst_lo.
-__device__ __forceinline__ void store_hi_lo16(const float (&v)[16], float scale, uint16_t* dst_hi,
-                                              uint16_t* dst_lo) {
-  uint32_t ph[8], pl[8];
+// Store 4 consecutive fp32 values (times lr_scale) as a bf16 hi part at
+// dst_hi and a bf16 lo part at dst_lo (8 bytes each).
+__device__ __forceinline__ void store_hi_lo4(const float (&v)[4], float scale, uint16_t* dst_hi,
+                                             uint16_t* dst_lo) {
+  float h[4], l[4];
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    float h0, l0, h1, l1;
-    split_hi_lo(__fmul_rn(v[2 * j], scale), h0, l0);
-    split_hi_lo(__fmul_rn(v[2 * j + 1], scale), h1, l1);
-    ph[j] = pack_bf16x2(h0, h1);
-    pl[j] = pack_bf16x2(l0, l1);
-  }
-  uint4* dh = reinterpret_cast<uint4*>(dst_hi);
-  uint4* dl = reinterpret_cast<uint4*>(dst_lo);
-  dh[0] = make_uint4(ph[0], ph[1], ph[2], ph[3]);
-  dh[1] = make_uint4(ph[4], ph[5], ph[6], ph[7]);
-  dl[0] = make_uint4(pl[0], pl[1], pl[2], pl[3]);
-  dl[1] = make_uint4(pl[4], pl[5], pl[6], pl[7]);
+  for (int j = 0; j < 4; ++j) split_hi_lo(__fmul_rn(v[j], scale), h[j], l[j]);
+  *reinterpret_cast<uint2*>(dst_hi) = make_uint2(pack_bf16x2(h[0], h[1]), pack_bf16x2(h[2], h[3]));
+  *reinterpret_cast<uint2*>(dst_lo) = make_uint2(pack_bf16x2(l[0], l[1]), pack_bf16x2(l[2], l[3]));
 }
 
 __global__ void __launch_bounds__(QA_THREADS, 1)
     quantize_act_kernel(const __grid_constant__ CUtensorMap tm_x,
-                        const __grid_constant__ CUtensorMap tm_l1, const QAParams p) {
+                        const __grid_constant__ CUtensorMap tm_l1,
+                        const __grid_constant__ CUtensorMap tm_codes, const QAParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int r = p.r;
   const bool has_lr = r > 0;
   const QALayout& L = p.L;
-  const int XST = L.xst, LST = L.lst;
+  const int XST = L.xst, LST = L.lst, NSTG = L.nstg;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bar_off);
   const uint32_t x_full0 = smem_u32(bars);
   const uint32_t x_empty0 = x_full0 + 8 * XST;
   const uint32_t l_full0 = x_empty0 + 8 * XST;
   const uint32_t l_empty0 = l_full0 + 8 * LST;
-  const uint32_t acc_full = l_empty0 + 8 * LST;
+  const uint32_t staged0 = l_empty0 + 8 * LST;
+  const uint32_t free0 = staged0 + 8 * NSTG;
+  const uint32_t acc_full = free0 + 8 * NSTG;
   const uint32_t s_bar = acc_full + 8;
   const uint32_t red_bar = acc_full + 16;
   const uint32_t drain_bar = acc_full + 24;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * XST + 2 * LST + 4);
+  uint32_t* tmem_holder =
+      reinterpret_cast<uint32_t*>(bars + 2 * XST + 2 * LST + 2 * NSTG + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   float* qlut = reinterpret_cast<float*>(smem + L.lut_off);  // 128 floats
   const float* s_sm = reinterpret_cast<const float*>(smem + L.s_off);
@@ -192,7 +212,9 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   const int rb = blockIdx.y;
   const int S = p.num_splits;
   const bool reduce = has_lr && S > 1;
+  const int own_cols = reduce ? r / S : r;     // columns of the result this rank finishes
   const int kchunks = ((p.K >> 6) + QA_BOXES - 1) / QA_BOXES;   // 128-column chunks
+  const int k64 = p.K >> 6;
   const int c_begin = split * p.chunks_per_split;
   const int c_end = min(kchunks, c_begin + p.chunks_per_split);
   const int nchunks = max(0, c_end - c_begin);
@@ -204,11 +226,15 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int i = 0; i < XST; ++i) {
       mbar_init(x_full0 + 8 * i, 1);
-      mbar_init(x_empty0 + 8 * i, QA_UNITS + (has_lr ? 1 : 0));  // its 4 units + the MMA
+      mbar_init(x_empty0 + 8 * i, QA_UNITS + (has_lr ? 1 : 0));  // its 8 units + the MMA
     }
     for (int i = 0; i < LST; ++i) {
       mbar_init(l_full0 + 8 * i, 1);
       mbar_init(l_empty0 + 8 * i, 1);
+    }
+    for (int i = 0; i < NSTG; ++i) {
+      mbar_init(staged0 + 8 * i, QA_UNITS);
+      mbar_init(free0 + 8 * i, 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(s_bar, 1);
@@ -216,12 +242,13 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
     mbar_fence_init();
-    // rank 0 of a K split expects the other ranks' partial sums
-    if (reduce && split == 0)
-      mbar_arrive_expect_tx(red_bar, (uint32_t)(S - 1) * QA_BM * (uint32_t)r * 4u);
+    // every rank of a K split owns r / S columns and expects the other
+    // ranks' partial sums of them
+    if (reduce) mbar_arrive_expect_tx(red_bar, qa_red_bytes(r, S));
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tm_x);
+    prefetch_tensormap(&tm_codes);
     if (has_lr) prefetch_tensormap(&tm_l1);
   }
   if (warp == 1 && has_lr) {
@@ -267,7 +294,7 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
             !mbar_wait(x_empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid))
           break;
         mbar_arrive_expect_tx(x_full0 + 8 * st, QA_X_BYTES);
-        // (a box past K reads zeros: the TMA fill)
+        // (a box past K or rows past M read zeros: the TMA fill)
         for (int b = 0; b < QA_BOXES; ++b)
           tma_load_2d(smem_u32(smem + st * QA_X_BYTES + b * QA_BOX_BYTES), &tm_x,
                       (c_begin + cl) * 128 + 64 * b, rb * QA_BM, x_full0 + 8 * st);
@@ -295,6 +322,36 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
         if (++st == LST) { st = 0; ph ^= 1; }
         if (++cl == nchunks) cl = 0;
       }
+    }
+    __syncwarp();
+  } else if (warp == 3) {
+    // ------------------------------------------ code / scale stores (TMA) ----
+    // A chunk's slot is written out once its 8 units have staged it; the
+    // slot is handed back when the stores have read it.
+    if (lane == 0) {
+      int cl = rot;
+      for (int i = 0; i < nchunks; ++i) {
+        const int slot = i % NSTG;
+        if (!mbar_wait(staged0 + 8 * slot, (uint32_t)(i / NSTG) & 1u, p.timeout_ns, abort_flag,
+                       (8u << 8) | kid))
+          break;
+        const int c = c_begin + cl;
+        const uint32_t src = smem_u32(smem + L.stg_off + slot * QA_STG_BYTES);
+        // codes: one 128-row x 64-byte box (columns past K/2, rows past M
+        // are clipped by the TMA)
+        tma_store_2d(&tm_codes, src, c * 64, rb * QA_BM);
+        // scales: the chunk's two 512-byte atoms (only the first when the
+        // chunk's second 64 columns lie past K), contiguous in the tiles
+        const int atoms = (2 * c + 1 < k64) ? 2 : 1;
+        bulk_store(p.sf_x + ((size_t)rb * k64 + 2 * c) * 512, src + QA_CODES_STG,
+                   512u * (uint32_t)atoms);
+        bulk_commit_group();
+        bulk_wait_read_all();
+        mbar_arrive(free0 + 8 * slot);
+        if (++cl == nchunks) cl = 0;
+      }
+      // no store may still be reading shared memory (or writing) at exit
+      bulk_wait_all();
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -338,29 +395,34 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
     bool ok = nchunks == 0 || mbar_wait_warp(s_bar, 0, p.timeout_ns, abort_flag, (3u << 8) | kid);
     for (int u = qw; ok && u < QA_UNITS * nchunks; u += QA_QWARPS) {
       const int i = u / QA_UNITS;
-      const int box = (u % QA_UNITS) >> 1;
+      const int box = (u % QA_UNITS) >> 2;
+      const int quarter = u & 3;
       const int cl = i + rot < nchunks ? i + rot : i + rot - nchunks;  // local chunk
       const int st = i % XST;
       const uint32_t ph = (uint32_t)(i / XST) & 1u;
       if (!mbar_wait_warp(x_full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) break;
-      const int row_t = 32 * (u & 1) + lane;
-      const int row = rb * QA_BM + row_t;
+      const int row_t = 32 * quarter + lane;
       const int col0 = (c_begin + cl) * 128 + 64 * box;   // first column of the unit
-      const uint8_t* xrow = smem + st * QA_X_BYTES + box * QA_BOX_BYTES + row_t * 128;
-      // copy this lane's row segment into registers, then hand the stage
-      // back so the next chunk can land while this one is quantized
+      const bool live = col0 < p.K;                       // else the zero box past K
       uint4 xr[8];
+      if (live) {
+        // copy this lane's row segment into registers, then hand the stage
+        // back so the next chunk can land while this one is quantized
+        const uint8_t* xrow = smem + st * QA_X_BYTES + box * QA_BOX_BYTES + row_t * 128;
 #pragma unroll
-      for (int j = 0; j < 8; ++j)
-        xr[j] = *reinterpret_cast<const uint4*>(xrow + ((j ^ (row_t & 7)) << 4));
+        for (int j = 0; j < 8; ++j)
+          xr[j] = *reinterpret_cast<const uint4*>(xrow + ((j ^ (row_t & 7)) << 4));
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) xr[j] = make_uint4(0, 0, 0, 0);
+      }
       // Hand the stage back only after the reads are done and ordered before
       // the next fill.  The fill is a TMA write (async proxy) after these
       // generic-proxy reads of the same bytes: each lane folds its loaded
       // words into one value (its loads have landed), the warp reduces those,
       // every lane fences the generic proxy against the async proxy, and
       // lane 0 releases.  Without the proxy fence an occasional refill
-      // overwrote a stage while a warp's reads of it were still being served
-      // (a few percent of launches had one unit wrong).
+      // overwrote a stage while a warp's reads of it were still being served.
       uint32_t dep = 0;
 #pragma unroll
       for (int j = 0; j < 8; ++j) dep ^= xr[j].x ^ xr[j].y ^ xr[j].z ^ xr[j].w;
@@ -368,53 +430,70 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
       fence_proxy_async_shared();
       __syncwarp();
       if (lane == 0) mbar_arrive_after(x_empty0 + 8 * st, dep);
-      if (col0 >= p.K) continue;  // the zero box past K: nothing to store
-      const float4* sp = reinterpret_cast<const float4*>(s_sm + cl * 128 + 64 * box);
       uint32_t cw[8];
       uint32_t sfw = 0;
+      if (live) {
+        const float4* sp = reinterpret_cast<const float4*>(s_sm + cl * 128 + 64 * box);
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        // 16 products x * s as 8 lane-pairs (one f32x2 multiply each)
-        const uint4 x0 = xr[2 * g], x1 = xr[2 * g + 1];
-        const ulonglong2* sp2 = reinterpret_cast<const ulonglong2*>(sp + 4 * g);
-        const ulonglong2 s0 = sp2[0], s1 = sp2[1], s2 = sp2[2], s3 = sp2[3];
-        uint64_t v[8];
-        v[0] = fmul_f32x2(bf16x2_to_f32x2(x0.x), s0.x);
-        v[1] = fmul_f32x2(bf16x2_to_f32x2(x0.y), s0.y);
-        v[2] = fmul_f32x2(bf16x2_to_f32x2(x0.z), s1.x);
-        v[3] = fmul_f32x2(bf16x2_to_f32x2(x0.w), s1.y);
-        v[4] = fmul_f32x2(bf16x2_to_f32x2(x1.x), s2.x);
-        v[5] = fmul_f32x2(bf16x2_to_f32x2(x1.y), s2.y);
-        v[6] = fmul_f32x2(bf16x2_to_f32x2(x1.z), s3.x);
-        v[7] = fmul_f32x2(bf16x2_to_f32x2(x1.w), s3.y);
-        float m[8];
+        for (int g = 0; g < 4; ++g) {
+          // 16 products x * s as 8 lane-pairs (one f32x2 multiply each)
+          const uint4 x0 = xr[2 * g], x1 = xr[2 * g + 1];
+          const ulonglong2* sp2 = reinterpret_cast<const ulonglong2*>(sp + 4 * g);
+          const ulonglong2 s0 = sp2[0], s1 = sp2[1], s2 = sp2[2], s3 = sp2[3];
+          uint64_t v[8];
+          v[0] = fmul_f32x2(bf16x2_to_f32x2(x0.x), s0.x);
+          v[1] = fmul_f32x2(bf16x2_to_f32x2(x0.y), s0.y);
+          v[2] = fmul_f32x2(bf16x2_to_f32x2(x0.z), s1.x);
+          v[3] = fmul_f32x2(bf16x2_to_f32x2(x0.w), s1.y);
+          v[4] = fmul_f32x2(bf16x2_to_f32x2(x1.x), s2.x);
+          v[5] = fmul_f32x2(bf16x2_to_f32x2(x1.y), s2.y);
+          v[6] = fmul_f32x2(bf16x2_to_f32x2(x1.z), s3.x);
+          v[7] = fmul_f32x2(bf16x2_to_f32x2(x1.w), s3.y);
+          float m[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float lo, hi;
-          unpack_f32x2(v[e], lo, hi);
-          m[e] = fmaxf(fabsf(lo), fabsf(hi));
+          for (int e = 0; e < 8; ++e) {
+            float lo, hi;
+            unpack_f32x2(v[e], lo, hi);
+            m[e] = fmaxf(fabsf(lo), fabsf(hi));
+          }
+          const float a = fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
+                                fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
+          const uint32_t code = cvt_e4m3x2(__fmul_rn(a, gs), 0.0f) & 0xFF;
+          const float q = qlut[code];
+          const uint64_t qq = pack_f32x2(q, q);
+          float t0[8], t1[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            unpack_f32x2(fmul_f32x2(v[e], qq), t0[2 * e], t0[2 * e + 1]);
+            unpack_f32x2(fmul_f32x2(v[4 + e], qq), t1[2 * e], t1[2 * e + 1]);
+          }
+          cw[2 * g] = cvt_e2m1x8(t0);
+          cw[2 * g + 1] = cvt_e2m1x8(t1);
+          sfw |= code << (8 * g);
         }
-        const float a = fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
-                              fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
-        const uint32_t code = cvt_e4m3x2(__fmul_rn(a, gs), 0.0f) & 0xFF;
-        const float q = qlut[code];
-        const uint64_t qq = pack_f32x2(q, q);
-        float t0[8], t1[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          unpack_f32x2(fmul_f32x2(v[e], qq), t0[2 * e], t0[2 * e + 1]);
-          unpack_f32x2(fmul_f32x2(v[4 + e], qq), t1[2 * e], t1[2 * e + 1]);
-        }
-        cw[2 * g] = cvt_e2m1x8(t0);
-        cw[2 * g + 1] = cvt_e2m1x8(t1);
-        sfw |= code << (8 * g);
       }
-      if (row < p.M) {
-        uint4* dst = reinterpret_cast<uint4*>(p.codes_x + (size_t)row * (p.K >> 1) + (col0 >> 1));
-        dst[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-        dst[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      // stage the unit's codes and scales; the slot must have been read out
+      // by the stores of the chunk that used it before
+      const int slot = i % NSTG;
+      if (i >= NSTG &&
+          !mbar_wait_warp(free0 + 8 * slot, (uint32_t)(i / NSTG - 1) & 1u, p.timeout_ns, abort_flag,
+                          (9u << 8) | kid))
+        break;
+      if (live) {
+        const uint32_t sbase = smem_u32(smem + L.stg_off + slot * QA_STG_BYTES);
+        // codes row of 64 bytes, 16-byte chunk c at slot c ^ ((row / 2) % 4)
+        // (the 64-byte swizzle of the store's tensor map); this unit holds
+        // chunks 2 box and 2 box + 1
+        const uint32_t rowb = sbase + (uint32_t)row_t * 64u;
+        const uint32_t sw = (uint32_t)(row_t >> 1) & 3u;
+        st_shared_v4(rowb + (((2u * box) ^ sw) << 4), cw[0], cw[1], cw[2], cw[3]);
+        st_shared_v4(rowb + (((2u * box + 1u) ^ sw) << 4), cw[4], cw[5], cw[6], cw[7]);
+        // scale word of the row in the chunk's atom `box`
+        st_shared_u32(sbase + QA_CODES_STG + (uint32_t)box * 512u + lane * 16u + quarter * 4u, sfw);
       }
-      *reinterpret_cast<uint32_t*>(p.sf_x + sf_tile_off(row, col0 >> 4, p.K)) = sfw;
+      fence_proxy_async_shared();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(staged0 + 8 * slot);
     }
   }
 
@@ -423,68 +502,87 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   if (has_lr && warp >= QA_QWARP0) {
     const bool ok = mbar_wait_warp(acc_full, 0, p.timeout_ns, abort_flag, (4u << 8) | kid);
     tc_fence_after();
-    // M = 64 accumulator: row m sits in lane (m % 16) + 32 (m / 16).  Warp w
-    // reads its lane quarter w % 4; lanes 0..15 hold rows 16 (w % 4) + lane.
+    // M = 128 accumulator: row m sits in tensor-memory lane m; warp w reads
+    // its lane quarter w % 4.  The four warps of one quarter split the r
+    // columns: slot (w - QA_QWARP0) / 4 takes columns [slot r/4, slot r/4 +
+    // r/4), in groups of four.
     const int quad = warp & 3;
-    const int slot = (warp - QA_QWARP0) >> 2;   // 0 .. QA_QWARPS / 4 - 1
-    const int lrow_t = quad * 16 + lane;
-    const int lrow = rb * QA_BM + lrow_t;
-    const bool own = lane < 16;
-    const uint32_t red_base = smem_u32(smem + L.red_off);
+    const int slot = (warp - QA_QWARP0) >> 2;
+    const int cw4 = r / 16;                       // groups of 4 columns per slot
+    const int row_t = quad * 32 + lane;
+    const int row = rb * QA_BM + row_t;
     const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
-    for (int ci = slot; ci < r / 16; ci += QA_QWARPS / 4) {
-      uint32_t hi[16], lo[16];
-      if (ok) {
-        tmem_ld16(tbase + 16 * ci, hi);
-        tmem_ld16(tbase + r + 16 * ci, lo);
-        tmem_wait_ld();
-      } else {
+    const uint32_t red_base = smem_u32(smem + L.red_off);
+    float own[8][4];                              // partials of the groups this rank owns
 #pragma unroll
-        for (int j = 0; j < 16; ++j) hi[j] = lo[j] = 0u;
-      }
-      float part[16];
+    for (int g = 0; g < 8; ++g) {
+      if (g < cw4) {
+        const int col = slot * 4 * cw4 + 4 * g;   // first of the group's 4 columns
+        uint32_t hi[4], lo[4];
+        // (a rank whose share of K is empty contributes zeros: its
+        // accumulator was never written)
+        if (ok && nchunks > 0) {
+          tmem_ld4(tbase + col, hi);
+          tmem_ld4(tbase + r + col, lo);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) part[j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
-      if (!reduce) {
-        if (own && lrow < p.M)
-          store_hi_lo16(part, p.lr_scale, p.xl1 + (size_t)lrow * p.klr + 16 * ci,
-                        p.xl1 + (size_t)lrow * p.klr + r + 16 * ci);
-      } else if (split != 0) {
-        // partial sums [row][r] of rank `split` into rank 0's buffer split-1
-        if (own) {
-          const uint32_t dst = map_to_rank(
-              red_base + 4u * (uint32_t)(((split - 1) * QA_BM + lrow_t) * r + 16 * ci), 0);
-          const uint32_t bar = map_to_rank(red_bar, 0);
-#pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            st_async_v4(dst + 4u * j, part[j], part[j + 1], part[j + 2], part[j + 3], bar);
+          for (int j = 0; j < 4; ++j) hi[j] = lo[j] = 0u;
         }
-      } else {
-        const bool got = mbar_wait_warp(red_bar, 0, p.timeout_ns, abort_flag, (6u << 8) | kid);
-        if (own && lrow < p.M) {
-          if (got) {
-            for (int sr = 1; sr < S; ++sr) {
-              const float4* q4 = reinterpret_cast<const float4*>(
-                  smem + L.red_off + 4u * (uint32_t)(((sr - 1) * QA_BM + lrow_t) * r + 16 * ci));
 #pragma unroll
-              for (int j = 0; j < 4; ++j) {
-                const float4 t = q4[j];
-                part[4 * j] += t.x;
-                part[4 * j + 1] += t.y;
-                part[4 * j + 2] += t.z;
-                part[4 * j + 3] += t.w;
-              }
-            }
+        for (int j = 0; j < 4; ++j) own[g][j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
+        if (reduce) {
+          const int owner = col / own_cols;
+          if (owner != split) {
+            // into the owner's buffer: [sender slot][128 rows][own_cols]
+            const int sslot = split < owner ? split : split - 1;
+            const uint32_t off = 4u * (uint32_t)((sslot * QA_BM + row_t) * own_cols +
+                                                 (col - owner * own_cols));
+            st_async_v4(map_to_rank(red_base + off, (uint32_t)owner), own[g][0], own[g][1],
+                        own[g][2], own[g][3], map_to_rank(red_bar, (uint32_t)owner));
           }
-          store_hi_lo16(part, p.lr_scale, p.xl1 + (size_t)lrow * p.klr + 16 * ci,
-                        p.xl1 + (size_t)lrow * p.klr + r + 16 * ci);
         }
       }
     }
-    // zero columns [2r, klr) of the rows this CTA finishes
-    if (split == 0 && slot == 0 && own && lrow < p.M) {
+    // finish the owned groups: the S partials added in rank order
+    const bool got = !reduce || mbar_wait_warp(red_bar, 0, p.timeout_ns, abort_flag, (6u << 8) | kid);
+#pragma unroll
+    for (int g = 0; g < 8; ++g) {
+      if (g < cw4) {
+        const int col = slot * 4 * cw4 + 4 * g;
+        if (reduce && col / own_cols != split) continue;
+        float sum[4];
+        if (reduce) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) sum[j] = 0.0f;
+          for (int sr = 0; sr < S; ++sr) {
+            float t[4];
+            if (sr == split || !got) {
+#pragma unroll
+              for (int j = 0; j < 4; ++j) t[j] = sr == split ? own[g][j] : 0.0f;
+            } else {
+              const int sslot = sr < split ? sr : sr - 1;
+              const float4 v = *reinterpret_cast<const float4*>(
+                  smem + L.red_off +
+                  4u * (uint32_t)((sslot * QA_BM + row_t) * own_cols + (col - split * own_cols)));
+              t[0] = v.x; t[1] = v.y; t[2] = v.z; t[3] = v.w;
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) sum[j] = sr == 0 ? t[j] : sum[j] + t[j];
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) sum[j] = own[g][j];
+        }
+        if (row < p.M)
+          store_hi_lo4(sum, p.lr_scale, p.xl1 + (size_t)row * p.klr + col,
+                       p.xl1 + (size_t)row * p.klr + r + col);
+      }
+    }
+    // zero columns [2r, klr) of this row block
+    if (split == 0 && slot == 0 && row < p.M) {
       for (int cpad = 2 * r; cpad < p.klr; cpad += 8)
-        *reinterpret_cast<uint4*>(p.xl1 + (size_t)lrow * p.klr + cpad) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(p.xl1 + (size_t)row * p.klr + cpad) = make_uint4(0, 0, 0, 0);
     }
   }
 

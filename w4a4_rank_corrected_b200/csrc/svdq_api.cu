@@ -121,17 +121,16 @@ svdq_status device_check(int* sms) {
 }
 
 // 2D tensor map over a row-major [rows][inner] matrix (128-byte swizzle
-// unless `swizzle` is false).
+// unless `swizzle` says otherwise).
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner,
               uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
-              bool swizzle = true) {
+              CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   const cuuint64_t dims[2] = {inner, rows};
   const cuuint64_t strides[1] = {row_bytes};
   const cuuint32_t box[2] = {box_inner, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return g_encode(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -161,15 +160,18 @@ cudaLaunchAttribute pdl_attr() {
   return a;
 }
 
-// Largest K split S (cluster size when the low-rank branch needs the
-// cross-CTA reduction) such that the whole grid is resident in one wave and
-// the split's shared-memory plan keeps a deep enough activation ring.
+// Largest K split S in {1, 2, 4, 8} (the cluster size when the low-rank
+// branch needs the cross-CTA reduction) such that the whole grid is resident
+// in one wave, the split's shared-memory plan keeps a deep enough activation
+// ring, and (with a low-rank branch) every rank owns a whole number of
+// 4-column groups of the result (r % S == 0, (r / S) % 4 == 0).
 int choose_splits(int tiles, int kchunks, int r, int sms) {
   int dev = 0;
   cudaGetDevice(&dev);
   int best = 1;
-  for (int S = 2; S <= 8; ++S) {
+  for (int S = 2; S <= 8; S *= 2) {
     if (S > kchunks || tiles * S > sms) break;
+    if (r > 0 && (r % S != 0 || (r / S) % 4 != 0)) break;
     const int cps = (kchunks + S - 1) / S;
     const QALayout L = qa_layout(r, cps, S);
     if (L.xst < QA_MIN_XST) break;
@@ -207,20 +209,23 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
                             uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, cudaStream_t s,
                             int sms) {
   const int K = w->K, r = w->r;
-  // 64-row tiles covering whole 128-row scale atoms (padding rows get zero
+  // 128-row tiles: one scale-factor atom row each (padding rows get zero
   // scales)
-  const int tiles = 2 * ((M + 127) / 128);
+  const int tiles = (M + QA_BM - 1) / QA_BM;
   const int KC = (K / 64 + QA_BOXES - 1) / QA_BOXES;  // 128-column chunks
   int S = choose_splits(tiles, KC, r, sms);
   const int cps = (KC + S - 1) / S;
-  S = (KC + cps - 1) / cps;
   const QALayout L = qa_layout(r, cps, S);
-  if (L.xst < QA_MIN_XST) return SVDQ_ERR_INVALID_ARG;  // K too large for one CTA's slice
-
-  CUtensorMap tm_x, tm_l1;
+  if (L.xst < QA_MIN_XST || L.nstg < QA_MIN_NSTG || (r > 0 && L.lst < 1))
+    return SVDQ_ERR_INVALID_ARG;  // K too large for one CTA's slice
+  CUtensorMap tm_x, tm_l1, tm_codes;
   std::memset(&tm_l1, 0, sizeof(tm_l1));
   if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M,
                 (uint64_t)ldx * 2, 64, QA_BM))
+    return SVDQ_ERR_CUDA;
+  // codes are stored in 128-row x 64-byte boxes, 64-byte swizzle
+  if (!make_map(&tm_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_x, (uint64_t)K / 2, (uint64_t)M,
+                (uint64_t)K / 2, 64, QA_BM, CU_TENSOR_MAP_SWIZZLE_64B))
     return SVDQ_ERR_CUDA;
   if (r > 0 && !make_map(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l1_mma, (uint64_t)K,
                          (uint64_t)(2 * r), (uint64_t)K * 2, 64, (uint32_t)(2 * r)))
@@ -228,7 +233,6 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
 
   QAParams p;
   p.smooth = w->smooth;
-  p.codes_x = codes_x;
   p.sf_x = sf_x;
   p.xl1 = xl1;
   p.M = M;
@@ -237,7 +241,7 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
   p.klr = klr_of(r);
   p.chunks_per_split = cps;
   p.num_splits = S;
-  p.L = L;
+  p.L = qa_layout(r, cps, S);
   uint32_t cols = 32;
   while (cols < (uint32_t)(2 * r)) cols <<= 1;
   p.tmem_cols = cols;
@@ -250,7 +254,7 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)S, (unsigned)tiles, 1);
   cfg.blockDim = dim3(QA_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = L.total;
+  cfg.dynamicSmemBytes = p.L.total;
   cfg.stream = s;
   cudaLaunchAttribute attr[2];
   attr[0] = pdl_attr();
@@ -263,7 +267,7 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
   }
-  if (cudaLaunchKernelEx(&cfg, quantize_act_kernel, tm_x, tm_l1, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, quantize_act_kernel, tm_x, tm_l1, tm_codes, p) != cudaSuccess) {
     cudaGetLastError();
     return SVDQ_ERR_CUDA;
   }
@@ -307,13 +311,16 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   std::memset(&tblr, 0, sizeof(tblr));
   // scale buffers as rows of 256 bytes (half a 512-byte atom), unswizzled
   const uint64_t sfa_rows = rup((size_t)M, 128) * (K / 16) / 256;
-  const uint64_t sfb_rows = rup((size_t)N, 256) * (K / 16) / 256;
+  // weight scales: two atom rows per 192-row tile
+  const uint64_t sfb_rows = (uint64_t)((N + G_BN - 1) / G_BN) * G_SFB_ROWS * (K / 16) / 256;
   if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_x, (uint64_t)K / 2, (uint64_t)M,
                 (uint64_t)K / 2, 128, G_BM) ||
       !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes_w, (uint64_t)K / 2, (uint64_t)N,
                 (uint64_t)K / 2, 128, G_BN_CTA) ||
-      !make_map(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT8, sf_x, 256, sfa_rows, 256, 256, 8, false) ||
-      !make_map(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->sf_w, 256, sfb_rows, 256, 256, 8, false) ||
+      !make_map(&tsa, CU_TENSOR_MAP_DATA_TYPE_UINT8, sf_x, 256, sfa_rows, 256, 256, 8,
+                CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_map(&tsb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->sf_w, 256, sfb_rows, 256, 256, 8,
+                CU_TENSOR_MAP_SWIZZLE_NONE) ||
       // Y is written in 128-row x 64-column boxes (128-byte swizzle)
       !make_map(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, (uint64_t)N, (uint64_t)M,
                 (uint64_t)ldy * 2, G_OUT_COLS, G_BM))
