@@ -246,11 +246,12 @@ def run_ours(args):
     sfs = [torch.empty(sf_bytes, dtype=torch.uint8, device=dev) for _ in range(nsets)]
     xl1s = [torch.empty((M, klr), dtype=torch.bfloat16, device=dev) if r else None
             for _ in range(nsets)]
+    scratches = [S.new_act_scratch(M, K, r, dev) for _ in range(nsets)]
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
         j = i % nsets
-        S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j], stream)
+        S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j], stream, scratches[j])
         S.svdq_gemm(weights[j], codes[j], sfs[j], xl1s[j], M, Ys[j], stream)
 
     sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ
@@ -276,7 +277,8 @@ def run_ours(args):
             for j in range(nsets):
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g):
-                    S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j])
+                    S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j],
+                                        scratch=scratches[j])
                     S.svdq_gemm(weights[j], codes[j], sfs[j], xl1s[j], M, Ys[j])
                 graphs.append(g)
             for j in range(nsets):
@@ -339,8 +341,8 @@ def run_ours(args):
     if args.kernel_seconds > 0 or args.kernel_launches > 0:
         kt = dict(min_launches=max(1, args.kernel_launches), min_seconds=args.kernel_seconds)
         q_ms, q_n = kernel_time_ms(lambda i: S.svdq_quantize_act(
-            weights[i % nsets], Xs[i % nsets], codes[i % nsets], sfs[i % nsets], xl1s[i % nsets]),
-            **kt)
+            weights[i % nsets], Xs[i % nsets], codes[i % nsets], sfs[i % nsets], xl1s[i % nsets],
+            scratch=scratches[i % nsets]), **kt)
         g_ms, g_n = kernel_time_ms(lambda i: S.svdq_gemm(
             weights[i % nsets], codes[i % nsets], sfs[i % nsets], xl1s[i % nsets], M,
             Ys[i % nsets]), **kt)

@@ -76,7 +76,7 @@ typedef struct svdq_sizes {
   size_t l1_mma_bytes;   /* bf16 [2r][K]      kernel operand, see pack     */
   size_t l2_mma_bytes;   /* bf16 [N][klr]     kernel operand, see pack     */
   size_t codes_w_bytes;  /* u8   [N][K/2]     E2M1 codes of R              */
-  size_t sf_w_bytes;     /* u8   MMA tiles    E4M3 scales of R, ceil(N/192) * 256 rows */
+  size_t sf_w_bytes;     /* u8   MMA tiles    E4M3 scales of R (rows padded to 256) */
   size_t bias_bytes;     /* bf16 [N]                                       */
 } svdq_sizes;
 
@@ -134,8 +134,7 @@ typedef struct svdq_packed_host {
   uint16_t* l1_mma;      /* [2r][K]    */
   uint16_t* l2_mma;      /* [N][klr]   */
   uint8_t*  codes_w;     /* [N][K/2], even k in the low nibble             */
-  uint8_t*  sf_w;        /* MMA tile layout, weight row n at atom-layout
-                            row svdq_weight_sf_row(n)                      */
+  uint8_t*  sf_w;        /* MMA tile layout (svdq_sf_tile_offset)          */
   uint16_t* bias;        /* [N] bf16, or NULL                              */
   float amax_x, amax_w;  /* static activation absmax A_x, residual absmax A_w */
   float g_x, gs_x, g_w, alpha, lr_scale;
@@ -156,13 +155,6 @@ svdq_status svdq_pack_weight(const float* W, const float* x_absmax,
  * table of "Bringing Nunchaku 4-bit diffusion inference to Diffusers").
  */
 int64_t svdq_sf_tile_offset(int row, int g, int K);
-
-/* Row of that atom layout that holds the scales of weight row n: the GEMM
- * reads the weight in tiles of 192 rows, each with two atom rows of its own
- * (rows 0-127 and 128-191 of the tile, the second padded with 64 zero rows),
- * so weight row n sits at (n / 192) * 256 + n % 192.  sf_w holds
- * ceil(N / 192) * 256 rows.  -1 for n < 0. */
-int svdq_weight_sf_row(int n);
 
 /* svdq_unswizzle_scales: host permutation from the MMA tile layout back to
  * plain row-major scales, sf_rowmajor[row][g] = sf_mma[svdq_sf_tile_offset(
@@ -185,12 +177,25 @@ typedef struct svdq_weight {
   const uint16_t* l2_mma;   /* device bf16 [N][klr]       (NULL if r == 0) */
   const uint16_t* bias;     /* device bf16 [N] or NULL                     */
   const uint8_t*  codes_w;  /* device u8 [N][K/2]                          */
-  const uint8_t*  sf_w;     /* device u8, MMA tiles, ceil(N/192)*256 rows  */
+  const uint8_t*  sf_w;     /* device u8, MMA tiles, rows padded to 256    */
 } svdq_weight;
 
-/* Bytes of the activation workspace for M tokens: codes_x [M][K/2],
- * sf_x (MMA tiles, rows padded to 128) and xl1 [M][klr] bf16, each region
- * 256-byte aligned.  0 on bad arguments. */
+/* Bytes of the activation kernel's scratch for M tokens (0 when r == 0):
+ * a K split of the activation kernel needs it for its low-rank partial
+ * sums.  Layout: 4096 bytes of arrival counters (one 32-bit word per 128-row
+ * block) followed by fp32 partial sums.  The counters must be ZERO before
+ * the scratch's first use; every launch that completes leaves them zero
+ * again, so a scratch buffer is zeroed once when it is allocated (after a
+ * SVDQ_ERR_TIMEOUT from svdq_device_error, zero it again).  0 on bad
+ * arguments. */
+size_t svdq_act_scratch_bytes(int M, int K, int r);
+
+/* Bytes of the forward's workspace for M tokens: the activation scratch
+ * (first, counters at offset 0), codes_x [M][K/2], sf_x (MMA tiles, rows
+ * padded to 128) and xl1 [M][klr] bf16, each region 256-byte aligned.  The
+ * first 4096 bytes must be zero before the workspace's first use (see
+ * svdq_act_scratch_bytes); the library leaves them zero.  0 on bad
+ * arguments. */
 size_t svdq_act_workspace_bytes(int M, int K, int r);
 
 /* svdq_quantize_act: activation kernel (one launch).
@@ -209,13 +214,16 @@ size_t svdq_act_workspace_bytes(int M, int K, int r);
  *   codes_x  device u8 [M][K/2]
  *   sf_x     device u8, MMA tiles, round_up(M,128) * K/16 bytes (pad rows 0)
  *   xl1      device bf16 [M][klr] (may be NULL if r == 0)
+ *   scratch  device, >= svdq_act_scratch_bytes(M, K, r), 256-byte aligned,
+ *            counters zeroed (see above); NULL (or too small) runs the kernel
+ *            without splitting K, which is slower for M below ~18000.
  * Reads X exactly once.  Returns SVDQ_ERR_INVALID_ARG when one CTA's share
- * of K does not fit its shared-memory plan (for large M, where K is split at
- * most two ways: K above roughly 36000 at r <= 32, 24000 at r = 128).
+ * of K does not fit its shared-memory plan (K above roughly 36000).
  */
 svdq_status svdq_quantize_act(const svdq_weight* w, const uint16_t* X, int M,
                               int64_t ldx, uint8_t* codes_x, uint8_t* sf_x,
-                              uint16_t* xl1, void* stream);
+                              uint16_t* xl1, void* scratch, size_t scratch_bytes,
+                              void* stream);
 
 /* svdq_gemm: the 4-bit GEMM kernel (one launch).
  * Source: the Korean rendering of "Bringing Nunchaku 4-bit diffusion
@@ -235,7 +243,8 @@ svdq_status svdq_gemm(const svdq_weight* w, const uint8_t* codes_x,
  * + bias ("Background: SVDQuant and Nunchaku"; the runtime SVDQW4A4Linear
  * layer that replaces nn.Linear in "Loading natively in Diffusers"):
  * svdq_quantize_act then svdq_gemm on one stream, with the intermediates in
- * `workspace` (device, >= svdq_act_workspace_bytes, 256-byte aligned). */
+ * `workspace` (device, >= svdq_act_workspace_bytes, 256-byte aligned, its
+ * first 4096 bytes zero before its first use). */
 svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t* X,
                                 int M, int64_t ldx, uint16_t* Y, int64_t ldy,
                                 void* workspace, size_t ws_bytes,
@@ -275,9 +284,11 @@ svdq_status svdq_linear_forward_host(const svdq_weight* w, const uint16_t* X_hos
  *     library's device code on the device.
  *   - M is limited by the scratch size: svdq_act_workspace_bytes(M, K, r)
  *     must be <= SVDQ_STATIC_WORKSPACE_BYTES, else SVDQ_ERR_WORKSPACE and
- *     nothing is launched (e.g. K = 3072, r = 32 allows M <= 9033).
- *   - Nothing in the scratch needs to start at zero: the activation kernel
- *     writes every byte the GEMM reads, padding rows included.
+ *     nothing is launched (e.g. K = 3072, r = 32 allows M <= 7618).
+ *   - The scratch starts zeroed (a module's device variables are zero when
+ *     it loads) and every call that completes leaves the activation
+ *     kernel's arrival counters at its start zero again; everything else in
+ *     it is written before it is read.
  *   - One scratch area per device: calls that overlap in time (different
  *     streams, or threads without ordering) race on it.  Calls in order on
  *     one stream are safe.

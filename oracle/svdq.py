@@ -45,9 +45,7 @@ Readings of what the pages leave open:
      the method's own 4-bit encodings; 1/(g_x g_w) undoes both tensor
      scales).
   R7 packed layouts: codes are two per byte, the even k in the low nibble;
-     block scales in the MMA tile layout (see `sf_to_mma_tiles`); the
-     weight's scales with each 192-row tile padded to 256 rows
-     (`sf_to_weight_tiles`).
+     block scales in the MMA tile layout (see `sf_to_mma_tiles`).
   R11f GELU between the MLP pair's layers, in a form a fused kernel and this
      oracle evaluate bit-identically: the tanh form of GELU,
        0.5 y (1 + tanh(u)),  u = sqrt(2/pi) (y + 0.044715 y^3),
@@ -227,21 +225,6 @@ def sf_to_mma_tiles(sf: np.ndarray, row_multiple: int = 128) -> np.ndarray:
     t = padded.reshape(nb, 4, 32, kb, 4)          # [b, q, p, c, j]
     t = t.transpose(0, 3, 2, 1, 4)                # [b, c, p, q, j]
     return np.ascontiguousarray(t).reshape(-1)
-
-
-def sf_to_weight_tiles(sf: np.ndarray, tile_rows: int = 192) -> np.ndarray:
-    """The weight's scales as the GEMM reads them (reading R7): the weight
-    is taken in tiles of `tile_rows` (192) rows, and each tile gets two atom
-    rows of its own (256 rows, the last 64 left zero), so weight row n sits
-    at row (n // 192) * 256 + n % 192 of the `sf_to_mma_tiles` layout."""
-    sf = np.asarray(sf, dtype=np.uint8)
-    rows, nsf = sf.shape
-    nt = -(-rows // tile_rows)
-    padded = np.zeros((nt * 256, nsf), dtype=np.uint8)
-    for t in range(nt):
-        n0, n1 = t * tile_rows, min(rows, (t + 1) * tile_rows)
-        padded[t * 256:t * 256 + (n1 - n0)] = sf[n0:n1]
-    return sf_to_mma_tiles(padded, row_multiple=256)
 
 
 def sf_from_mma_tiles(tiled: np.ndarray, rows: int, K: int) -> np.ndarray:

@@ -36,7 +36,7 @@ def prepare(W, cx, r, bias=None, seed=0):
         op = O.pack(W, cx, 0)
     assert np.array_equal(lp.smooth, op.s)
     assert np.array_equal(lp.codes_w, O.pack_nibbles(op.codes_w))
-    assert np.array_equal(lp.sf_w, O.sf_to_weight_tiles(op.sf_w))
+    assert np.array_equal(lp.sf_w, O.sf_to_mma_tiles(op.sf_w, row_multiple=256))
     return lp, op, lp.to_device("cuda", bias)
 
 

@@ -40,7 +40,7 @@ def test_query_sizes():
     sz = S.svdq_query_sizes(9216, 3072, 32)
     assert (sz.N, sz.K, sz.r, sz.klr) == (9216, 3072, 32, 64)
     assert sz.codes_w_bytes == 9216 * 1536
-    assert sz.sf_w_bytes == 48 * 256 * 192       # 48 tiles of 192 rows, 256 rows each
+    assert sz.sf_w_bytes == 9216 * 192
     sz = S.svdq_query_sizes(48, 192, 16)
     assert sz.klr == 64 and sz.sf_w_bytes == 256 * 12
     for bad in [(9216, 3000, 32), (9210, 3072, 32), (9216, 3072, 40), (9216, 3072, 144),
@@ -62,22 +62,14 @@ def test_sf_tile_offset_matches_oracle_layout():
     assert S.svdq_sf_tile_offset(0, 0, 100) == -1
 
 
-def test_weight_sf_row_matches_oracle_layout():
-    rng = np.random.default_rng(1)
-    N, K = 496, 256
-    sf = rng.integers(0, 127, (N, K // 16)).astype(np.uint8)
-    tiled = O.sf_to_weight_tiles(sf)
-    assert tiled.size == S.svdq_query_sizes(N, K, 16).sf_w_bytes
-    for _ in range(1000):
-        n, g = int(rng.integers(N)), int(rng.integers(K // 16))
-        assert tiled[S.svdq_sf_tile_offset(S.lib.svdq_weight_sf_row(n), g, K)] == sf[n, g]
-    assert S.lib.svdq_weight_sf_row(-1) == -1
-
-
 def test_workspace_bytes():
     M, K, r = 4608, 3072, 32
     ws = S.svdq_act_workspace_bytes(M, K, r)
-    assert ws >= M * K // 2 + M * K // 16 + M * 64 * 2
+    sc = S.svdq_act_scratch_bytes(M, K, r)
+    # counters, then the partial sums of up to 8 ranks (at most 160 row blocks in all)
+    assert sc == 4096 + min(8 * 4608, 160 * 128) * 32 * 4
+    assert S.svdq_act_scratch_bytes(M, K, 0) == 0
+    assert ws >= sc + M * K // 2 + M * K // 16 + M * 64 * 2
     assert ws % 256 == 0
     assert S.svdq_act_workspace_bytes(100, 3000, 32) == 0
 
@@ -96,15 +88,17 @@ def test_argument_validation_before_any_launch():
     w = _fake_weight()
     X, C, SF, XL = 0x20000000, 0x30000000, 0x40000000, 0x50000000
     # null weight / null pointers / bad shapes
-    assert L.svdq_quantize_act(None, X, 16, 256, C, SF, XL, None) == 1
-    assert L.svdq_quantize_act(ctypes.byref(w), None, 16, 256, C, SF, XL, None) == 1
-    assert L.svdq_quantize_act(ctypes.byref(w), X, -1, 256, C, SF, XL, None) == 1
-    assert L.svdq_quantize_act(ctypes.byref(w), X, 16, 128, C, SF, XL, None) == 1  # ldx < K
+    SC, NS = 0x58000000, S.svdq_act_scratch_bytes(16, 256, 32)
+    assert L.svdq_quantize_act(None, X, 16, 256, C, SF, XL, SC, NS, None) == 1
+    assert L.svdq_quantize_act(ctypes.byref(w), None, 16, 256, C, SF, XL, SC, NS, None) == 1
+    assert L.svdq_quantize_act(ctypes.byref(w), X, -1, 256, C, SF, XL, SC, NS, None) == 1
+    assert L.svdq_quantize_act(ctypes.byref(w), X, 16, 128, C, SF, XL, SC, NS, None) == 1  # ldx < K
     bad = _fake_weight(K=200)
-    assert L.svdq_quantize_act(ctypes.byref(bad), X, 16, 256, C, SF, XL, None) == 1
+    assert L.svdq_quantize_act(ctypes.byref(bad), X, 16, 256, C, SF, XL, SC, NS, None) == 1
     # misalignment
-    assert L.svdq_quantize_act(ctypes.byref(w), X + 2, 16, 256, C, SF, XL, None) == 3
-    assert L.svdq_quantize_act(ctypes.byref(w), X, 16, 260, C, SF, XL, None) == 3
+    assert L.svdq_quantize_act(ctypes.byref(w), X + 2, 16, 256, C, SF, XL, SC, NS, None) == 3
+    assert L.svdq_quantize_act(ctypes.byref(w), X, 16, 260, C, SF, XL, SC, NS, None) == 3
+    assert L.svdq_quantize_act(ctypes.byref(w), X, 16, 256, C, SF, XL, SC + 16, NS, None) == 3
     assert L.svdq_gemm(ctypes.byref(w), C, SF, XL, 16, 0x60000008, 256, None) == 3
     mis = _fake_weight(base=0x10000004)
     assert L.svdq_gemm(ctypes.byref(mis), C, SF, XL, 16, 0x60000000, 256, None) == 3

@@ -224,11 +224,56 @@ def test_activation_kernel_repeats_bit_identical():
     X, W, b = SI.random_layer(24, M, K, N)
     lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
     Xd = to_dev_bf16(X)
-    c0, s0, x0 = (t.clone() for t in S.svdq_quantize_act(dw, Xd))
+    scratch = S.new_act_scratch(M, K, r)
+    c0, s0, x0 = (t.clone() for t in S.svdq_quantize_act(dw, Xd, scratch=scratch))
     for _ in range(20):
-        c, sf, xl1 = S.svdq_quantize_act(dw, Xd)
+        c, sf, xl1 = S.svdq_quantize_act(dw, Xd, scratch=scratch)
         assert torch.equal(c, c0) and torch.equal(sf, s0)
         assert torch.equal(xl1.view(torch.int16), x0.view(torch.int16))
+    # the K split's arrival counters are back at zero after every launch
+    assert int(scratch[:4096].count_nonzero()) == 0
+
+
+@pytest.mark.parametrize("M,K,r", [(4608, 3072, 32), (256, 3072, 32), (300, 1024, 16),
+                                   (1000, 1536, 64)])
+def test_activation_kernel_split_matches_unsplit(M, K, r):
+    """The activation kernel with its K split (scratch given) and without
+    (no scratch: one CTA per row block walks all of K): the same codes and
+    scales bit for bit; the low-rank operand differs only by the order of
+    the fp32 additions."""
+    import ctypes
+    S = _S()
+    X, W, b = SI.random_layer(M + K + r, M, K, 64)
+    lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
+    Xd = to_dev_bf16(X)
+    c1, s1, x1 = S.svdq_quantize_act(dw, Xd)
+    c2 = torch.empty_like(c1)
+    s2 = torch.zeros_like(s1)
+    x2 = torch.empty_like(x1)
+    st = S.lib.svdq_quantize_act(ctypes.byref(dw.struct), Xd.data_ptr(), M, K, c2.data_ptr(),
+                                 s2.data_ptr(), x2.data_ptr(), None, 0,
+                                 torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    torch.cuda.synchronize()
+    assert torch.equal(c1, c2) and torch.equal(s1, s2)
+    check_activation(c2, s2, x2, X, op, M, K, r)
+    a = F.bf16_bits_to_f64(from_dev_bf16(x1)[:, :r]) + F.bf16_bits_to_f64(from_dev_bf16(x1)[:, r:2 * r])
+    c = F.bf16_bits_to_f64(from_dev_bf16(x2)[:, :r]) + F.bf16_bits_to_f64(from_dev_bf16(x2)[:, r:2 * r])
+    assert np.max(np.abs(a - c)) <= 1e-5 * np.max(np.abs(c))
+
+
+def test_activation_scratch_counters_not_zeroed_is_reported():
+    """A scratch whose arrival counters were not zeroed is caught: the kernel
+    records error code (10 << 8) | 1, which svdq_device_error returns."""
+    S = _S()
+    M, K, r = 4608, 3072, 32
+    X, W, b = SI.random_layer(41, M, K, 64)
+    lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
+    scratch = S.new_act_scratch(M, K, r)
+    scratch[:4096].fill_(0x7F)                # counters far above any split count
+    S.svdq_quantize_act(dw, to_dev_bf16(X), scratch=scratch)
+    assert S.svdq_device_error() == (10 << 8) | 1
+    assert S.svdq_device_error() == 0
 
 
 # ---------------------------------------------------- full-size workloads ----

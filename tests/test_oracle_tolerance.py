@@ -112,22 +112,3 @@ def test_sf_atom_golden_offsets(golden_dir):
     tp = O.sf_to_mma_tiles(pad)
     assert int(tp.sum()) == rows * G
 
-
-def test_weight_scale_tiles_place_rows_by_hand():
-    """The GEMM's weight-scale layout: 192-row tiles, each padded to two atom
-    rows.  Hand-placed rows: weight row 0 -> atom-layout row 0; 191 -> 191;
-    192 -> 256 (second tile); 200 -> 264; 383 -> 447; rows 192..255 of the
-    layout (the first tile's padding) hold zeros."""
-    K = 64
-    rows = 400
-    G = K // 16
-    sf = np.zeros((rows, G), np.uint8)
-    for n in range(rows):
-        sf[n, :] = 1 + (n % 200)
-    tiled = O.sf_to_weight_tiles(sf)
-    assert tiled.size == 3 * 256 * G                   # ceil(400 / 192) = 3 tiles
-    flat_rows = O.sf_from_mma_tiles(tiled, 3 * 256, K)
-    for n, row in [(0, 0), (191, 191), (192, 256), (200, 264), (383, 447), (384, 512), (399, 527)]:
-        assert np.array_equal(flat_rows[row], sf[n]), (n, row)
-    assert not flat_rows[192:256].any() and not flat_rows[448:512].any()
-    assert not flat_rows[528:].any()

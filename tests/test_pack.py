@@ -25,7 +25,7 @@ def _check_pack(W, cx, r, svd_quality=True):
     assert np.float32(p.amax_w) == A_w
     assert np.float32(p.g_w) == O.tensor_encode_scale(A_w)
     assert np.array_equal(p.codes_w, O.pack_nibbles(codes))
-    assert np.array_equal(p.sf_w, O.sf_to_weight_tiles(sf))
+    assert np.array_equal(p.sf_w, O.sf_to_mma_tiles(sf, row_multiple=256))
     assert np.float32(p.lr_scale) == np.float32(np.float32(p.g_x) * np.float32(p.g_w))
     assert np.float32(p.alpha) == np.float32(np.float32(1.0) / np.float32(p.lr_scale))
     if r == 0:

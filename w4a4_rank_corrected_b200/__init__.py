@@ -26,6 +26,7 @@ __all__ = [
     "SvdqError", "PackedWeight", "DeviceWeight", "svdq_query_sizes", "svdq_pack_weight",
     "svdq_quantize_act", "svdq_gemm", "svdq_linear_forward", "svdq_act_workspace_bytes",
     "svdq_linear_forward_host", "svdq_linear_forward_static", "svdq_unswizzle_scales",
+    "svdq_act_scratch_bytes", "new_workspace", "new_act_scratch",
     "svdq_device_error", "svdq_selftest_timeout", "svdq_debug_convert", "svdq_sf_tile_offset",
     "svdq_status_string", "SVDQW4A4Linear", "lib", "STATUS",
 ]
@@ -86,9 +87,9 @@ def _load() -> ctypes.CDLL:
         "svdq_linear_forward_host": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P, P, P,
                                          SZ, P]),
         "svdq_sf_tile_offset": (I64, [I, I, I]),
-        "svdq_weight_sf_row": (I, [I]),
         "svdq_act_workspace_bytes": (SZ, [I, I, I]),
-        "svdq_quantize_act": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P, P, P]),
+        "svdq_act_scratch_bytes": (SZ, [I, I, I]),
+        "svdq_quantize_act": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P, P, P, SZ, P]),
         "svdq_gemm": (I, [ctypes.POINTER(SvdqWeight), P, P, P, I, P, I64, P]),
         "svdq_linear_forward": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P, SZ, P]),
         "svdq_linear_forward_static": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P]),
@@ -127,6 +128,25 @@ def svdq_sf_tile_offset(row: int, g: int, K: int) -> int:
 
 def svdq_act_workspace_bytes(M: int, K: int, r: int) -> int:
     return int(lib.svdq_act_workspace_bytes(M, K, r))
+
+
+def svdq_act_scratch_bytes(M: int, K: int, r: int) -> int:
+    return int(lib.svdq_act_scratch_bytes(M, K, r))
+
+
+def new_workspace(M: int, K: int, r: int, device="cuda"):
+    """A forward workspace, zeroed (its arrival counters must start at zero;
+    the library leaves them zero after every call)."""
+    import torch
+    return torch.zeros(max(svdq_act_workspace_bytes(M, K, r), 256), dtype=torch.uint8,
+                       device=device)
+
+
+def new_act_scratch(M: int, K: int, r: int, device="cuda"):
+    """Scratch for svdq_quantize_act, zeroed; None when r == 0."""
+    import torch
+    n = svdq_act_scratch_bytes(M, K, r)
+    return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
 
 
 # ---------------------------------------------------------------- pack ----
@@ -290,8 +310,11 @@ def _keep_alive_on(stream, *tensors):
             t.record_stream(stream)
 
 
-def svdq_quantize_act(w: DeviceWeight, X, codes_x=None, sf_x=None, xl1=None, stream=None):
-    """Returns (codes_x u8 [M, K/2], sf_x u8 tiles, xl1 bf16 [M, klr] or None)."""
+def svdq_quantize_act(w: DeviceWeight, X, codes_x=None, sf_x=None, xl1=None, stream=None,
+                      scratch=None):
+    """Returns (codes_x u8 [M, K/2], sf_x u8 tiles, xl1 bf16 [M, klr] or None).
+    `scratch` (from new_act_scratch) lets the kernel split K; one is made
+    here when not given."""
     import torch
     _check_x(X, w.K)
     M = X.shape[0]
@@ -307,8 +330,12 @@ def svdq_quantize_act(w: DeviceWeight, X, codes_x=None, sf_x=None, xl1=None, str
     if xl1 is None and w.r > 0:
         xl1 = torch.empty((M, klr), dtype=torch.bfloat16, device=dev)
         made.append(xl1)
+    if scratch is None and w.r > 0:
+        scratch = new_act_scratch(M, w.K, w.r, dev)
+        made.append(scratch)
     _check(lib.svdq_quantize_act(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
-                                 codes_x.data_ptr(), sf_x.data_ptr(), _ptr(xl1),
+                                 codes_x.data_ptr(), sf_x.data_ptr(), _ptr(xl1), _ptr(scratch),
+                                 0 if scratch is None else scratch.numel(),
                                  _stream_ptr(stream)), "svdq_quantize_act")
     _keep_alive_on(stream, *made)
     return codes_x, sf_x, xl1
@@ -335,9 +362,8 @@ def svdq_linear_forward(w: DeviceWeight, X, Y=None, workspace=None, stream=None)
     if Y is None:
         Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
         made.append(Y)
-    need = svdq_act_workspace_bytes(M, w.K, w.r)
     if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+        workspace = new_workspace(M, w.K, w.r, X.device)
         made.append(workspace)
     _check(lib.svdq_linear_forward(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
                                    Y.data_ptr(), Y.stride(0), workspace.data_ptr(),
@@ -402,8 +428,7 @@ class HostStreamer:
         self.w, self.M = w, M
         self.X = [torch.empty((M, w.K), dtype=torch.bfloat16, device=device) for _ in range(2)]
         self.Y = [torch.empty((M, w.N), dtype=torch.bfloat16, device=device) for _ in range(2)]
-        need = max(svdq_act_workspace_bytes(M, w.K, w.r), 256)
-        self.ws = [torch.empty(need, dtype=torch.uint8, device=device) for _ in range(2)]
+        self.ws = [new_workspace(M, w.K, w.r, device) for _ in range(2)]
         self.streams = [torch.cuda.Stream(device=device) for _ in range(2)]
         self.n = 0
 
@@ -469,6 +494,6 @@ class SVDQW4A4Linear(_linear_module_base()):
         M = X2.shape[0]
         need = svdq_act_workspace_bytes(M, self.packed.K, self.packed.r)
         if self._ws is None or self._ws.numel() < need or self._ws.device != X.device:
-            self._ws = torch.empty(max(need, 256), dtype=torch.uint8, device=X.device)
+            self._ws = new_workspace(M, self.packed.K, self.packed.r, X.device)
         Y = svdq_linear_forward(self.dev, X2, workspace=self._ws)
         return Y.reshape(*lead, self.out_features)

@@ -294,14 +294,8 @@ int64_t sf_tile_offset(int row, int g, int K) {
   return ((int64_t)(row / 128) * kb + g / 4) * 512 + (row % 32) * 16 + ((row % 128) / 32) * 4 + (g % 4);
 }
 
-// Row of the scale-atom layout that holds weight row n: the GEMM takes the
-// weight in tiles of 192 rows, each with its own two atom rows (128 + 64
-// rows, the last 64 rows of the second atom row left zero).
-static inline int weight_sf_row(int n) { return (n / 192) * 256 + n % 192; }
-
 // NVFP4 of rows x K float32 (row-major): codes two per byte (even k low
-// nibble) and E4M3 scales in the MMA tile layout (weight rows placed by
-// weight_sf_row).
+// nibble) and E4M3 scales in the MMA tile layout.
 static void quantize_nvfp4_rows(const float* T, int rows, int K, float g, float gs,
                                 uint8_t* codes, uint8_t* sf_tiled) {
 #pragma omp parallel for schedule(static)
@@ -312,7 +306,7 @@ static void quantize_nvfp4_rows(const float* T, int rows, int K, float g, float 
       for (int j = 0; j < 16; ++j) a = std::max(a, std::fabs(t[gi * 16 + j]));
       const uint8_t s = e4m3_code(a * gs);
       const float q = (s == 0) ? 0.0f : g / e4m3_value(s);
-      sf_tiled[sf_tile_offset(weight_sf_row(n), gi, K)] = s;
+      sf_tiled[sf_tile_offset(n, gi, K)] = s;
       for (int j = 0; j < 16; j += 2) {
         const uint8_t lo = e2m1_code(t[gi * 16 + j] * q);
         const uint8_t hi = e2m1_code(t[gi * 16 + j + 1] * q);
@@ -342,12 +336,10 @@ extern "C" svdq_status svdq_query_sizes(int N, int K, int r, svdq_sizes* out) {
   out->l1_mma_bytes = (size_t)2 * r * K * 2;
   out->l2_mma_bytes = (size_t)N * out->klr * 2;
   out->codes_w_bytes = (size_t)N * (K / 2);
-  out->sf_w_bytes = (size_t)((N + 191) / 192) * 256 * (K / 16);
+  out->sf_w_bytes = round_up((size_t)N, 256) * (K / 16);
   out->bias_bytes = (size_t)N * 2;
   return SVDQ_OK;
 }
-
-extern "C" int svdq_weight_sf_row(int n) { return n < 0 ? -1 : weight_sf_row(n); }
 
 extern "C" int64_t svdq_sf_tile_offset(int row, int g, int K) {
   if (row < 0 || g < 0 || K <= 0 || K % 64 || g >= K / 16) return -1;

@@ -8,11 +8,13 @@
 // pass over the activations.  The B200 design:
 //
 //   * one CTA owns 128 rows x a contiguous slice of K, walked in chunks of
-//     128 columns.  The host picks how many CTAs split K (S = 1, 2, 4 or 8,
-//     a thread-block cluster when S > 1) so that the whole grid is resident
-//     in one wave.  128 rows per CTA (one full scale-factor atom row) means
-//     every byte of the low-rank operand that reaches an SM serves 128 rows
-//     of X;
+//     128 columns.  The host picks how many CTAs split K (S = 1 .. 8) so that
+//     the grid fills the machine in one wave.  128 rows per CTA (one full
+//     scale-factor atom row) means every byte of the low-rank operand that
+//     reaches an SM serves 128 rows of X.  The split ranks are independent
+//     CTAs, not a cluster: clusters of 4 or more CTAs with this much shared
+//     memory cannot all be resident at once on the 148 SMs, which cost half
+//     the machine at 4608 tokens;
 //   * the slice's smoothing factors are loaded once (bulk copy) and stay in
 //     shared memory;
 //   * warp 0 streams X chunks [128 rows x 128 columns] bf16, as two
@@ -42,13 +44,13 @@
 //     tensor memory.  L1' holds smooth * L1 split into bf16 hi and lo
 //     halves, so X L1' = X_hat L1 to ~2^-16 relative (X itself is exact);
 //   * at the end the accumulator is read back (tcgen05.ld) and hi + lo
-//     columns are summed.  In a K split the r output columns are shared out
-//     among the S ranks (rank o owns columns [o r/S, (o+1) r/S)): every rank
-//     pushes its partial sums of the columns it does not own into the
-//     owner's shared memory with st.async (the bytes are counted on a
-//     barrier there), and each owner adds the S partials of its columns in
-//     rank order (deterministic) and stores them times lr_scale as a bf16
-//     hi/lo pair for the GEMM's up-projection.
+//     columns are summed.  Without a K split the result goes straight out,
+//     times lr_scale, as a bf16 hi/lo pair for the GEMM's up-projection.  In
+//     a K split every rank writes its fp32 partial sums to a scratch buffer
+//     (L2-resident, 16 KB per rank and row block at r = 32) and bumps the row
+//     block's arrival counter; the rank that arrives last adds the S
+//     partials in rank order (deterministic whoever is last), stores the
+//     hi/lo pair and resets the counter to zero for the next launch.
 #pragma once
 #include "ptx.cuh"
 
@@ -90,23 +92,21 @@ constexpr uint32_t QA_SMEM_BUDGET = 224 * 1024;  // + 1.5 KB: within the 227 KB 
 struct QALayout {
   int xst, lst, nstg;        // ring depths (X, low-rank operand, output staging)
   uint32_t l1_bytes;         // one low-rank stage: two boxes of 2r rows x 128 bytes
-  uint32_t l1_off, stg_off, s_off, red_off, lut_off, bar_off;
+  uint32_t l1_off, stg_off, s_off, lut_off, bar_off;
   uint32_t total;            // bytes to request (incl. alignment slack)
 };
 
-// Bytes of one rank's reduction buffer: the (S - 1) other ranks' partial
-// sums of the r / S columns it owns, 128 rows each, fp32.
-__host__ __device__ inline uint32_t qa_red_bytes(int r, int num_splits) {
-  if (r <= 0 || num_splits <= 1) return 0u;
-  return (uint32_t)(num_splits - 1) * QA_BM * (uint32_t)(r / num_splits) * 4u;
-}
+// Scratch of a K split: a zeroed arrival counter per 128-row block (the
+// first QA_CNT_BYTES bytes), then fp32 partial sums [S][blocks * 128][r].
+constexpr uint32_t QA_CNT_BYTES = 4096;
+constexpr int QA_MAX_SPLITS = 8;
+constexpr int QA_MAX_PART_ROWS = 160 * QA_BM;   // S * blocks <= 160 whenever S > 1
 
-__host__ __device__ inline QALayout qa_layout(int r, int chunks_per_split, int num_splits) {
+__host__ __device__ inline QALayout qa_layout(int r, int chunks_per_split) {
   QALayout L;
   L.l1_bytes = (uint32_t)QA_BOXES * 256u * (uint32_t)r;
   const uint32_t s_bytes = (uint32_t)QA_BOXES * 256u * (uint32_t)chunks_per_split;
-  const uint32_t red_bytes = qa_red_bytes(r, num_splits);
-  const uint32_t fixed = s_bytes + red_bytes + 512u + 512u;
+  const uint32_t fixed = s_bytes + 512u + 512u;
   const int lmax = chunks_per_split < QA_MAX_LST ? (chunks_per_split > 0 ? chunks_per_split : 1)
                                                  : QA_MAX_LST;
   // Preference: the deeper X ring, then two staging slots and two low-rank
@@ -137,8 +137,7 @@ __host__ __device__ inline QALayout qa_layout(int r, int chunks_per_split, int n
   L.l1_off = (uint32_t)L.xst * QA_X_BYTES;
   L.stg_off = L.l1_off + (uint32_t)L.lst * L.l1_bytes;      // multiple of 1024
   L.s_off = L.stg_off + (uint32_t)L.nstg * QA_STG_BYTES;
-  L.red_off = L.s_off + s_bytes;
-  L.lut_off = L.red_off + red_bytes;
+  L.lut_off = L.s_off + s_bytes;
   L.bar_off = L.lut_off + 512u;
   L.total = 1024u + L.bar_off + 512u;
   return L;
@@ -148,6 +147,8 @@ struct QAParams {
   const float* smooth;
   uint8_t* sf_x;
   uint16_t* xl1;
+  unsigned int* counters;   // K split: one zeroed counter per 128-row block
+  float* part;              // K split: fp32 partials [S][blocks * 128][r]
   int M, K, r, klr;
   int chunks_per_split;
   int num_splits;
@@ -199,20 +200,19 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   const uint32_t free0 = staged0 + 8 * NSTG;
   const uint32_t acc_full = free0 + 8 * NSTG;
   const uint32_t s_bar = acc_full + 8;
-  const uint32_t red_bar = acc_full + 16;
   const uint32_t drain_bar = acc_full + 24;
   uint32_t* tmem_holder =
       reinterpret_cast<uint32_t*>(bars + 2 * XST + 2 * LST + 2 * NSTG + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_holder + 2);
   float* qlut = reinterpret_cast<float*>(smem + L.lut_off);  // 128 floats
   const float* s_sm = reinterpret_cast<const float*>(smem + L.s_off);
 
   const uint32_t warp = warp_id(), lane = lane_id();
-  const int split = blockIdx.x;  // = rank in the cluster when S > 1
+  const int split = blockIdx.x;  // rank in the K split
   const int rb = blockIdx.y;
   const int S = p.num_splits;
   const bool reduce = has_lr && S > 1;
-  const int own_cols = reduce ? r / S : r;     // columns of the result this rank finishes
   const int kchunks = ((p.K >> 6) + QA_BOXES - 1) / QA_BOXES;   // 128-column chunks
   const int k64 = p.K >> 6;
   const int c_begin = split * p.chunks_per_split;
@@ -238,13 +238,10 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
     }
     mbar_init(acc_full, 1);
     mbar_init(s_bar, 1);
-    mbar_init(red_bar, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
+    *last_flag = 0;
     mbar_fence_init();
-    // every rank of a K split owns r / S columns and expects the other
-    // ranks' partial sums of them
-    if (reduce) mbar_arrive_expect_tx(red_bar, qa_red_bytes(r, S));
   }
   if (warp == 0 && lane == 0) {
     prefetch_tensormap(&tm_x);
@@ -263,9 +260,6 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  // every rank's barriers exist before any rank stores into another's
-  // shared memory (the matching wait comes before the epilogue)
-  if (reduce) cluster_arrive();
   const uint32_t tmem = has_lr ? *tmem_holder : 0u;
   // Everything above overlaps the tail of the previous kernel in the stream;
   // from here on this kernel reads and writes memory that kernel may touch.
@@ -498,7 +492,6 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   }
 
   // ----------------------------------------- low-rank epilogue (X L1) ----
-  if (reduce) cluster_wait();
   if (has_lr && warp >= QA_QWARP0) {
     const bool ok = mbar_wait_warp(acc_full, 0, p.timeout_ns, abort_flag, (4u << 8) | kid);
     tc_fence_after();
@@ -512,8 +505,8 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
     const int row_t = quad * 32 + lane;
     const int row = rb * QA_BM + row_t;
     const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t red_base = smem_u32(smem + L.red_off);
-    float own[8][4];                              // partials of the groups this rank owns
+    const size_t part_rows = (size_t)gridDim.y * QA_BM;
+    float own[8][4];                              // this rank's sums of the slot's groups
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
       if (g < cw4) {
@@ -531,58 +524,63 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
         }
 #pragma unroll
         for (int j = 0; j < 4; ++j) own[g][j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
-        if (reduce) {
-          const int owner = col / own_cols;
-          if (owner != split) {
-            // into the owner's buffer: [sender slot][128 rows][own_cols]
-            const int sslot = split < owner ? split : split - 1;
-            const uint32_t off = 4u * (uint32_t)((sslot * QA_BM + row_t) * own_cols +
-                                                 (col - owner * own_cols));
-            st_async_v4(map_to_rank(red_base + off, (uint32_t)owner), own[g][0], own[g][1],
-                        own[g][2], own[g][3], map_to_rank(red_bar, (uint32_t)owner));
-          }
-        }
+        if (reduce)
+          *reinterpret_cast<float4*>(p.part + ((size_t)split * part_rows + row) * r + col) =
+              make_float4(own[g][0], own[g][1], own[g][2], own[g][3]);
       }
     }
-    // finish the owned groups: the S partials added in rank order
-    const bool got = !reduce || mbar_wait_warp(red_bar, 0, p.timeout_ns, abort_flag, (6u << 8) | kid);
+    bool last = !reduce;
+    if (reduce) {
+      // every partial of this CTA is written before the count goes up; the
+      // CTA that brings the count to S sees every rank's partials
+      __threadfence();
+      named_barrier_sync(1, 32 * QA_QWARPS);
+      if (warp == QA_QWARP0 && lane == 0) {
+        const unsigned int prev = atomicAdd(p.counters + rb, 1u);
+        if (prev >= (unsigned int)S) record_error((10u << 8) | kid);  // counters not zeroed
+        if (prev == (unsigned int)(S - 1)) {
+          *last_flag = 1;
+          p.counters[rb] = 0u;   // ready for the next launch (stream order)
+        }
+      }
+      named_barrier_sync(1, 32 * QA_QWARPS);
+      last = *last_flag != 0;
+      if (last) __threadfence();
+    }
+    if (last) {
 #pragma unroll
-    for (int g = 0; g < 8; ++g) {
-      if (g < cw4) {
-        const int col = slot * 4 * cw4 + 4 * g;
-        if (reduce && col / own_cols != split) continue;
-        float sum[4];
-        if (reduce) {
+      for (int g = 0; g < 8; ++g) {
+        if (g < cw4) {
+          const int col = slot * 4 * cw4 + 4 * g;
+          float sum[4];
+          if (reduce) {
+            // the S partials in rank order, this rank's from registers
+            for (int sr = 0; sr < S; ++sr) {
+              float t[4];
+              if (sr == split) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j) sum[j] = 0.0f;
-          for (int sr = 0; sr < S; ++sr) {
-            float t[4];
-            if (sr == split || !got) {
+                for (int j = 0; j < 4; ++j) t[j] = own[g][j];
+              } else {
+                const float4 v = ld_cg_f4(p.part + ((size_t)sr * part_rows + row) * r + col);
+                t[0] = v.x; t[1] = v.y; t[2] = v.z; t[3] = v.w;
+              }
 #pragma unroll
-              for (int j = 0; j < 4; ++j) t[j] = sr == split ? own[g][j] : 0.0f;
-            } else {
-              const int sslot = sr < split ? sr : sr - 1;
-              const float4 v = *reinterpret_cast<const float4*>(
-                  smem + L.red_off +
-                  4u * (uint32_t)((sslot * QA_BM + row_t) * own_cols + (col - split * own_cols)));
-              t[0] = v.x; t[1] = v.y; t[2] = v.z; t[3] = v.w;
+              for (int j = 0; j < 4; ++j) sum[j] = sr == 0 ? t[j] : sum[j] + t[j];
             }
+          } else {
 #pragma unroll
-            for (int j = 0; j < 4; ++j) sum[j] = sr == 0 ? t[j] : sum[j] + t[j];
+            for (int j = 0; j < 4; ++j) sum[j] = own[g][j];
           }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) sum[j] = own[g][j];
+          if (row < p.M)
+            store_hi_lo4(sum, p.lr_scale, p.xl1 + (size_t)row * p.klr + col,
+                         p.xl1 + (size_t)row * p.klr + r + col);
         }
-        if (row < p.M)
-          store_hi_lo4(sum, p.lr_scale, p.xl1 + (size_t)row * p.klr + col,
-                       p.xl1 + (size_t)row * p.klr + r + col);
       }
-    }
-    // zero columns [2r, klr) of this row block
-    if (split == 0 && slot == 0 && row < p.M) {
-      for (int cpad = 2 * r; cpad < p.klr; cpad += 8)
-        *reinterpret_cast<uint4*>(p.xl1 + (size_t)row * p.klr + cpad) = make_uint4(0, 0, 0, 0);
+      // zero columns [2r, klr) of this row block
+      if (slot == 0 && row < p.M) {
+        for (int cpad = 2 * r; cpad < p.klr; cpad += 8)
+          *reinterpret_cast<uint4*>(p.xl1 + (size_t)row * p.klr + cpad) = make_uint4(0, 0, 0, 0);
+      }
     }
   }
 
@@ -610,8 +608,6 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
     }
     __syncthreads();
   }
-  // no rank leaves while another may still store into its shared memory
-  if (reduce) cluster_sync();
   if (warp == 1 && has_lr) {
     tc_fence_after();
     tmem_dealloc(tmem, p.tmem_cols);

@@ -61,14 +61,7 @@ struct DeviceInfo {
   bool ok = false;
   int num_sms = 0;
   bool attrs_set = false;
-  // max co-resident clusters of the activation kernel per cluster size S
-  // (1..8; every shared-memory plan holds one CTA per SM, so r does not
-  // matter); -1 = not queried yet
-  int max_clusters[9];
   int gemm_pairs = -1;  // max co-resident CTA pairs of the GEMM kernel
-  DeviceInfo() {
-    for (int& v : max_clusters) v = -1;
-  }
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -160,64 +153,42 @@ cudaLaunchAttribute pdl_attr() {
   return a;
 }
 
-// Largest K split S in {1, 2, 4, 8} (the cluster size when the low-rank
-// branch needs the cross-CTA reduction) such that the whole grid is resident
-// in one wave, the split's shared-memory plan keeps a deep enough activation
-// ring, and (with a low-rank branch) every rank owns a whole number of
-// 4-column groups of the result (r % S == 0, (r / S) % 4 == 0).
-int choose_splits(int tiles, int kchunks, int r, int sms) {
-  int dev = 0;
-  cudaGetDevice(&dev);
+// K split S (1 .. 8): the largest such that the grid (S x row blocks) stays
+// within one wave of one CTA per SM, every rank gets a chunk of K, the
+// split's shared-memory plan keeps a deep enough activation ring, and (with
+// a low-rank branch) the partial sums fit the scratch buffer.  No scratch
+// means no split.
+int choose_splits(int tiles, int kchunks, int r, int sms, bool have_scratch) {
   int best = 1;
-  for (int S = 2; S <= 8; S *= 2) {
+  if (r > 0 && !have_scratch) return 1;
+  for (int S = 2; S <= QA_MAX_SPLITS; ++S) {
     if (S > kchunks || tiles * S > sms) break;
-    if (r > 0 && (r % S != 0 || (r / S) % 4 != 0)) break;
+    if (r > 0 && (size_t)S * tiles * QA_BM > (size_t)QA_MAX_PART_ROWS) break;
     const int cps = (kchunks + S - 1) / S;
-    const QALayout L = qa_layout(r, cps, S);
-    if (L.xst < QA_MIN_XST) break;
-    if (r > 0) {
-      std::lock_guard<std::mutex> lk(g_mu);   // the caches are shared by host threads
-      int& cached = g_dev[dev].max_clusters[S];
-      if (cached < 0) {
-        cudaLaunchConfig_t cfg;
-        std::memset(&cfg, 0, sizeof(cfg));
-        cfg.gridDim = dim3((unsigned)S, 1, 1);
-        cfg.blockDim = dim3(QA_THREADS, 1, 1);
-        cfg.dynamicSmemBytes = L.total;
-        cudaLaunchAttribute attr;
-        attr.id = cudaLaunchAttributeClusterDimension;
-        attr.val.clusterDim.x = (unsigned)S;
-        attr.val.clusterDim.y = 1;
-        attr.val.clusterDim.z = 1;
-        cfg.attrs = &attr;
-        cfg.numAttrs = 1;
-        int n = 0;
-        if (cudaOccupancyMaxActiveClusters(&n, quantize_act_kernel, &cfg) != cudaSuccess) {
-          cudaGetLastError();
-          n = 0;
-        }
-        cached = n;
-      }
-      if (tiles > cached) continue;
-    }
+    if ((kchunks + cps - 1) / cps < S) continue;      // a rank would get no chunk
+    const QALayout L = qa_layout(r, cps);
+    if (L.xst < QA_MIN_XST) continue;
     best = S;
   }
   return best;
 }
 
 svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int64_t ldx,
-                            uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, cudaStream_t s,
-                            int sms) {
+                            uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, void* scratch,
+                            size_t scratch_bytes, cudaStream_t s, int sms) {
   const int K = w->K, r = w->r;
   // 128-row tiles: one scale-factor atom row each (padding rows get zero
   // scales)
   const int tiles = (M + QA_BM - 1) / QA_BM;
   const int KC = (K / 64 + QA_BOXES - 1) / QA_BOXES;  // 128-column chunks
-  int S = choose_splits(tiles, KC, r, sms);
+  const bool have_scratch = scratch != nullptr && scratch_bytes >= svdq_act_scratch_bytes(M, K, r) &&
+                            svdq_act_scratch_bytes(M, K, r) > 0;
+  const int S = choose_splits(tiles, KC, r, sms, have_scratch);
   const int cps = (KC + S - 1) / S;
-  const QALayout L = qa_layout(r, cps, S);
+  const QALayout L = qa_layout(r, cps);
   if (L.xst < QA_MIN_XST || L.nstg < QA_MIN_NSTG || (r > 0 && L.lst < 1))
     return SVDQ_ERR_INVALID_ARG;  // K too large for one CTA's slice
+
   CUtensorMap tm_x, tm_l1, tm_codes;
   std::memset(&tm_l1, 0, sizeof(tm_l1));
   if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M,
@@ -235,13 +206,16 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
   p.smooth = w->smooth;
   p.sf_x = sf_x;
   p.xl1 = xl1;
+  p.counters = static_cast<unsigned int*>(scratch);
+  p.part = scratch ? reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + QA_CNT_BYTES)
+                   : nullptr;
   p.M = M;
   p.K = K;
   p.r = r;
   p.klr = klr_of(r);
   p.chunks_per_split = cps;
   p.num_splits = S;
-  p.L = qa_layout(r, cps, S);
+  p.L = L;
   uint32_t cols = 32;
   while (cols < (uint32_t)(2 * r)) cols <<= 1;
   p.tmem_cols = cols;
@@ -256,17 +230,10 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
   cfg.blockDim = dim3(QA_THREADS, 1, 1);
   cfg.dynamicSmemBytes = p.L.total;
   cfg.stream = s;
-  cudaLaunchAttribute attr[2];
+  cudaLaunchAttribute attr[1];
   attr[0] = pdl_attr();
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (r > 0 && S > 1) {
-    attr[1].id = cudaLaunchAttributeClusterDimension;
-    attr[1].val.clusterDim.x = (unsigned)S;
-    attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
-    cfg.numAttrs = 2;
-  }
   if (cudaLaunchKernelEx(&cfg, quantize_act_kernel, tm_x, tm_l1, tm_codes, p) != cudaSuccess) {
     cudaGetLastError();
     return SVDQ_ERR_CUDA;
@@ -311,8 +278,7 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   std::memset(&tblr, 0, sizeof(tblr));
   // scale buffers as rows of 256 bytes (half a 512-byte atom), unswizzled
   const uint64_t sfa_rows = rup((size_t)M, 128) * (K / 16) / 256;
-  // weight scales: two atom rows per 192-row tile
-  const uint64_t sfb_rows = (uint64_t)((N + G_BN - 1) / G_BN) * G_SFB_ROWS * (K / 16) / 256;
+  const uint64_t sfb_rows = rup((size_t)N, 256) * (K / 16) / 256;
   if (!make_map(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codes_x, (uint64_t)K / 2, (uint64_t)M,
                 (uint64_t)K / 2, 128, G_BM) ||
       !make_map(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, w->codes_w, (uint64_t)K / 2, (uint64_t)N,
@@ -364,6 +330,7 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   return SVDQ_OK;
 }
 
+size_t ws_scratch(int M, int K, int r) { return rup(svdq_act_scratch_bytes(M, K, r), 256); }
 size_t ws_codes(int M, int K) { return rup((size_t)M * (K / 2), 256); }
 size_t ws_sf(int M, int K) { return rup(rup((size_t)M, 128) * (K / 16), 256); }
 size_t ws_xl1(int M, int r) { return rup((size_t)M * klr_of(r) * 2, 256); }
@@ -386,25 +353,35 @@ extern "C" const char* svdq_status_string(svdq_status s) {
 
 extern "C" const char* svdq_version(void) { return "svdq-b200 0.1"; }
 
+extern "C" size_t svdq_act_scratch_bytes(int M, int K, int r) {
+  if (M < 0 || K <= 0 || K % 64 || r < 0 || r > 128 || (r && r % 16)) return 0;
+  if (r == 0) return 0;
+  const size_t rows = std::min((size_t)QA_MAX_SPLITS * rup((size_t)M, QA_BM),
+                               (size_t)QA_MAX_PART_ROWS);
+  return QA_CNT_BYTES + rows * (size_t)r * 4;
+}
+
 extern "C" size_t svdq_act_workspace_bytes(int M, int K, int r) {
   if (M < 0 || K <= 0 || K % 64 || r < 0 || r > 128 || (r && r % 16)) return 0;
-  return ws_codes(M, K) + ws_sf(M, K) + (r > 0 ? ws_xl1(M, r) : 0);
+  return ws_scratch(M, K, r) + ws_codes(M, K) + ws_sf(M, K) + (r > 0 ? ws_xl1(M, r) : 0);
 }
 
 extern "C" svdq_status svdq_quantize_act(const svdq_weight* w, const uint16_t* X, int M,
                                          int64_t ldx, uint8_t* codes_x, uint8_t* sf_x,
-                                         uint16_t* xl1, void* stream) {
+                                         uint16_t* xl1, void* scratch, size_t scratch_bytes,
+                                         void* stream) {
   svdq_status st = check_weight(w);
   if (st != SVDQ_OK) return st;
   if (M < 0 || ldx < w->K) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   if (!X || !codes_x || !sf_x || (w->r > 0 && !xl1)) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || ldx % 8 || !aligned16(codes_x) || !aligned16(sf_x) ||
-      (xl1 && !aligned16(xl1)))
+      (xl1 && !aligned16(xl1)) || (scratch && (reinterpret_cast<uintptr_t>(scratch) & 255)))
     return SVDQ_ERR_MISALIGNED;
   int sms = 0;
   if ((st = device_check(&sms)) != SVDQ_OK) return st;
-  return launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, (cudaStream_t)stream, sms);
+  return launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, scratch, scratch_bytes,
+                         (cudaStream_t)stream, sms);
 }
 
 extern "C" svdq_status svdq_gemm(const svdq_weight* w, const uint8_t* codes_x,
@@ -437,11 +414,15 @@ extern "C" svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t*
   int sms = 0;
   if ((st = device_check(&sms)) != SVDQ_OK) return st;
   uint8_t* base = static_cast<uint8_t*>(workspace);
-  uint8_t* codes_x = base;
+  uint8_t* scratch = base;
+  const size_t scratch_bytes = ws_scratch(M, w->K, w->r);
+  uint8_t* codes_x = base + scratch_bytes;
   uint8_t* sf_x = codes_x + ws_codes(M, w->K);
   uint16_t* xl1 = w->r > 0 ? reinterpret_cast<uint16_t*>(sf_x + ws_sf(M, w->K)) : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
-  if ((st = launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, s, sms)) != SVDQ_OK) return st;
+  if ((st = launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, scratch_bytes ? scratch : nullptr,
+                            scratch_bytes, s, sms)) != SVDQ_OK)
+    return st;
   return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, s, sms);
 }
 

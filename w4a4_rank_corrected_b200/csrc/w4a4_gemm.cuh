@@ -7,71 +7,73 @@
 // merged into the 4-bit compute kernel.  The B200 design:
 //
 //   * CTA pairs (thread-block clusters of 2) share one tensor-core MMA
-//     (tcgen05 cta_group::2): a pair computes a 256 x 192 output tile, each
-//     CTA holds its 128 rows of the activation codes and half (96 rows) of
+//     (tcgen05 cta_group::2): a pair computes a 256 x 256 output tile, each
+//     CTA holds its 128 rows of the activation codes and half (128 rows) of
 //     the weight codes in its own shared memory and its 128 rows of the fp32
-//     accumulator in its own tensor memory;
-//   * two accumulators (tensor-memory columns [0, 192) and [192, 384)): the
-//     MMA works on tile t + 1 while the epilogue drains tile t, so the
-//     tensor core never waits for a tile boundary.  The per-stage scale
-//     factors take the columns after them ([384, 480), double-buffered);
+//     accumulator in its own tensor memory.  Per unit of MMA work each SM
+//     moves half the weight bytes through shared memory that a single-SM
+//     128 x 256 tile would, which is what keeps the tensor core fed;
 //   * warp 0 of each CTA (the whole warp waits, one elected lane issues)
-//     streams, per 256-deep K step, its A and B code tiles (TMA, 128-byte
-//     swizzle) and the scale atoms (its own 128 rows of activation scales,
-//     all 192 (padded to 256) rows of weight scales) into a 5-deep ring;
+//     streams, per 256-deep K step, its A and B code tiles
+//     (TMA, 128-byte swizzle) and the scale atoms (TMA; its own 128 rows of
+//     activation scales, all 256 rows of weight scales) into a 5-deep ring;
 //     every load is counted on the leader CTA's barrier (cta_group::2 form,
 //     no multicast);
+//   * each pair works through a contiguous run of output tiles in M-major
+//     order; for K <= 3072 the activation scales of the current 256-row
+//     block stay in tensor memory (192 columns beside the 256-column
+//     accumulator) and are loaded and copied only when the run enters a new
+//     row block, which takes a third of the scale copies off the MMA
+//     issuer's path (each copy beyond about one per MMA stalls it);
 //   * warp 1 of the leader (converged; an elected lane issues each
-//     instruction) copies the scale atoms into both CTAs' tensor memory
-//     (tcgen05.cp cta_group::2) and issues
+//     instruction) copies the scale atoms into both CTAs' tensor
+//     memory (tcgen05.cp cta_group::2) and issues
 //     tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 (M = 256,
-//     N = 192, K = 64); after the K loop it streams the low-rank operands
+//     N = 256, K = 64); after the K loop it streams the low-rank operands
 //     (xl1 hi|lo and L2, bf16) through the same ring into the SAME
 //     accumulator with kind::f16 MMAs (xl1 was pre-multiplied by
 //     g_x g_w = 1/alpha); completions are multicast to both CTAs;
-//   * warps 2..13 of each CTA: warp w drains tensor-memory lane quarter
-//     w % 4, columns [64 c, 64 c + 64) with c = (w - 2) / 4, releases the
-//     accumulator to the leader, then computes Y = bf16(alpha * acc + bias)
-//     (bias staged per tile in shared memory).  The four warps of one column
-//     group write a 128-row x 64-column box into a 16 KB shared-memory
-//     buffer (128-byte swizzle: a thread's row of 128 bytes lands in eight
-//     different bank groups across each eight rows) that one thread stores
-//     with TMA.
-//
-// Weight scales: each 192-row tile of the weight has its own two atom rows
-// (128 + 64 rows, padded with 64 zero rows), so a tile's scales are two
-// whole 512-byte atoms per 64-deep K step.  In row terms: weight row n sits
-// at row (n / 192) * 256 + n % 192 of the atom layout.
+//   * warps 2..9 of each CTA drain its accumulator (four 32-column
+//     tcgen05.ld, one wait), release it to the leader, and only then compute
+//     Y = bf16(alpha * acc + bias) (bias staged per tile in shared memory),
+//     overlapping the next tile's main loop.  Each group of four warps owns
+//     128 columns and writes them as two 128-row x 64-column boxes through a
+//     16 KB shared-memory buffer (128-byte swizzle, so the row-per-thread
+//     writes are free of bank conflicts) that one thread stores with TMA:
+//     one bulk store per box instead of a 16-byte global store per thread
+//     and row, which scattered each warp instruction over 32 rows and held
+//     the MMA issuer back.
 #pragma once
 #include "ptx.cuh"
 
 namespace svdq_dev {
 
 constexpr int G_STAGES = 5;
-constexpr int G_EPI_WARPS = 12;
+constexpr int G_EPI_WARPS = 8;
 constexpr int G_THREADS = 32 * (2 + G_EPI_WARPS);
 constexpr int G_BM = 128;                    // rows per CTA (pair tile: 256)
-constexpr int G_BN = 192;                    // columns per pair tile (MMA N)
-constexpr int G_BN_CTA = 96;                 // weight rows held per CTA
-constexpr int G_SFB_ROWS = 256;              // weight-scale rows per tile (padded)
+constexpr int G_BN = 256;                    // columns per pair tile (MMA N)
+constexpr int G_BN_CTA = 128;                // weight rows held per CTA
 constexpr uint32_t G_A_BYTES = 128 * 128;    // 128 rows x 128 B
-constexpr uint32_t G_B_BYTES = 96 * 128;     // 96 rows x 128 B
+constexpr uint32_t G_B_BYTES = 128 * 128;    // 128 rows x 128 B
 constexpr uint32_t G_SFA_BYTES = 4 * 512;    // 4 atoms (K = 256)
-constexpr uint32_t G_SFB_BYTES = 8 * 512;    // 2 atom rows x 4 atoms
+constexpr uint32_t G_SFB_BYTES = 8 * 512;    // 2 row blocks x 4 atoms
 constexpr uint32_t G_STAGE_BYTES = G_A_BYTES + G_B_BYTES + G_SFA_BYTES + G_SFB_BYTES;
 constexpr uint32_t G_TMEM_COLS = 512;
-constexpr uint32_t G_ACC_STRIDE = G_BN;      // accumulator b at columns [192 b, 192 b + 192)
-constexpr uint32_t G_SF_TMEM = 2 * G_BN;     // 384: scale buffers after the accumulators
-constexpr uint32_t G_SF_TMEM_STRIDE = 48;    // 16 cols SFA + 32 cols SFB per stage
-static_assert(G_SF_TMEM + 2 * G_SF_TMEM_STRIDE <= G_TMEM_COLS, "tensor memory plan");
+constexpr uint32_t G_SF_TMEM = 256;          // scale buffers after the accumulator
+constexpr uint32_t G_SF_TMEM_STRIDE = 48;    // 16 cols SFA + 32 cols SFB
+// Resident activation scales: 4 columns per 64-deep K step, all of K, for
+// K <= 3072 (192 columns); then the weight scales double-buffer after them.
+constexpr int G_SFA_RES_MAX_K64 = 48;
+constexpr uint32_t G_SFB_RES_TMEM = G_SF_TMEM + 4 * G_SFA_RES_MAX_K64;  // 448
+constexpr uint32_t G_SFB_RES_STRIDE = 32;
 constexpr uint32_t G_BIAS_BYTES = 2 * G_BN * 4;   // two fp32 bias tiles
 constexpr int G_OUT_COLS = 64;                    // columns per output box (128 bytes)
-constexpr int G_OUT_BOXES = G_BN / G_OUT_COLS;    // 3
-constexpr uint32_t G_OUT_BOX_BYTES = G_BM * 128;  // one box: 128 rows x 128 bytes
-constexpr uint32_t G_OUT_BYTES = G_OUT_BOXES * G_OUT_BOX_BYTES;
+constexpr uint32_t G_OUT_HALF_BYTES = G_BM * 128; // one box: 128 rows x 128 bytes
+constexpr uint32_t G_OUT_BYTES = 2 * G_OUT_HALF_BYTES;
 constexpr uint32_t G_FP4_TX = 2 * G_STAGE_BYTES;  // bytes per FP4 stage, both CTAs
+constexpr uint32_t G_FP4_TX_NOSFA = 2 * (G_STAGE_BYTES - G_SFA_BYTES);
 constexpr uint32_t G_LR_TX = 2 * (G_A_BYTES + G_B_BYTES);
-static_assert(G_EPI_WARPS == 4 * G_OUT_BOXES, "one warp per lane quarter and column box");
 
 __host__ __device__ inline uint32_t gemm_smem_bytes() {
   return 1024u + G_STAGES * G_STAGE_BYTES + G_OUT_BYTES + G_BIAS_BYTES + 256u;  // + barriers
@@ -97,25 +99,26 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  const uint32_t out_s = smem_u32(smem + G_STAGES * G_STAGE_BYTES);  // [3][128 rows][128 B]
+  const uint32_t out_s = smem_u32(smem + G_STAGES * G_STAGE_BYTES);  // [2][128 rows][128 B]
   float* bias_s =
-      reinterpret_cast<float*>(smem + G_STAGES * G_STAGE_BYTES + G_OUT_BYTES);  // [2][192]
+      reinterpret_cast<float*>(smem + G_STAGES * G_STAGE_BYTES + G_OUT_BYTES);  // [2][256]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + G_STAGES * G_STAGE_BYTES + G_OUT_BYTES +
                                                G_BIAS_BYTES);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * G_STAGES;
-  const uint32_t acc_full0 = full0 + 16 * G_STAGES;   // two: one per accumulator
-  const uint32_t acc_empty0 = acc_full0 + 16;         // two
-  const uint32_t drain_bar = acc_full0 + 32;
-  const uint32_t bias_bar0 = acc_full0 + 40;          // two: one per bias buffer
-  const uint32_t peer_bar = acc_full0 + 56;           // the pair CTA's final load count
-  // per output box: "staged" (its 4 warps wrote it) and "free" (the store
-  // issued from it has finished reading it)
-  const uint32_t out_staged0 = acc_full0 + 64;        // three
-  const uint32_t out_free0 = out_staged0 + 8 * G_OUT_BOXES;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * G_STAGES + 8 + 2 * G_OUT_BOXES);
+  const uint32_t acc_full = full0 + 16 * G_STAGES;
+  const uint32_t acc_empty = acc_full + 8;
+  const uint32_t drain_bar = acc_full + 16;
+  const uint32_t bias_bar0 = acc_full + 24;  // two: one per bias buffer
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bars + 2 * G_STAGES + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile int* peer_issued = reinterpret_cast<volatile int*>(tmem_holder + 2);
+  // per output buffer: "staged" (its 4 warps wrote it) and "free" (the
+  // store issued from it has finished reading it)
+  const uint32_t out_staged0 = smem_u32(bars + 2 * G_STAGES + 6);
+  const uint32_t out_free0 = out_staged0 + 16;
+  // the pair CTA's final load count (error path): a barrier and a word
+  const uint32_t peer_bar = smem_u32(bars + 2 * G_STAGES + 10);
+  volatile int* peer_issued = reinterpret_cast<volatile int*>(bars + 2 * G_STAGES + 11);
 
   const uint32_t warp = warp_id(), lane = lane_id();
   const uint32_t rank = cluster_ctarank();      // 0 = leader of the pair
@@ -127,11 +130,12 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   const int num_tiles = num_m * num_n;
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
   // Each pair takes a contiguous run of tiles in M-major order (tile t is
-  // M block t / num_n, N block t % num_n): consecutive tiles share their
-  // activation rows, which then mostly come from L2.
+  // M block t / num_n, N block t % num_n), so consecutive tiles mostly share
+  // their activation rows and those rows' scales stay in tensor memory.
   const int t_begin = (int)(((long long)pair * num_tiles) / num_pairs);
   const int t_end = (int)(((long long)(pair + 1) * num_tiles) / num_pairs);
   const int k64 = K >> 6;
+  const bool sfa_res = k64 <= G_SFA_RES_MAX_K64;
   const int kb_total = (k64 + 3) >> 2;
   const int lr_chunks = has_lr ? (p.klr >> 6) : 0;
   const unsigned int kid = 2;
@@ -141,19 +145,18 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       mbar_init(full0 + 8 * i, 1);
       mbar_init(empty0 + 8 * i, 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(acc_full0 + 8 * b, 1);
-      mbar_init(acc_empty0 + 8 * b, 2 * G_EPI_WARPS);
-      mbar_init(bias_bar0 + 8 * b, 32 * G_EPI_WARPS);
-    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 2 * G_EPI_WARPS);
     mbar_init(drain_bar, 1);
-    mbar_init(peer_bar, 1);
-    for (int h = 0; h < G_OUT_BOXES; ++h) {
-      mbar_init(out_staged0 + 8 * h, 4);
+    mbar_init(bias_bar0, 32 * G_EPI_WARPS);
+    mbar_init(bias_bar0 + 8, 32 * G_EPI_WARPS);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(out_staged0 + 8 * h, G_EPI_WARPS / 2);
       mbar_init(out_free0 + 8 * h, 1);
     }
-    *abort_flag = 0;
+    mbar_init(peer_bar, 1);
     *peer_issued = 0;
+    *abort_flag = 0;
     mbar_fence_init();
   }
   if (warp == 0 && lane == 0) {
@@ -177,7 +180,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
   const uint32_t lead_full0 = map_to_rank(full0, 0);
-  const uint32_t lead_acc_empty0 = map_to_rank(acc_empty0, 0);
+  const uint32_t lead_acc_empty = map_to_rank(acc_empty, 0);
   // The prologue above overlaps the previous kernel; the activation codes,
   // scales and low-rank operand it produced are read only after this.
   grid_dependency_wait();
@@ -190,6 +193,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     bool stop = false;
     for (int tile = t_begin; tile < t_end && !stop; ++tile) {
       const int mb = tile / num_n, nb = tile % num_n;
+      const bool load_sfa = !sfa_res || tile == t_begin || nb == 0;
       const int row0 = mb * 2 * G_BM + (int)rank * G_BM;     // this CTA's A rows
       const int brow0 = nb * G_BN + (int)rank * G_BN_CTA;    // this CTA's B rows
       const int sfa_blk = mb * 2 + (int)rank;                // 128-row scale block
@@ -202,13 +206,14 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         }
         if (elect_one()) {
           const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
-          if (leader) mbar_arrive_expect_tx(full0 + 8 * st, G_FP4_TX);
+          if (leader) mbar_arrive_expect_tx(full0 + 8 * st, load_sfa ? G_FP4_TX : G_FP4_TX_NOSFA);
           const uint32_t fb = lead_full0 + 8 * st;
           tma_load_2d_pair(sb, &tm_a, kb * 128, row0, fb);
           tma_load_2d_pair(sb + G_A_BYTES, &tm_b, kb * 128, brow0, fb);
           // scale atoms: rows of 256 bytes = half atoms; 4 atoms = 8 rows
-          tma_load_2d_pair(sb + G_A_BYTES + G_B_BYTES, &tm_sfa, 0, (sfa_blk * k64 + 4 * kb) * 2,
-                           fb);
+          if (load_sfa)
+            tma_load_2d_pair(sb + G_A_BYTES + G_B_BYTES, &tm_sfa, 0,
+                             (sfa_blk * k64 + 4 * kb) * 2, fb);
           for (int hh = 0; hh < 2; ++hh)
             tma_load_2d_pair(sb + G_A_BYTES + G_B_BYTES + G_SFA_BYTES + hh * 2048, &tm_sfb, 0,
                              ((2 * nb + hh) * k64 + 4 * kb) * 2, fb);
@@ -234,9 +239,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         issued = it + 1;
       }
     }
-    // The peer CTA's loads complete on the leader's barriers: it tells the
-    // leader how many stages it issued (remote store, then a remote arrive
-    // that releases it), so an aborted leader can drain them all.
+    // The other CTA's loads complete on the leader's barriers: it reports
+    // how many stages it issued (remote store, then a remote arrive that
+    // releases it), so an aborted leader can drain every one of them.
     if (!leader && lane == 0) {
       st_cluster_u32(map_to_rank(smem_u32((const void*)peer_issued), 0), (uint32_t)issued);
       mbar_arrive_release_cluster(map_to_rank(peer_bar, 0));
@@ -254,14 +259,13 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       // overlaps the tensor-core work instead of preceding the next issue)
       bool ready = false;
       for (int tile = t_begin; tile < t_end && !stop; ++tile, ++tcount) {
-        const int ab = tcount & 1;                 // accumulator of this tile
-        const uint32_t acc = tmem + (uint32_t)ab * G_ACC_STRIDE;
-        // the accumulator is free once the epilogue has drained the tile
-        // that used it two tiles ago
-        if (!mbar_wait_warp(acc_empty0 + 8 * ab, ((tcount >> 1) & 1) ^ 1, p.timeout_ns, abort_flag,
-                            (2u << 8) | kid))
+        // (the accumulator is free only once every MMA of the previous tile
+        // has completed, so resident scales may be overwritten after this)
+        if (!mbar_wait_warp(acc_empty, (tcount & 1) ^ 1, p.timeout_ns, abort_flag, (2u << 8) | kid))
           break;
         tc_fence_after();
+        const bool load_sfa = !sfa_res || tile == t_begin || tile % num_n == 0;
+        uint32_t accumulate = 0;
         for (int kb = 0; kb < kb_total; ++kb, ++it) {
           const int st = it % G_STAGES;
           const uint32_t ph = (it / G_STAGES) & 1;
@@ -275,8 +279,10 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           const uint32_t sb = smem_u32(smem + st * G_STAGE_BYTES);
           const uint32_t sfa_s = sb + G_A_BYTES + G_B_BYTES;
           const uint32_t sfb_s = sfa_s + G_SFA_BYTES;
-          const uint32_t sfa_t = tmem + G_SF_TMEM + (it & 1) * G_SF_TMEM_STRIDE;
-          const uint32_t sfb_t = sfa_t + 16;
+          const uint32_t sfa_t = sfa_res ? tmem + G_SF_TMEM + 16 * kb
+                                         : tmem + G_SF_TMEM + (it & 1) * G_SF_TMEM_STRIDE;
+          const uint32_t sfb_t = sfa_res ? tmem + G_SFB_RES_TMEM + (it & 1) * G_SFB_RES_STRIDE
+                                         : sfa_t + 16;
           // Every stage runs all four 64-deep steps, fixed and fully
           // unrolled: a loop bounded at run time (or a per-step guard) around
           // elect.sync here cut the issue rate by up to half.  A short last
@@ -285,7 +291,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           if (elect_one()) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              tmem_copy_32x128b_x4_pair(sfa_t + 4 * kk, sdesc_sf_block(sfa_s + 512 * kk));
+              if (load_sfa)
+                tmem_copy_32x128b_x4_pair(sfa_t + 4 * kk, sdesc_sf_block(sfa_s + 512 * kk));
               tmem_copy_32x128b_x4_pair(sfb_t + 8 * kk, sdesc_sf_block(sfb_s + 512 * kk));
               tmem_copy_32x128b_x4_pair(sfb_t + 8 * kk + 4,
                                         sdesc_sf_block(sfb_s + 2048 + 512 * kk));
@@ -296,10 +303,11 @@ __global__ void __launch_bounds__(G_THREADS, 1)
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {  // K = 64 E2M1 = 32 bytes per MMA
             if (elect_one())
-              mma_nvfp4_pair(acc, da + 2 * kk, db + 2 * kk, id_fp4, sfa_t + 4 * kk,
-                             sfb_t + 8 * kk, (kb | kk) > 0 ? 1u : 0u);
+              mma_nvfp4_pair(tmem, da + 2 * kk, db + 2 * kk, id_fp4, sfa_t + 4 * kk,
+                             sfb_t + 8 * kk, kk > 0 ? 1u : accumulate);
             __syncwarp();
           }
+          accumulate = 1;
           ready = mbar_test_warp(full0 + 8 * ((it + 1) % G_STAGES), ((it + 1) / G_STAGES) & 1);
           if (elect_one()) tc_commit_pair(empty0 + 8 * st, 0x3);
           __syncwarp();
@@ -318,102 +326,107 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           // zeros, so a partial last chunk adds exactly zero
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
-            if (elect_one()) mma_bf16_pair(acc, da + 2 * kk, db + 2 * kk, id_lr, 1u);
+            if (elect_one()) mma_bf16_pair(tmem, da + 2 * kk, db + 2 * kk, id_lr, 1u);
             __syncwarp();
           }
           ready = mbar_test_warp(full0 + 8 * ((it + 1) % G_STAGES), ((it + 1) / G_STAGES) & 1);
           if (elect_one()) tc_commit_pair(empty0 + 8 * st, 0x3);
           __syncwarp();
         }
-        if (elect_one()) tc_commit_pair(acc_full0 + 8 * ab, 0x3);
+        if (elect_one()) tc_commit_pair(acc_full, 0x3);
         __syncwarp();
       }
     }
   } else {
     // -------------------------------------------------------- epilogue ----
     const int quad = warp & 3;                 // tensor-memory lane quarter
-    const int cg = (warp - 2) >> 2;            // column box: [64 cg, 64 cg + 64)
-    const int et = threadIdx.x - 64;           // 0 .. 32 G_EPI_WARPS - 1
+    const int half = (warp - 2) >> 2;          // columns [128 half, 128 half + 128)
+    const int et = threadIdx.x - 64;           // 0..255
     const float alpha = p.alpha;
     const int row_t = quad * 32 + lane;        // this thread's row of the CTA's 128
-    const uint32_t obuf = out_s + cg * G_OUT_BOX_BYTES;
-    const uint32_t staged = out_staged0 + 8 * cg, freed = out_free0 + 8 * cg;
-    // one thread per column box issues its bulk stores
+    const uint32_t obuf = out_s + half * G_OUT_HALF_BYTES;
+    const uint32_t staged = out_staged0 + 8 * half, freed = out_free0 + 8 * half;
+    // one thread per group of four warps issues the group's bulk stores
     const bool issuer = ((warp - 2) & 3) == 0 && lane == 0;
+    int use = 0;                               // boxes this group has staged
     int tcount = 0;
-    bool ok = true;
-    for (int tile = t_begin; tile < t_end && ok; ++tile, ++tcount) {
+    for (int tile = t_begin; tile < t_end; ++tile, ++tcount) {
       const int mb = tile / num_n, nb = tile % num_n;
-      const int ab = tcount & 1;
       // stage this tile's bias (fp32) while the main loop runs.  Buffer
       // tcount&1 was last read for tile tcount-2, which every thread had
       // finished before arriving on the other buffer's barrier.
       float* bt = bias_s + (tcount & 1) * G_BN;
       const uint32_t bb = bias_bar0 + 8 * (tcount & 1);
-      if (et < G_BN) {
+      {
         const int n = nb * G_BN + et;
         bt[et] = (p.bias && n < N) ? bf16_lo_f32(p.bias[n]) : 0.0f;
       }
       mbar_arrive(bb);
       if (!mbar_wait_warp(bb, (tcount >> 1) & 1, p.timeout_ns, abort_flag, (5u << 8) | kid)) break;
-      if (!mbar_wait_warp(acc_full0 + 8 * ab, (tcount >> 1) & 1, p.timeout_ns, abort_flag,
-                          (4u << 8) | kid))
-        break;
+      if (!mbar_wait_warp(acc_full, tcount & 1, p.timeout_ns, abort_flag, (4u << 8) | kid)) break;
       tc_fence_after();
-      const uint32_t tbase =
-          tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)ab * G_ACC_STRIDE + cg * G_OUT_COLS;
-      uint32_t acc[2][32];
+      const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + half * 128;
+      uint32_t acc[4][32];
       tmem_ld32(tbase, acc[0]);
       tmem_ld32(tbase + 32, acc[1]);
+      tmem_ld32(tbase + 64, acc[2]);
+      tmem_ld32(tbase + 96, acc[3]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(lead_acc_empty0 + 8 * ab);   // accumulator free again
+      if (lane == 0) mbar_arrive_cluster(lead_acc_empty);   // accumulator free again
       const int row0 = mb * 2 * G_BM + (int)rank * G_BM;   // first row of this CTA's box
-      // the box buffer is free once the store issued from it has read it
-      if (tcount > 0) {
-        if (issuer) {
-          bulk_wait_read_all();
-          mbar_arrive(freed);
-        }
-        __syncwarp();
-        if (!mbar_wait_warp(freed, (tcount - 1) & 1, p.timeout_ns, abort_flag, (7u << 8) | kid)) {
-          ok = false;
-          break;
-        }
-      }
-      // 64 columns of this thread's row: 8 chunks of 16 bytes, chunk j at
-      // slot j ^ (row % 8) of the row's 128 bytes (the 128-byte swizzle)
+      bool ok = true;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int ch = j >> 2;
-        const int cb = 8 * (j & 3);
-        const int c0 = cg * G_OUT_COLS + ch * 32 + cb;
-        uint32_t o[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float y0 = fmaf(alpha, __uint_as_float(acc[ch][cb + 2 * q]), bt[c0 + 2 * q]);
-          const float y1 = fmaf(alpha, __uint_as_float(acc[ch][cb + 2 * q + 1]), bt[c0 + 2 * q + 1]);
-          o[q] = pack_bf16x2(y0, y1);
-        }
-        st_shared_v4(obuf + row_t * 128 + ((j ^ (row_t & 7)) << 4), o[0], o[1], o[2], o[3]);
-      }
-      fence_proxy_async_shared();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(staged);
-      if (issuer) {
-        const int x = nb * G_BN + cg * G_OUT_COLS;
-        // a box wholly past N or M has nothing to write
-        if (mbar_wait(staged, tcount & 1, p.timeout_ns, abort_flag, (8u << 8) | kid)) {
-          if (x < N && row0 < M) {
-            tma_store_2d(&tm_y, obuf, x, row0);
+      for (int sb = 0; sb < 2; ++sb, ++use) {
+        // the buffer is free once the store issued from it has read it
+        if (use > 0) {
+          if (issuer) {
+            bulk_wait_read_all();
+            mbar_arrive(freed);
           }
-          bulk_commit_group();
-        } else {
-          ok = false;
+          __syncwarp();
+          if (!mbar_wait_warp(freed, (use - 1) & 1, p.timeout_ns, abort_flag, (7u << 8) | kid)) {
+            ok = false;
+            break;
+          }
         }
+        // 64 columns of this thread's row: 8 chunks of 16 bytes, chunk j at
+        // slot j ^ (row % 8) of the row's 128 bytes (the 128-byte swizzle)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int ch = 2 * sb + (j >> 2);
+          const int cb = 8 * (j & 3);
+          const int c0 = half * 128 + ch * 32 + cb;
+          uint32_t o[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float y0 = fmaf(alpha, __uint_as_float(acc[ch][cb + 2 * q]), bt[c0 + 2 * q]);
+            const float y1 =
+                fmaf(alpha, __uint_as_float(acc[ch][cb + 2 * q + 1]), bt[c0 + 2 * q + 1]);
+            o[q] = pack_bf16x2(y0, y1);
+          }
+          st_shared_v4(obuf + row_t * 128 + ((j ^ (row_t & 7)) << 4), o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(staged);
+        if (issuer) {
+          const int x = nb * G_BN + half * 128 + sb * G_OUT_COLS;
+          // a box wholly past N or M has nothing to write
+          if (mbar_wait(staged, use & 1, p.timeout_ns, abort_flag, (8u << 8) | kid)) {
+            if (x < N && row0 < M) {
+              tma_store_2d(&tm_y, obuf, x, row0);
+              bulk_commit_group();
+            }
+          } else {
+            ok = false;
+          }
+        }
+        ok = __all_sync(0xffffffffu, ok) != 0;   // the issuer's verdict, warp-wide
+        if (!ok) break;
       }
-      ok = __all_sync(0xffffffffu, ok) != 0;   // the issuer's verdict, warp-wide
+      if (!ok) break;
     }
     // no store may still be reading shared memory (or writing Y) at exit
     if (issuer) bulk_wait_all();
@@ -424,19 +437,23 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   __syncthreads();
   if (*abort_flag) {
     // The leader's barriers count both CTAs' loads.  Drain the stages either
-    // CTA issued: the peer reports its count (bounded wait); a stage only the
-    // peer issued was never armed here, so arm it with the peer's bytes.
+    // CTA issued: the other CTA reports its count (bounded wait); a stage
+    // that only it issued was never armed here, so arm it with its bytes.
+    // Then drain the tensor-core work in flight.
     if (leader && warp == 0 && lane == 0) {
       mbar_wait_drain_cluster(peer_bar, 0, p.timeout_ns);
       const int peer = *peer_issued;
       const int hi = max(issued, peer);
+      const int per_tile = kb_total + lr_chunks;
       for (int i = max(0, hi - G_STAGES); i < hi; ++i) {
         const uint32_t fb = full0 + 8 * (i % G_STAGES);
         if (i >= issued) {
-          // the stage's kind follows from its position in the tile sequence
-          const int per_tile = kb_total + lr_chunks;
+          // the stage's bytes follow from its place in the tile sequence
+          // (the same rule the producers use)
+          const int tile = t_begin + i / per_tile;
           const bool lr_stage = (i % per_tile) >= kb_total;
-          mbar_arrive_expect_tx(fb, (lr_stage ? G_LR_TX : G_FP4_TX) / 2);
+          const bool with_sfa = !sfa_res || tile == t_begin || tile % num_n == 0;
+          mbar_arrive_expect_tx(fb, (lr_stage ? G_LR_TX : with_sfa ? G_FP4_TX : G_FP4_TX_NOSFA) / 2);
         }
         mbar_wait_drain(fb, (i / G_STAGES) & 1, p.timeout_ns);
       }
