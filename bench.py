@@ -57,6 +57,8 @@ def parse_args():
                     help="replay each step from a CUDA graph (small layers are launch-bound)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--pair", action="store_true",
+                    help="time the MLP pair of the workload (fc1 -> GELU -> fc2) as one step")
     ap.add_argument("--kernel-seconds", type=float, default=1.0,
                     help="device time of the per-kernel timing batches (each kernel alone)")
     ap.add_argument("--kernel-launches", type=int, default=1000,
@@ -246,12 +248,11 @@ def run_ours(args):
     sfs = [torch.empty(sf_bytes, dtype=torch.uint8, device=dev) for _ in range(nsets)]
     xl1s = [torch.empty((M, klr), dtype=torch.bfloat16, device=dev) if r else None
             for _ in range(nsets)]
-    scratches = [S.new_act_scratch(M, K, r, dev) for _ in range(nsets)]
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
         j = i % nsets
-        S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j], stream, scratches[j])
+        S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j], stream)
         S.svdq_gemm(weights[j], codes[j], sfs[j], xl1s[j], M, Ys[j], stream)
 
     sampler = ClockSampler(local if "CUDA_VISIBLE_DEVICES" not in os.environ
@@ -277,8 +278,7 @@ def run_ours(args):
             for j in range(nsets):
                 g = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(g):
-                    S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j],
-                                        scratch=scratches[j])
+                    S.svdq_quantize_act(weights[j], Xs[j], codes[j], sfs[j], xl1s[j])
                     S.svdq_gemm(weights[j], codes[j], sfs[j], xl1s[j], M, Ys[j])
                 graphs.append(g)
             for j in range(nsets):
@@ -341,8 +341,8 @@ def run_ours(args):
     if args.kernel_seconds > 0 or args.kernel_launches > 0:
         kt = dict(min_launches=max(1, args.kernel_launches), min_seconds=args.kernel_seconds)
         q_ms, q_n = kernel_time_ms(lambda i: S.svdq_quantize_act(
-            weights[i % nsets], Xs[i % nsets], codes[i % nsets], sfs[i % nsets], xl1s[i % nsets],
-            scratch=scratches[i % nsets]), **kt)
+            weights[i % nsets], Xs[i % nsets], codes[i % nsets], sfs[i % nsets], xl1s[i % nsets]),
+            **kt)
         g_ms, g_n = kernel_time_ms(lambda i: S.svdq_gemm(
             weights[i % nsets], codes[i % nsets], sfs[i % nsets], xl1s[i % nsets], M,
             Ys[i % nsets]), **kt)
@@ -550,10 +550,115 @@ def run_reference(args):
     print(json.dumps(out), flush=True)
 
 
+def run_pair(args):
+    """One step = the whole MLP pair of the workload (flux_mlp, or the fc1/fc2
+    layers of flux_block): svdq_mlp_forward, i.e. fc1's activation kernel,
+    fc1's GEMM with the GELU epilogue, fc2's activation kernel on H, fc2's
+    GEMM.  Reported beside it: the same pair with GELU as a separate pass
+    (torch, bf16) between the layers."""
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    import w4a4_rank_corrected_b200 as S
+    spec = SI.workload_specs()[args.workload]
+    wl = SI.make_workload(spec.name)
+    names = [l.spec.name for l in wl.layers]
+    i1 = names.index("fc1")
+    l1, l2 = wl.layers[i1], wl.layers[i1 + 1]
+    M, K1, N1, N2 = l1.spec.M, l1.spec.K, l1.spec.N, l2.spec.N
+    X0 = wl.X_bf16 if i1 == 0 else SI.draw_activations(
+        np.random.default_rng(spec.seed * 7919 + rank), M, K1, spec.x_dist, spec.x_outliers,
+        spec.x_scale)
+    if rank > 0 and i1 == 0:
+        X0 = rank_activations(spec, rank, M, K1)
+    p1 = S.svdq_pack_weight(l1.W, SI.channel_absmax(X0), l1.spec.r, bias_bf16=l1.bias_bf16)
+    w1 = p1.to_device(dev)
+    Xd = torch.from_numpy(X0.view(np.int16)).to(dev).view(torch.bfloat16)
+    # fc2 is calibrated on the pair's own GELU output
+    Hcal = S.svdq_debug_gelu(S.svdq_linear_forward(w1, Xd))
+    hbits = Hcal.view(torch.int16).cpu().numpy().view(np.uint16)
+    p2 = S.svdq_pack_weight(l2.W, SI.channel_absmax(hbits), l2.spec.r, bias_bf16=l2.bias_bf16)
+    nsets = max(1, min(args.sets, 2))
+    W1 = [p1.to_device(dev) for _ in range(nsets)]
+    W2 = [p2.to_device(dev) for _ in range(nsets)]
+    Xs = [Xd.clone() for _ in range(nsets)]
+    Hs = [torch.empty((M, N1), dtype=torch.bfloat16, device=dev) for _ in range(nsets)]
+    Ys = [torch.empty((M, N2), dtype=torch.bfloat16, device=dev) for _ in range(nsets)]
+    wss = [S.new_mlp_workspace(M, W1[j], W2[j], dev) for j in range(nsets)]
+
+    def fused(i):
+        j = i % nsets
+        S.svdq_mlp_forward(W1[j], W2[j], Xs[j], Hs[j], Ys[j], wss[j])
+
+    def unfused(i):
+        j = i % nsets
+        Y1 = S.svdq_linear_forward(W1[j], Xs[j], Hs[j], wss[j])
+        G = torch.nn.functional.gelu(Y1, approximate="tanh")
+        S.svdq_linear_forward(W2[j], G, Ys[j], wss[j])
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for i in range(args.warmup):
+        fused(i)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(args.steps):
+        fused(i)
+    b.record()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(a.elapsed_time(b), world, dev) / args.steps
+    for i in range(args.warmup):
+        unfused(i)
+    torch.cuda.synchronize(dev)
+    a.record()
+    for i in range(args.steps):
+        unfused(i)
+    b.record()
+    torch.cuda.synchronize(dev)
+    ms_unfused = max_over_ranks(a.elapsed_time(b), world, dev) / args.steps
+    clocks = sampler.stop()
+    err = S.svdq_device_error()
+    if err:
+        raise SystemExit(f"device error code {err:#x}")
+    flops = 2.0 * M * (N1 * K1 + N2 * N1)
+    out = {"metric": METRIC, "value": round(world * flops / (ms * 1e-3) / 1e12, 2), "unit": "TFLOPS",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+           "config": {"workload": f"{spec.name}: MLP pair fc1 {K1}->{N1}, GELU, fc2 {N1}->{N2}",
+                      "M": M, "r": l1.spec.r,
+                      "us_per_pair": round(ms * 1e3, 2),
+                      "us_per_pair_unfused_gelu": round(ms_unfused * 1e3, 2),
+                      "path": "svdq_mlp_forward: fc1 activation kernel, fc1 GEMM with the GELU "
+                              "epilogue, fc2 activation kernel, fc2 GEMM; the unfused figure runs "
+                              "torch's bf16 tanh GELU between the layers instead",
+                      "l2": f"{nsets} rotating sets"},
+           "gpu_launches": 4 * args.steps, "clocks": clocks}
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.pair:
+        run_pair(args)
     else:
         run_ours(args)
 

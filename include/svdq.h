@@ -180,22 +180,9 @@ typedef struct svdq_weight {
   const uint8_t*  sf_w;     /* device u8, MMA tiles, rows padded to 256    */
 } svdq_weight;
 
-/* Bytes of the activation kernel's scratch for M tokens (0 when r == 0):
- * a K split of the activation kernel needs it for its low-rank partial
- * sums.  Layout: 4096 bytes of arrival counters (one 32-bit word per 128-row
- * block) followed by fp32 partial sums.  The counters must be ZERO before
- * the scratch's first use; every launch that completes leaves them zero
- * again, so a scratch buffer is zeroed once when it is allocated (after a
- * SVDQ_ERR_TIMEOUT from svdq_device_error, zero it again).  0 on bad
- * arguments. */
-size_t svdq_act_scratch_bytes(int M, int K, int r);
-
-/* Bytes of the forward's workspace for M tokens: the activation scratch
- * (first, counters at offset 0), codes_x [M][K/2], sf_x (MMA tiles, rows
- * padded to 128) and xl1 [M][klr] bf16, each region 256-byte aligned.  The
- * first 4096 bytes must be zero before the workspace's first use (see
- * svdq_act_scratch_bytes); the library leaves them zero.  0 on bad
- * arguments. */
+/* Bytes of the activation workspace for M tokens: codes_x [M][K/2],
+ * sf_x (MMA tiles, rows padded to 128) and xl1 [M][klr] bf16, each region
+ * 256-byte aligned.  0 on bad arguments. */
 size_t svdq_act_workspace_bytes(int M, int K, int r);
 
 /* svdq_quantize_act: activation kernel (one launch).
@@ -214,16 +201,16 @@ size_t svdq_act_workspace_bytes(int M, int K, int r);
  *   codes_x  device u8 [M][K/2]
  *   sf_x     device u8, MMA tiles, round_up(M,128) * K/16 bytes (pad rows 0)
  *   xl1      device bf16 [M][klr] (may be NULL if r == 0)
- *   scratch  device, >= svdq_act_scratch_bytes(M, K, r), 256-byte aligned,
- *            counters zeroed (see above); NULL (or too small) runs the kernel
- *            without splitting K, which is slower for M below ~18000.
- * Reads X exactly once.  Returns SVDQ_ERR_INVALID_ARG when one CTA's share
- * of K does not fit its shared-memory plan (K above roughly 36000).
+ * Reads X exactly once.  Two kernel forms by batch size: 128-row tiles over
+ * all of K when there are enough rows to give most SMs a tile of their own
+ * (about 15k rows and up), else 64-row tiles with K split within a cluster.
+ * Returns SVDQ_ERR_INVALID_ARG when one CTA's share of K does not fit its
+ * shared-memory plan (for large M: K above roughly 36000 at r <= 32, 24000
+ * at r = 128).
  */
 svdq_status svdq_quantize_act(const svdq_weight* w, const uint16_t* X, int M,
                               int64_t ldx, uint8_t* codes_x, uint8_t* sf_x,
-                              uint16_t* xl1, void* scratch, size_t scratch_bytes,
-                              void* stream);
+                              uint16_t* xl1, void* stream);
 
 /* svdq_gemm: the 4-bit GEMM kernel (one launch).
  * Source: the Korean rendering of "Bringing Nunchaku 4-bit diffusion
@@ -239,12 +226,44 @@ svdq_status svdq_gemm(const svdq_weight* w, const uint8_t* codes_x,
                       const uint8_t* sf_x, const uint16_t* xl1, int M,
                       uint16_t* Y, int64_t ldy, void* stream);
 
+/* svdq_gemm_gelu: svdq_gemm for the first linear of an MLP pair, with the
+ * pair's GELU fused into the epilogue.  Source: the fused GELU/MLP kernels
+ * the pages name as part of the original engine's speed ("Bringing Nunchaku
+ * 4-bit diffusion inference to Diffusers", Vietnamese rendering, section
+ * "Introducing Nunchaku Lite").  Writes H = bf16(GELU(bf16(alpha * acc +
+ * bias))) instead of Y; GELU is the tanh form evaluated as y / (1 +
+ * e^(-2u)), u = sqrt(2/pi) (y + 0.044715 y^3), in a fixed sequence of
+ * round-to-nearest fp32 operations (e^x from basic operations: a degree-7
+ * Taylor series of 2^f times 2^n), so it is reproducible bit for bit; see
+ * svdq_debug_gelu.  H is never materialized as Y first.  Arguments and
+ * errors as svdq_gemm (H in place of Y). */
+svdq_status svdq_gemm_gelu(const svdq_weight* w, const uint8_t* codes_x,
+                           const uint8_t* sf_x, const uint16_t* xl1, int M,
+                           uint16_t* H, int64_t ldh, void* stream);
+
+/* Bytes of the workspace of svdq_mlp_forward (the larger of the two
+ * layers' forward workspaces).  0 on bad arguments. */
+size_t svdq_mlp_workspace_bytes(int M, int K1, int N1, int r1, int r2);
+
+/* svdq_mlp_forward: a Flux MLP pair, fc1 -> GELU -> fc2, in four launches on
+ * one stream: the activation kernel of fc1, the GEMM of fc1 with the GELU
+ * epilogue (svdq_gemm_gelu), the activation kernel of fc2 on H, the GEMM of
+ * fc2.  w2->K must equal w1->N.
+ *   X  device bf16 [M][ldx]   (fc1 input)
+ *   H  device bf16 [M][ldh]   (GELU(fc1 output), caller-owned, also fc2's input)
+ *   Y  device bf16 [M][ldy]   (fc2 output)
+ *   workspace  >= svdq_mlp_workspace_bytes, 256-byte aligned.
+ * Errors as svdq_linear_forward. */
+svdq_status svdq_mlp_forward(const svdq_weight* w1, const svdq_weight* w2,
+                             const uint16_t* X, int M, int64_t ldx, uint16_t* H,
+                             int64_t ldh, uint16_t* Y, int64_t ldy, void* workspace,
+                             size_t ws_bytes, void* stream);
+
 /* svdq_linear_forward: the whole layer, Y = Q(X_hat) Q(R)^T + (X_hat L1) L2
  * + bias ("Background: SVDQuant and Nunchaku"; the runtime SVDQW4A4Linear
  * layer that replaces nn.Linear in "Loading natively in Diffusers"):
  * svdq_quantize_act then svdq_gemm on one stream, with the intermediates in
- * `workspace` (device, >= svdq_act_workspace_bytes, 256-byte aligned, its
- * first 4096 bytes zero before its first use). */
+ * `workspace` (device, >= svdq_act_workspace_bytes, 256-byte aligned). */
 svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t* X,
                                 int M, int64_t ldx, uint16_t* Y, int64_t ldy,
                                 void* workspace, size_t ws_bytes,
@@ -284,11 +303,9 @@ svdq_status svdq_linear_forward_host(const svdq_weight* w, const uint16_t* X_hos
  *     library's device code on the device.
  *   - M is limited by the scratch size: svdq_act_workspace_bytes(M, K, r)
  *     must be <= SVDQ_STATIC_WORKSPACE_BYTES, else SVDQ_ERR_WORKSPACE and
- *     nothing is launched (e.g. K = 3072, r = 32 allows M <= 7618).
- *   - The scratch starts zeroed (a module's device variables are zero when
- *     it loads) and every call that completes leaves the activation
- *     kernel's arrival counters at its start zero again; everything else in
- *     it is written before it is read.
+ *     nothing is launched (e.g. K = 3072, r = 32 allows M <= 9033).
+ *   - Nothing in the scratch needs to start at zero: the activation kernel
+ *     writes every byte the GEMM reads, padding rows included.
  *   - One scratch area per device: calls that overlap in time (different
  *     streams, or threads without ordering) race on it.  Calls in order on
  *     one stream are safe.
@@ -318,6 +335,10 @@ svdq_status svdq_selftest_timeout(int timeout_us, void* stream);
  * activation kernel uses.  in/out device pointers, n >= 0. */
 svdq_status svdq_debug_convert(const float* in, uint8_t* e2m1_out,
                                uint8_t* e4m3_out, int64_t n, void* stream);
+
+/* Diagnostic: the epilogue GELU of svdq_gemm_gelu on n bf16 values
+ * (device in/out, bf16 bit patterns). */
+svdq_status svdq_debug_gelu(const uint16_t* in, uint16_t* out, int64_t n, void* stream);
 
 #ifdef __cplusplus
 }

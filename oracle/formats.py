@@ -113,14 +113,16 @@ def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
 
 def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """float64 -> bfloat16, ONE rounding (nearest, ties to even) straight
-    from the float64 value.  Magnitudes below the smallest normal bf16
-    (2^-126) are flushed to a signed zero (they never occur for the
-    low-rank factors; documented as a reading)."""
+    from the float64 value, with gradual underflow: below the smallest
+    normal bf16 (2^-126) the values are the multiples of 2^-133 (7 mantissa
+    bits, exponent field 0), so |x| rounds to the nearest such multiple,
+    ties to the even one; the result keeps the sign (a value that rounds to
+    zero gives a signed zero)."""
     x = np.ascontiguousarray(x, dtype=np.float64)
     bits = x.view(np.uint64)
     sign = (bits >> np.uint64(63)).astype(np.uint64)
     mag_bits = bits & np.uint64(0x7FFFFFFFFFFFFFFF)
-    # keep sign+exponent(11)+7 mantissa bits: drop the low 45 bits
+    # normal range: keep sign+exponent(11)+7 mantissa bits, drop the low 45
     keep = mag_bits >> np.uint64(45)
     rem = mag_bits & np.uint64((1 << 45) - 1)
     half = np.uint64(1 << 44)
@@ -128,20 +130,33 @@ def f64_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     keep = keep + up.astype(np.uint64)
     rounded = (keep << np.uint64(45)).view(np.float64)
     f = rounded.astype(np.float32)       # exact: 8 significant bits
-    f = np.where(np.abs(rounded) < 2.0 ** -126, np.float32(0.0), f)
     fb = f.view(np.uint32) >> np.uint32(16)
+    # subnormal range: the count of 2^-133 steps, rounded half to even
+    # (np.rint); a count of 128 is the smallest normal, 0x0080, as it should
+    mag = np.abs(x)
+    tiny = mag < 2.0 ** -126
+    steps = np.rint(np.where(tiny, mag, 0.0) * 2.0 ** 133).astype(np.uint32)
+    fb = np.where(tiny, steps, fb)
     fb = fb.astype(np.uint16) | (sign.astype(np.uint16) << np.uint16(15))
     return fb
 
 
 def bf16_round_exact(x: float) -> Fraction:
-    """Brute force (exact rationals): nearest bf16 value to x, ties to even.
-    Used only by the pins."""
+    """Brute force (exact rationals): nearest bf16 value to x, ties to even,
+    with the subnormal grid (multiples of 2^-133) below 2^-126.  Used only by
+    the pins."""
     fx = Fraction(x)
     if fx == 0:
         return Fraction(0)
     s = -1 if fx < 0 else 1
     a = abs(fx)
+    if a < Fraction(2) ** -126:
+        scaled = a * Fraction(2) ** 133
+        lo = int(scaled)
+        frac = scaled - lo
+        if frac > Fraction(1, 2) or (frac == Fraction(1, 2) and lo % 2 == 1):
+            lo += 1
+        return s * Fraction(lo) * Fraction(2) ** -133
     e = 0
     while a >= 2:
         a /= 2

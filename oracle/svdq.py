@@ -408,8 +408,10 @@ def gelu_tanh_f32(y: np.ndarray) -> np.ndarray:
     u = sqrt(2/pi) (y + 0.044715 y^3), each step one float32 rounding:
     y2 = y y, y3 = y2 y, v = 0.044715 y3, w = y + v, u = c w, E = exp(-2u),
     d = 1 + E, h = y / d.  For finite y: h = y exactly for large y (E
-    underflows to 2^-126), and h = -0 once e^(-2u) passes 2^128 (true
-    values below 2^-120 in magnitude, which a bf16 result flushes anyway)."""
+    underflows to 2^-126), and h = -0 once e^(-2u) passes 2^128 (where the
+    true value is below 2^-120 in magnitude: an absolute error under
+    2^-120).  Tiny inputs keep gradual underflow: for y below 2^-126 the
+    result is y / 2 rounded in the float32 subnormal range."""
     y = np.asarray(y, F32)
     with np.errstate(over="ignore", divide="ignore", invalid="ignore"):
         return _gelu_steps(y)

@@ -65,11 +65,7 @@ def test_sf_tile_offset_matches_oracle_layout():
 def test_workspace_bytes():
     M, K, r = 4608, 3072, 32
     ws = S.svdq_act_workspace_bytes(M, K, r)
-    sc = S.svdq_act_scratch_bytes(M, K, r)
-    # counters, then the partial sums of up to 8 ranks (at most 160 row blocks in all)
-    assert sc == 4096 + min(8 * 4608, 160 * 128) * 32 * 4
-    assert S.svdq_act_scratch_bytes(M, K, 0) == 0
-    assert ws >= sc + M * K // 2 + M * K // 16 + M * 64 * 2
+    assert ws >= M * K // 2 + M * K // 16 + M * 64 * 2
     assert ws % 256 == 0
     assert S.svdq_act_workspace_bytes(100, 3000, 32) == 0
 
@@ -88,17 +84,15 @@ def test_argument_validation_before_any_launch():
     w = _fake_weight()
     X, C, SF, XL = 0x20000000, 0x30000000, 0x40000000, 0x50000000
     # null weight / null pointers / bad shapes
-    SC, NS = 0x58000000, S.svdq_act_scratch_bytes(16, 256, 32)
-    assert L.svdq_quantize_act(None, X, 16, 256, C, SF, XL, SC, NS, None) == 1
-    assert L.svdq_quantize_act(ctypes.byref(w), None, 16, 256, C, SF, XL, SC, NS, None) == 1
-    assert L.svdq_quantize_act(ctypes.byref(w), X, -1, 256, C, SF, XL, SC, NS, None) == 1
-    assert L.svdq_quantize_act(ctypes.byref(w), X, 16, 128, C, SF, XL, SC, NS, None) == 1  # ldx < K
+    assert L.svdq_quantize_act(None, X, 16, 256, C, SF, XL, None) == 1
+    assert L.svdq_quantize_act(ctypes.byref(w), None, 16, 256, C, SF, XL, None) == 1
+    assert L.svdq_quantize_act(ctypes.byref(w), X, -1, 256, C, SF, XL, None) == 1
+    assert L.svdq_quantize_act(ctypes.byref(w), X, 16, 128, C, SF, XL, None) == 1  # ldx < K
     bad = _fake_weight(K=200)
-    assert L.svdq_quantize_act(ctypes.byref(bad), X, 16, 256, C, SF, XL, SC, NS, None) == 1
+    assert L.svdq_quantize_act(ctypes.byref(bad), X, 16, 256, C, SF, XL, None) == 1
     # misalignment
-    assert L.svdq_quantize_act(ctypes.byref(w), X + 2, 16, 256, C, SF, XL, SC, NS, None) == 3
-    assert L.svdq_quantize_act(ctypes.byref(w), X, 16, 260, C, SF, XL, SC, NS, None) == 3
-    assert L.svdq_quantize_act(ctypes.byref(w), X, 16, 256, C, SF, XL, SC + 16, NS, None) == 3
+    assert L.svdq_quantize_act(ctypes.byref(w), X + 2, 16, 256, C, SF, XL, None) == 3
+    assert L.svdq_quantize_act(ctypes.byref(w), X, 16, 260, C, SF, XL, None) == 3
     assert L.svdq_gemm(ctypes.byref(w), C, SF, XL, 16, 0x60000008, 256, None) == 3
     mis = _fake_weight(base=0x10000004)
     assert L.svdq_gemm(ctypes.byref(mis), C, SF, XL, 16, 0x60000000, 256, None) == 3

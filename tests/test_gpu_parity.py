@@ -224,56 +224,31 @@ def test_activation_kernel_repeats_bit_identical():
     X, W, b = SI.random_layer(24, M, K, N)
     lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
     Xd = to_dev_bf16(X)
-    scratch = S.new_act_scratch(M, K, r)
-    c0, s0, x0 = (t.clone() for t in S.svdq_quantize_act(dw, Xd, scratch=scratch))
+    c0, s0, x0 = (t.clone() for t in S.svdq_quantize_act(dw, Xd))
     for _ in range(20):
-        c, sf, xl1 = S.svdq_quantize_act(dw, Xd, scratch=scratch)
+        c, sf, xl1 = S.svdq_quantize_act(dw, Xd)
         assert torch.equal(c, c0) and torch.equal(sf, s0)
         assert torch.equal(xl1.view(torch.int16), x0.view(torch.int16))
-    # the K split's arrival counters are back at zero after every launch
-    assert int(scratch[:4096].count_nonzero()) == 0
 
 
-@pytest.mark.parametrize("M,K,r", [(4608, 3072, 32), (256, 3072, 32), (300, 1024, 16),
-                                   (1000, 1536, 64)])
-def test_activation_kernel_split_matches_unsplit(M, K, r):
-    """The activation kernel with its K split (scratch given) and without
-    (no scratch: one CTA per row block walks all of K): the same codes and
-    scales bit for bit; the low-rank operand differs only by the order of
-    the fp32 additions."""
-    import ctypes
+@pytest.mark.parametrize("M,K,N,r", [(15361, 320, 64, 48), (16000, 3072, 128, 32),
+                                     (15500, 192, 64, 0), (20000, 1024, 96, 128)])
+def test_activation_kernel_128_row_tiles(M, K, N, r):
+    """Batches of about 15k rows and more take the 128-row activation kernel
+    (the others the 64-row one): bit-exact codes and scales on every row,
+    the low-rank operand within tolerance, ragged M and K tails, r from 0 to
+    128; and the whole layer on one row of every 128-row block."""
     S = _S()
-    X, W, b = SI.random_layer(M + K + r, M, K, 64)
+    X, W, b = SI.random_layer(M + K, M, K, N)
     lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
     Xd = to_dev_bf16(X)
-    c1, s1, x1 = S.svdq_quantize_act(dw, Xd)
-    c2 = torch.empty_like(c1)
-    s2 = torch.zeros_like(s1)
-    x2 = torch.empty_like(x1)
-    st = S.lib.svdq_quantize_act(ctypes.byref(dw.struct), Xd.data_ptr(), M, K, c2.data_ptr(),
-                                 s2.data_ptr(), x2.data_ptr(), None, 0,
-                                 torch.cuda.current_stream().cuda_stream)
-    assert st == 0
+    codes, sf, xl1 = S.svdq_quantize_act(dw, Xd)
+    Y = S.svdq_linear_forward(dw, Xd)
     torch.cuda.synchronize()
-    assert torch.equal(c1, c2) and torch.equal(s1, s2)
-    check_activation(c2, s2, x2, X, op, M, K, r)
-    a = F.bf16_bits_to_f64(from_dev_bf16(x1)[:, :r]) + F.bf16_bits_to_f64(from_dev_bf16(x1)[:, r:2 * r])
-    c = F.bf16_bits_to_f64(from_dev_bf16(x2)[:, :r]) + F.bf16_bits_to_f64(from_dev_bf16(x2)[:, r:2 * r])
-    assert np.max(np.abs(a - c)) <= 1e-5 * np.max(np.abs(c))
-
-
-def test_activation_scratch_counters_not_zeroed_is_reported():
-    """A scratch whose arrival counters were not zeroed is caught: the kernel
-    records error code (10 << 8) | 1, which svdq_device_error returns."""
-    S = _S()
-    M, K, r = 4608, 3072, 32
-    X, W, b = SI.random_layer(41, M, K, 64)
-    lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
-    scratch = S.new_act_scratch(M, K, r)
-    scratch[:4096].fill_(0x7F)                # counters far above any split count
-    S.svdq_quantize_act(dw, to_dev_bf16(X), scratch=scratch)
-    assert S.svdq_device_error() == (10 << 8) | 1
-    assert S.svdq_device_error() == 0
+    check_activation(codes, sf, xl1, X, op, M, K, r)
+    rows = rows_every_block(M, extra=16, seed=M)
+    Y_ref, _, _, _ = O.linear_reference(X, op, b, rows=rows)
+    check_output(from_dev_bf16(Y)[rows], Y_ref)
 
 
 # ---------------------------------------------------- full-size workloads ----
@@ -296,7 +271,7 @@ def test_workload_parity(name):
     lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
     Xd = to_dev_bf16(X)
     codes, sf, xl1 = S.svdq_quantize_act(dw, Xd)
-    ws = torch.empty(S.svdq_act_workspace_bytes(M, K, r), dtype=torch.uint8, device="cuda")
+    ws = S.new_workspace(M, K, r)
     Y = S.svdq_linear_forward(dw, Xd, workspace=ws)
     torch.cuda.synchronize()
     check_activation(codes, sf, xl1, X, op, M, K, r)
@@ -389,7 +364,7 @@ def test_host_forward_strided_host_buffers():
     Yh = Yh_full[:, :N]
     Xd = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
     Yd = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    ws = torch.empty(S.svdq_act_workspace_bytes(M, K, r), dtype=torch.uint8, device="cuda")
+    ws = S.new_workspace(M, K, r)
     S.svdq_linear_forward_host(dw, Xh, Yh, Xd, Yd, ws)
     torch.cuda.synchronize()
     ref = from_dev_bf16(S.svdq_linear_forward(dw, to_dev_bf16(X)))
@@ -421,4 +396,72 @@ def test_forward_on_side_stream_without_workspace():
     torch.cuda.synchronize()
     for Y in outs:
         assert np.array_equal(from_dev_bf16(Y), ref)
+    assert S.svdq_device_error() == 0
+
+
+# ------------------------------------------------- fused GELU (MLP pair) ----
+
+def test_epilogue_gelu_matches_oracle_on_every_bf16():
+    """The GEMM epilogue's GELU against the oracle's bit-reproducible tanh
+    GELU (reading R11f) on every bf16 bit pattern: identical bits for every
+    finite input and for +-inf (NaN inputs give NaN on both sides)."""
+    S = _S()
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    got = from_dev_bf16(S.svdq_debug_gelu(to_dev_bf16(bits)))
+    want = O.gelu_bf16(bits)
+    g, w = F.bf16_bits_to_f64(got), F.bf16_bits_to_f64(want)
+    nan = np.isnan(F.bf16_bits_to_f64(bits))
+    assert np.array_equal(np.isnan(g), np.isnan(w))
+    both = ~np.isnan(w) & ~nan
+    bad = np.nonzero(got[both] != want[both])[0]
+    assert bad.size == 0, (bits[both][bad[:5]], got[both][bad[:5]], want[both][bad[:5]])
+
+
+@pytest.mark.parametrize("M,K,N,r", [(129, 320, 272, 32), (300, 768, 784, 16),
+                                     (4608, 3072, 12288, 32)])
+def test_gemm_gelu_equals_gemm_then_gelu(M, K, N, r):
+    """The fused epilogue writes exactly GELU of what the plain GEMM writes:
+    H == gelu(Y) bit for bit (the same bf16 y, the same GELU steps)."""
+    S = _S()
+    X, W, b = SI.random_layer(M + N, M, K, N)
+    lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
+    codes, sf, xl1 = S.svdq_quantize_act(dw, to_dev_bf16(X))
+    Y = S.svdq_gemm(dw, codes, sf, xl1, M)
+    H = S.svdq_gemm_gelu(dw, codes, sf, xl1, M)
+    torch.cuda.synchronize()
+    assert torch.equal(H.view(torch.int16), S.svdq_debug_gelu(Y).view(torch.int16))
+    assert S.svdq_device_error() == 0
+
+
+def test_mlp_pair_fused_parity():
+    """svdq_mlp_forward on the Flux MLP pair (config 2): fc1 with the GELU
+    epilogue, fc2 on its output.  H equals the oracle's GELU (reading R11f)
+    of fc1's bf16 output bit for bit; fc2's codes and scales bit-exact
+    against the oracle fed the GPU's H on every row; fc1's output and Y
+    within tolerance on at least one row of every 128-row block."""
+    S = _S()
+    wl = SI.make_workload("flux_mlp")
+    X = wl.X_bf16
+    fc1, fc2 = wl.layers
+    M = X.shape[0]
+    # fc2 is calibrated on the unfused chain's GELU output (the same values)
+    lp1, op1, dw1 = prepare(fc1.W, SI.channel_absmax(X), 32, fc1.bias_bf16)
+    Y1 = S.svdq_linear_forward(dw1, to_dev_bf16(X))
+    Hcal = from_dev_bf16(S.svdq_debug_gelu(Y1))
+    lp2, op2, dw2 = prepare(fc2.W, SI.channel_absmax(Hcal), 32, fc2.bias_bf16)
+    H, Y = S.svdq_mlp_forward(dw1, dw2, to_dev_bf16(X))
+    torch.cuda.synchronize()
+    Hb = from_dev_bf16(H)
+    # the fused GELU is exactly the oracle's GELU of fc1's bf16 output, and
+    # that output is within tolerance of fc1's float64 reference
+    assert np.array_equal(Hb, Hcal)
+    assert np.array_equal(Hb, O.gelu_bf16(from_dev_bf16(Y1)))
+    rows = rows_every_block(M, seed=21)
+    Y1r, _, _, _ = O.linear_reference(X, op1, fc1.bias_bf16, rows=rows)
+    check_output(from_dev_bf16(Y1)[rows], Y1r)
+    codes2, sf2, xl2 = S.svdq_quantize_act(dw2, H)
+    torch.cuda.synchronize()
+    check_activation(codes2, sf2, xl2, Hb, op2, M, fc2.spec.K, 32)
+    Y2r, _, _, _ = O.linear_reference(Hb, op2, fc2.bias_bf16, rows=rows)
+    check_output(from_dev_bf16(Y)[rows], Y2r)
     assert S.svdq_device_error() == 0

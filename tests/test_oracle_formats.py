@@ -98,10 +98,34 @@ def test_bf16_from_f64_brute_force():
         base = (1 + k / 128.0) * 2.0 ** rnd.randint(-20, 20)
         half = 2.0 ** -8 * 2.0 ** np.floor(np.log2(base))
         xs.extend([base + half, base + half * (1 + 2 ** -40), base + half * (1 - 2 ** -40)])
+    # the subnormal range and its edge: ties and near-ties of the 2^-133 grid
+    for k in range(300):
+        n = rnd.randint(0, 130)
+        xs.extend([(n + 0.5) * 2.0 ** -133, (n + 0.5 + 2 ** -30) * 2.0 ** -133,
+                   (n + rnd.random()) * 2.0 ** -133, -(n + rnd.random()) * 2.0 ** -133])
+    xs.extend([2.0 ** -126, 2.0 ** -126 * (1 - 2 ** -9), 2.0 ** -134, 2.0 ** -135, 1e-300])
     x = np.array(xs, np.float64)
     got = F.bf16_bits_to_f64(F.f64_to_bf16_bits(x))
     for xi, gi in zip(x, got):
         assert float(F.bf16_round_exact(float(xi))) == gi, xi
+
+
+def test_bf16_from_f32_matches_torch_including_subnormals():
+    """An independent conversion: torch's float32 -> bfloat16 (round to
+    nearest even, with subnormals), on every float32 with a 16-bit
+    significand prefix near each binade edge plus the whole subnormal
+    range's grid points and ties."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(4)
+    hi = rng.integers(0, 1 << 16, 20000, dtype=np.uint32)
+    lo = np.array([0, 0x7FFF, 0x8000, 0x8001, 0xFFFF], np.uint32)
+    bits = (hi[:, None] << 16 | lo[None, :]).reshape(-1)
+    f = bits.view(np.float32)
+    f = f[np.isfinite(f)]
+    ref = torch.from_numpy(f).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = F.f64_to_bf16_bits(f.astype(np.float64))
+    bad = np.nonzero(ref != got)[0]
+    assert bad.size == 0, (f[bad[:5]], ref[bad[:5]], got[bad[:5]])
 
 
 def _load_golden(golden_dir):

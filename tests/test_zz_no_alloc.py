@@ -36,7 +36,7 @@ def test_static_forward_rejects_before_any_launch():
     w = _fake_weight()
     X, Y = 0x20000000, 0x30000000
     Mmax = _max_rows(3072, 32)
-    assert Mmax == 7618   # the example the header gives
+    assert Mmax == 9033   # the example the header gives
     over = L.svdq_linear_forward_static(w, X, Mmax + 1, 3072, Y, 256, None)
     assert over == 4  # SVDQ_ERR_WORKSPACE
     assert L.svdq_linear_forward_static(w, X, 0, 3072, Y, 256, None) == 0

@@ -26,7 +26,8 @@ __all__ = [
     "SvdqError", "PackedWeight", "DeviceWeight", "svdq_query_sizes", "svdq_pack_weight",
     "svdq_quantize_act", "svdq_gemm", "svdq_linear_forward", "svdq_act_workspace_bytes",
     "svdq_linear_forward_host", "svdq_linear_forward_static", "svdq_unswizzle_scales",
-    "svdq_act_scratch_bytes", "new_workspace", "new_act_scratch",
+    "new_workspace", "svdq_gemm_gelu",
+    "svdq_mlp_forward", "svdq_mlp_workspace_bytes", "new_mlp_workspace", "svdq_debug_gelu",
     "svdq_device_error", "svdq_selftest_timeout", "svdq_debug_convert", "svdq_sf_tile_offset",
     "svdq_status_string", "SVDQW4A4Linear", "lib", "STATUS",
 ]
@@ -88,14 +89,18 @@ def _load() -> ctypes.CDLL:
                                          SZ, P]),
         "svdq_sf_tile_offset": (I64, [I, I, I]),
         "svdq_act_workspace_bytes": (SZ, [I, I, I]),
-        "svdq_act_scratch_bytes": (SZ, [I, I, I]),
-        "svdq_quantize_act": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P, P, P, SZ, P]),
+        "svdq_quantize_act": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P, P, P]),
         "svdq_gemm": (I, [ctypes.POINTER(SvdqWeight), P, P, P, I, P, I64, P]),
         "svdq_linear_forward": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P, SZ, P]),
         "svdq_linear_forward_static": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P]),
         "svdq_device_error": (I, [P, ctypes.POINTER(I)]),
         "svdq_selftest_timeout": (I, [I, P]),
         "svdq_debug_convert": (I, [P, P, P, I64, P]),
+        "svdq_debug_gelu": (I, [P, P, I64, P]),
+        "svdq_gemm_gelu": (I, [ctypes.POINTER(SvdqWeight), P, P, P, I, P, I64, P]),
+        "svdq_mlp_workspace_bytes": (SZ, [I, I, I, I, I]),
+        "svdq_mlp_forward": (I, [ctypes.POINTER(SvdqWeight), ctypes.POINTER(SvdqWeight), P, I, I64,
+                                 P, I64, P, I64, P, SZ, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -130,23 +135,11 @@ def svdq_act_workspace_bytes(M: int, K: int, r: int) -> int:
     return int(lib.svdq_act_workspace_bytes(M, K, r))
 
 
-def svdq_act_scratch_bytes(M: int, K: int, r: int) -> int:
-    return int(lib.svdq_act_scratch_bytes(M, K, r))
-
-
 def new_workspace(M: int, K: int, r: int, device="cuda"):
-    """A forward workspace, zeroed (its arrival counters must start at zero;
-    the library leaves them zero after every call)."""
+    """A forward workspace of svdq_act_workspace_bytes(M, K, r) bytes."""
     import torch
-    return torch.zeros(max(svdq_act_workspace_bytes(M, K, r), 256), dtype=torch.uint8,
+    return torch.empty(max(svdq_act_workspace_bytes(M, K, r), 256), dtype=torch.uint8,
                        device=device)
-
-
-def new_act_scratch(M: int, K: int, r: int, device="cuda"):
-    """Scratch for svdq_quantize_act, zeroed; None when r == 0."""
-    import torch
-    n = svdq_act_scratch_bytes(M, K, r)
-    return torch.zeros(n, dtype=torch.uint8, device=device) if n else None
 
 
 # ---------------------------------------------------------------- pack ----
@@ -310,11 +303,8 @@ def _keep_alive_on(stream, *tensors):
             t.record_stream(stream)
 
 
-def svdq_quantize_act(w: DeviceWeight, X, codes_x=None, sf_x=None, xl1=None, stream=None,
-                      scratch=None):
-    """Returns (codes_x u8 [M, K/2], sf_x u8 tiles, xl1 bf16 [M, klr] or None).
-    `scratch` (from new_act_scratch) lets the kernel split K; one is made
-    here when not given."""
+def svdq_quantize_act(w: DeviceWeight, X, codes_x=None, sf_x=None, xl1=None, stream=None):
+    """Returns (codes_x u8 [M, K/2], sf_x u8 tiles, xl1 bf16 [M, klr] or None)."""
     import torch
     _check_x(X, w.K)
     M = X.shape[0]
@@ -330,12 +320,8 @@ def svdq_quantize_act(w: DeviceWeight, X, codes_x=None, sf_x=None, xl1=None, str
     if xl1 is None and w.r > 0:
         xl1 = torch.empty((M, klr), dtype=torch.bfloat16, device=dev)
         made.append(xl1)
-    if scratch is None and w.r > 0:
-        scratch = new_act_scratch(M, w.K, w.r, dev)
-        made.append(scratch)
     _check(lib.svdq_quantize_act(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
-                                 codes_x.data_ptr(), sf_x.data_ptr(), _ptr(xl1), _ptr(scratch),
-                                 0 if scratch is None else scratch.numel(),
+                                 codes_x.data_ptr(), sf_x.data_ptr(), _ptr(xl1),
                                  _stream_ptr(stream)), "svdq_quantize_act")
     _keep_alive_on(stream, *made)
     return codes_x, sf_x, xl1
@@ -371,6 +357,64 @@ def svdq_linear_forward(w: DeviceWeight, X, Y=None, workspace=None, stream=None)
            "svdq_linear_forward")
     _keep_alive_on(stream, *made)
     return Y
+
+
+def svdq_gemm_gelu(w: DeviceWeight, codes_x, sf_x, xl1, M: int, H=None, stream=None):
+    """The GEMM with the MLP pair's GELU in its epilogue: H = GELU(layer output)."""
+    import torch
+    made = []
+    if H is None:
+        H = torch.empty((M, w.N), dtype=torch.bfloat16, device=codes_x.device)
+        made.append(H)
+    _check(lib.svdq_gemm_gelu(ctypes.byref(w.struct), codes_x.data_ptr(), sf_x.data_ptr(),
+                              _ptr(xl1), M, H.data_ptr(), H.stride(0), _stream_ptr(stream)),
+           "svdq_gemm_gelu")
+    _keep_alive_on(stream, *made)
+    return H
+
+
+def svdq_mlp_workspace_bytes(M: int, K1: int, N1: int, r1: int, r2: int) -> int:
+    return int(lib.svdq_mlp_workspace_bytes(M, K1, N1, r1, r2))
+
+
+def new_mlp_workspace(M: int, w1: "DeviceWeight", w2: "DeviceWeight", device="cuda"):
+    import torch
+    return torch.empty(max(svdq_mlp_workspace_bytes(M, w1.K, w1.N, w1.r, w2.r), 256),
+                       dtype=torch.uint8, device=device)
+
+
+def svdq_mlp_forward(w1: DeviceWeight, w2: DeviceWeight, X, H=None, Y=None, workspace=None,
+                     stream=None):
+    """fc1 -> GELU (fused into fc1's epilogue) -> fc2.  Returns (H, Y)."""
+    import torch
+    _check_x(X, w1.K)
+    M = X.shape[0]
+    made = []
+    if H is None:
+        H = torch.empty((M, w1.N), dtype=torch.bfloat16, device=X.device)
+        made.append(H)
+    if Y is None:
+        Y = torch.empty((M, w2.N), dtype=torch.bfloat16, device=X.device)
+        made.append(Y)
+    if workspace is None:
+        workspace = new_mlp_workspace(M, w1, w2, X.device)
+        made.append(workspace)
+    _check(lib.svdq_mlp_forward(ctypes.byref(w1.struct), ctypes.byref(w2.struct), X.data_ptr(), M,
+                                X.stride(0), H.data_ptr(), H.stride(0), Y.data_ptr(), Y.stride(0),
+                                workspace.data_ptr(), workspace.numel(), _stream_ptr(stream)),
+           "svdq_mlp_forward")
+    _keep_alive_on(stream, *made)
+    return H, Y
+
+
+def svdq_debug_gelu(y_bf16):
+    """The epilogue's GELU on a bf16 tensor (diagnostic)."""
+    import torch
+    y = y_bf16.contiguous()
+    out = torch.empty_like(y)
+    _check(lib.svdq_debug_gelu(y.data_ptr(), out.data_ptr(), y.numel(), _stream_ptr(None)),
+           "svdq_debug_gelu")
+    return out
 
 
 SVDQ_STATIC_WORKSPACE_BYTES = 16 << 20

@@ -1,5 +1,8 @@
-// Activation kernel of the SVDQuant W4A4 linear: smoothing, NVFP4
-// quantization and the fused low-rank down-projection, in one pass over X.
+// Activation kernel of the SVDQuant W4A4 linear, 128-row tiles: smoothing,
+// NVFP4 quantization and the fused low-rank down-projection, in one pass
+// over X.  This is the form for large token counts (one 128-row tile per SM
+// or more, about 15k rows and up); smaller batches use the 64-row kernel
+// (quantize_act64.cuh), which splits K within a cluster.
 //
 // The fusion is the one described for the Nunchaku engine in the Korean
 // rendering of "Bringing Nunchaku 4-bit diffusion inference to Diffusers"
@@ -7,14 +10,10 @@
 // is merged into the quantization kernel so the 16-bit branch costs no extra
 // pass over the activations.  The B200 design:
 //
-//   * one CTA owns 128 rows x a contiguous slice of K, walked in chunks of
-//     128 columns.  The host picks how many CTAs split K (S = 1 .. 8) so that
-//     the grid fills the machine in one wave.  128 rows per CTA (one full
-//     scale-factor atom row) means every byte of the low-rank operand that
-//     reaches an SM serves 128 rows of X.  The split ranks are independent
-//     CTAs, not a cluster: clusters of 4 or more CTAs with this much shared
-//     memory cannot all be resident at once on the 148 SMs, which cost half
-//     the machine at 4608 tokens;
+//   * one CTA owns 128 rows x all of K, walked in chunks of 128 columns.
+//     128 rows per CTA (one full scale-factor atom row) means every byte of
+//     the low-rank operand that reaches an SM serves 128 rows of X, and the
+//     scales of a chunk are two whole 512-byte atoms;
 //   * the slice's smoothing factors are loaded once (bulk copy) and stay in
 //     shared memory;
 //   * warp 0 streams X chunks [128 rows x 128 columns] bf16, as two
@@ -43,14 +42,12 @@
 //     [128 x 64] times L1' [2r x 64]^T into a 128 x 2r fp32 accumulator in
 //     tensor memory.  L1' holds smooth * L1 split into bf16 hi and lo
 //     halves, so X L1' = X_hat L1 to ~2^-16 relative (X itself is exact);
-//   * at the end the accumulator is read back (tcgen05.ld) and hi + lo
-//     columns are summed.  Without a K split the result goes straight out,
-//     times lr_scale, as a bf16 hi/lo pair for the GEMM's up-projection.  In
-//     a K split every rank writes its fp32 partial sums to a scratch buffer
-//     (L2-resident, 16 KB per rank and row block at r = 32) and bumps the row
-//     block's arrival counter; the rank that arrives last adds the S
-//     partials in rank order (deterministic whoever is last), stores the
-//     hi/lo pair and resets the counter to zero for the next launch.
+//   * at the end the accumulator is read back (tcgen05.ld), hi + lo columns
+//     are summed and stored times lr_scale as a bf16 hi/lo pair for the
+//     GEMM's up-projection.  (A K split of this kernel across CTAs was tried:
+//     its cross-CTA reduction of the partial sums cost more at the end of
+//     the kernel than the split gained, so small batches use the 64-row
+//     kernel instead.)
 #pragma once
 #include "ptx.cuh"
 
@@ -95,12 +92,6 @@ struct QALayout {
   uint32_t l1_off, stg_off, s_off, lut_off, bar_off;
   uint32_t total;            // bytes to request (incl. alignment slack)
 };
-
-// Scratch of a K split: a zeroed arrival counter per 128-row block (the
-// first QA_CNT_BYTES bytes), then fp32 partial sums [S][blocks * 128][r].
-constexpr uint32_t QA_CNT_BYTES = 4096;
-constexpr int QA_MAX_SPLITS = 8;
-constexpr int QA_MAX_PART_ROWS = 160 * QA_BM;   // S * blocks <= 160 whenever S > 1
 
 __host__ __device__ inline QALayout qa_layout(int r, int chunks_per_split) {
   QALayout L;
@@ -147,8 +138,6 @@ struct QAParams {
   const float* smooth;
   uint8_t* sf_x;
   uint16_t* xl1;
-  unsigned int* counters;   // K split: one zeroed counter per 128-row block
-  float* part;              // K split: fp32 partials [S][blocks * 128][r]
   int M, K, r, klr;
   int chunks_per_split;
   int num_splits;
@@ -204,15 +193,12 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   uint32_t* tmem_holder =
       reinterpret_cast<uint32_t*>(bars + 2 * XST + 2 * LST + 2 * NSTG + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_holder + 2);
   float* qlut = reinterpret_cast<float*>(smem + L.lut_off);  // 128 floats
   const float* s_sm = reinterpret_cast<const float*>(smem + L.s_off);
 
   const uint32_t warp = warp_id(), lane = lane_id();
-  const int split = blockIdx.x;  // rank in the K split
+  const int split = blockIdx.x;  // always 0: one CTA walks all of K
   const int rb = blockIdx.y;
-  const int S = p.num_splits;
-  const bool reduce = has_lr && S > 1;
   const int kchunks = ((p.K >> 6) + QA_BOXES - 1) / QA_BOXES;   // 128-column chunks
   const int k64 = p.K >> 6;
   const int c_begin = split * p.chunks_per_split;
@@ -240,7 +226,6 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
     mbar_init(s_bar, 1);
     mbar_init(drain_bar, 1);
     *abort_flag = 0;
-    *last_flag = 0;
     mbar_fence_init();
   }
   if (warp == 0 && lane == 0) {
@@ -505,15 +490,11 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
     const int row_t = quad * 32 + lane;
     const int row = rb * QA_BM + row_t;
     const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16);
-    const size_t part_rows = (size_t)gridDim.y * QA_BM;
-    float own[8][4];                              // this rank's sums of the slot's groups
 #pragma unroll
     for (int g = 0; g < 8; ++g) {
       if (g < cw4) {
         const int col = slot * 4 * cw4 + 4 * g;   // first of the group's 4 columns
         uint32_t hi[4], lo[4];
-        // (a rank whose share of K is empty contributes zeros: its
-        // accumulator was never written)
         if (ok && nchunks > 0) {
           tmem_ld4(tbase + col, hi);
           tmem_ld4(tbase + r + col, lo);
@@ -522,65 +503,18 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) hi[j] = lo[j] = 0u;
         }
+        float sum[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) own[g][j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
-        if (reduce)
-          *reinterpret_cast<float4*>(p.part + ((size_t)split * part_rows + row) * r + col) =
-              make_float4(own[g][0], own[g][1], own[g][2], own[g][3]);
+        for (int j = 0; j < 4; ++j) sum[j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
+        if (row < p.M)
+          store_hi_lo4(sum, p.lr_scale, p.xl1 + (size_t)row * p.klr + col,
+                       p.xl1 + (size_t)row * p.klr + r + col);
       }
     }
-    bool last = !reduce;
-    if (reduce) {
-      // every partial of this CTA is written before the count goes up; the
-      // CTA that brings the count to S sees every rank's partials
-      __threadfence();
-      named_barrier_sync(1, 32 * QA_QWARPS);
-      if (warp == QA_QWARP0 && lane == 0) {
-        const unsigned int prev = atomicAdd(p.counters + rb, 1u);
-        if (prev >= (unsigned int)S) record_error((10u << 8) | kid);  // counters not zeroed
-        if (prev == (unsigned int)(S - 1)) {
-          *last_flag = 1;
-          p.counters[rb] = 0u;   // ready for the next launch (stream order)
-        }
-      }
-      named_barrier_sync(1, 32 * QA_QWARPS);
-      last = *last_flag != 0;
-      if (last) __threadfence();
-    }
-    if (last) {
-#pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        if (g < cw4) {
-          const int col = slot * 4 * cw4 + 4 * g;
-          float sum[4];
-          if (reduce) {
-            // the S partials in rank order, this rank's from registers
-            for (int sr = 0; sr < S; ++sr) {
-              float t[4];
-              if (sr == split) {
-#pragma unroll
-                for (int j = 0; j < 4; ++j) t[j] = own[g][j];
-              } else {
-                const float4 v = ld_cg_f4(p.part + ((size_t)sr * part_rows + row) * r + col);
-                t[0] = v.x; t[1] = v.y; t[2] = v.z; t[3] = v.w;
-              }
-#pragma unroll
-              for (int j = 0; j < 4; ++j) sum[j] = sr == 0 ? t[j] : sum[j] + t[j];
-            }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) sum[j] = own[g][j];
-          }
-          if (row < p.M)
-            store_hi_lo4(sum, p.lr_scale, p.xl1 + (size_t)row * p.klr + col,
-                         p.xl1 + (size_t)row * p.klr + r + col);
-        }
-      }
-      // zero columns [2r, klr) of this row block
-      if (slot == 0 && row < p.M) {
-        for (int cpad = 2 * r; cpad < p.klr; cpad += 8)
-          *reinterpret_cast<uint4*>(p.xl1 + (size_t)row * p.klr + cpad) = make_uint4(0, 0, 0, 0);
-      }
+    // zero columns [2r, klr) of this row block
+    if (slot == 0 && row < p.M) {
+      for (int cpad = 2 * r; cpad < p.klr; cpad += 8)
+        *reinterpret_cast<uint4*>(p.xl1 + (size_t)row * p.klr + cpad) = make_uint4(0, 0, 0, 0);
     }
   }
 

@@ -13,6 +13,7 @@
 #include "../../include/svdq.h"
 #include "ptx.cuh"
 #include "quantize_act.cuh"
+#include "quantize_act64.cuh"
 #include "w4a4_gemm.cuh"
 
 namespace svdq_dev {
@@ -30,6 +31,15 @@ __global__ void selftest_timeout_kernel(uint64_t timeout_ns) {
   if (threadIdx.x == 0)
     mbar_wait(smem_u32(&bar), 0, timeout_ns, &abort_flag, (7u << 8) | 3u);
   __syncthreads();
+}
+
+// The epilogue's GELU on arbitrary bf16 inputs, one value per thread.
+__global__ void debug_gelu_kernel(const uint16_t* in, uint16_t* out, int64_t n, GeluConsts gc) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const float y = __uint_as_float((uint32_t)in[i] << 16);
+  const float h = gelu_bf16_value(y, gc);
+  out[i] = (uint16_t)(__float_as_uint(h) >> 16);
 }
 
 // The hardware conversions of the activation kernel, one value per thread.
@@ -61,7 +71,14 @@ struct DeviceInfo {
   bool ok = false;
   int num_sms = 0;
   bool attrs_set = false;
+  // max co-resident clusters of the 64-row activation kernel per cluster
+  // size S (1..8; every shared-memory plan holds one CTA per SM, so r does
+  // not matter); -1 = not queried yet
+  int q64_clusters[9];
   int gemm_pairs = -1;  // max co-resident CTA pairs of the GEMM kernel
+  DeviceInfo() {
+    for (int& v : q64_clusters) v = -1;
+  }
 };
 constexpr int kMaxDevices = 64;
 DeviceInfo g_dev[kMaxDevices];
@@ -89,8 +106,11 @@ svdq_status device_check(int* sms) {
   if (!d.ok) return SVDQ_ERR_UNSUPPORTED_ARCH;
   if (!d.attrs_set) {
     const uint32_t qa_max = 1024u + QA_SMEM_BUDGET + 512u;  // every qa_layout fits
+    const uint32_t q64_max = 1024u + Q64_SMEM_BUDGET + 512u;
     if (cudaFuncSetAttribute(quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)qa_max) != cudaSuccess ||
+        cudaFuncSetAttribute(quantize_act64_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)q64_max) != cudaSuccess ||
         cudaFuncSetAttribute(w4a4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)gemm_smem_bytes()) != cudaSuccess) {
       cudaGetLastError();
@@ -153,38 +173,125 @@ cudaLaunchAttribute pdl_attr() {
   return a;
 }
 
-// K split S (1 .. 8): the largest such that the grid (S x row blocks) stays
-// within one wave of one CTA per SM, every rank gets a chunk of K, the
-// split's shared-memory plan keeps a deep enough activation ring, and (with
-// a low-rank branch) the partial sums fit the scratch buffer.  No scratch
-// means no split.
-int choose_splits(int tiles, int kchunks, int r, int sms, bool have_scratch) {
+// Largest K split S (cluster size when the low-rank branch needs the
+// cross-CTA reduction) such that the whole grid is resident in one wave and
+// the split's shared-memory plan keeps a deep enough activation ring.
+int choose_splits64(int tiles, int kchunks, int r, int sms) {
+  int dev = 0;
+  cudaGetDevice(&dev);
   int best = 1;
-  if (r > 0 && !have_scratch) return 1;
-  for (int S = 2; S <= QA_MAX_SPLITS; ++S) {
+  for (int S = 2; S <= 8; ++S) {
     if (S > kchunks || tiles * S > sms) break;
-    if (r > 0 && (size_t)S * tiles * QA_BM > (size_t)QA_MAX_PART_ROWS) break;
     const int cps = (kchunks + S - 1) / S;
-    if ((kchunks + cps - 1) / cps < S) continue;      // a rank would get no chunk
-    const QALayout L = qa_layout(r, cps);
-    if (L.xst < QA_MIN_XST) continue;
+    const Q64Layout L = q64_layout(r, cps, S);
+    if (L.xst < Q64_MIN_XST) break;
+    if (r > 0) {
+      std::lock_guard<std::mutex> lk(g_mu);   // the caches are shared by host threads
+      int& cached = g_dev[dev].q64_clusters[S];
+      if (cached < 0) {
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof(cfg));
+        cfg.gridDim = dim3((unsigned)S, 1, 1);
+        cfg.blockDim = dim3(Q64_THREADS, 1, 1);
+        cfg.dynamicSmemBytes = L.total;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = (unsigned)S;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, quantize_act64_kernel, &cfg) != cudaSuccess) {
+          cudaGetLastError();
+          n = 0;
+        }
+        cached = n;
+      }
+      if (tiles > cached) continue;
+    }
     best = S;
   }
   return best;
 }
 
-svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int64_t ldx,
-                            uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, void* scratch,
-                            size_t scratch_bytes, cudaStream_t s, int sms) {
+svdq_status launch_quantize64(const svdq_weight* w, const uint16_t* X, int M, int64_t ldx,
+                            uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, cudaStream_t s,
+                            int sms) {
+  const int K = w->K, r = w->r;
+  // 64-row tiles covering whole 128-row scale atoms (padding rows get zero
+  // scales)
+  const int tiles = 2 * ((M + 127) / 128);
+  const int KC = (K / 64 + Q64_BOXES - 1) / Q64_BOXES;  // 128-column chunks
+  int S = choose_splits64(tiles, KC, r, sms);
+  const int cps = (KC + S - 1) / S;
+  S = (KC + cps - 1) / cps;
+  const Q64Layout L = q64_layout(r, cps, S);
+  if (L.xst < Q64_MIN_XST) return SVDQ_ERR_INVALID_ARG;  // K too large for one CTA's slice
+
+  CUtensorMap tm_x, tm_l1;
+  std::memset(&tm_l1, 0, sizeof(tm_l1));
+  if (!make_map(&tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, (uint64_t)K, (uint64_t)M,
+                (uint64_t)ldx * 2, 64, Q64_BM))
+    return SVDQ_ERR_CUDA;
+  if (r > 0 && !make_map(&tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, w->l1_mma, (uint64_t)K,
+                         (uint64_t)(2 * r), (uint64_t)K * 2, 64, (uint32_t)(2 * r)))
+    return SVDQ_ERR_CUDA;
+
+  Q64Params p;
+  p.smooth = w->smooth;
+  p.codes_x = codes_x;
+  p.sf_x = sf_x;
+  p.xl1 = xl1;
+  p.M = M;
+  p.K = K;
+  p.r = r;
+  p.klr = klr_of(r);
+  p.chunks_per_split = cps;
+  p.num_splits = S;
+  p.L = L;
+  uint32_t cols = 32;
+  while (cols < (uint32_t)(2 * r)) cols <<= 1;
+  p.tmem_cols = cols;
+  p.g_x = w->g_x;
+  p.gs_x = w->gs_x;
+  p.lr_scale = w->lr_scale;
+  p.timeout_ns = kDefaultTimeoutNs;
+
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)S, (unsigned)tiles, 1);
+  cfg.blockDim = dim3(Q64_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = L.total;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0] = pdl_attr();
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (r > 0 && S > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)S;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
+  if (cudaLaunchKernelEx(&cfg, quantize_act64_kernel, tm_x, tm_l1, p) != cudaSuccess) {
+    cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
+}
+
+// The 128-row kernel: one CTA per 128-row block, all of K.
+svdq_status launch_quantize128(const svdq_weight* w, const uint16_t* X, int M, int64_t ldx,
+                               uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, cudaStream_t s) {
   const int K = w->K, r = w->r;
   // 128-row tiles: one scale-factor atom row each (padding rows get zero
   // scales)
   const int tiles = (M + QA_BM - 1) / QA_BM;
   const int KC = (K / 64 + QA_BOXES - 1) / QA_BOXES;  // 128-column chunks
-  const bool have_scratch = scratch != nullptr && scratch_bytes >= svdq_act_scratch_bytes(M, K, r) &&
-                            svdq_act_scratch_bytes(M, K, r) > 0;
-  const int S = choose_splits(tiles, KC, r, sms, have_scratch);
-  const int cps = (KC + S - 1) / S;
+  const int S = 1;
+  const int cps = KC;
   const QALayout L = qa_layout(r, cps);
   if (L.xst < QA_MIN_XST || L.nstg < QA_MIN_NSTG || (r > 0 && L.lst < 1))
     return SVDQ_ERR_INVALID_ARG;  // K too large for one CTA's slice
@@ -206,9 +313,6 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
   p.smooth = w->smooth;
   p.sf_x = sf_x;
   p.xl1 = xl1;
-  p.counters = static_cast<unsigned int*>(scratch);
-  p.part = scratch ? reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) + QA_CNT_BYTES)
-                   : nullptr;
   p.M = M;
   p.K = K;
   p.r = r;
@@ -241,6 +345,20 @@ svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int6
   return SVDQ_OK;
 }
 
+// Which activation kernel: the 128-row kernel once 128-row blocks alone
+// nearly fill the machine (>= 120 blocks on 148 SMs: every byte of the
+// low-rank operand then serves 128 rows and no K split is needed); below
+// that the 64-row kernel, whose K split within a cluster keeps every SM
+// busy.
+svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int64_t ldx,
+                            uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, cudaStream_t s,
+                            int sms) {
+  const int tiles128 = (M + QA_BM - 1) / QA_BM;
+  if (tiles128 * 148 >= 120 * sms)
+    return launch_quantize128(w, X, M, ldx, codes_x, sf_x, xl1, s);
+  return launch_quantize64(w, X, M, ldx, codes_x, sf_x, xl1, s, sms);
+}
+
 int gemm_max_pairs(int sms) {
   int dev = 0;
   cudaGetDevice(&dev);
@@ -271,7 +389,7 @@ int gemm_max_pairs(int sms) {
 
 svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint8_t* sf_x,
                         const uint16_t* xl1, int M, uint16_t* Y, int64_t ldy, cudaStream_t s,
-                        int sms) {
+                        int sms, bool gelu = false) {
   const int N = w->N, K = w->K, r = w->r, klr = klr_of(r);
   CUtensorMap ta, tb, tsa, tsb, talr, tblr, ty;
   std::memset(&talr, 0, sizeof(talr));
@@ -307,6 +425,8 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   p.klr = klr;
   p.alpha = w->alpha;
   p.timeout_ns = kDefaultTimeoutNs;
+  p.gelu = gelu ? 1 : 0;
+  p.gc = gelu_consts_host();
   const int tiles = ((M + 2 * G_BM - 1) / (2 * G_BM)) * ((N + G_BN - 1) / G_BN);
   const int pairs = std::max(1, std::min(tiles, gemm_max_pairs(sms)));
   cudaLaunchConfig_t cfg;
@@ -330,7 +450,6 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   return SVDQ_OK;
 }
 
-size_t ws_scratch(int M, int K, int r) { return rup(svdq_act_scratch_bytes(M, K, r), 256); }
 size_t ws_codes(int M, int K) { return rup((size_t)M * (K / 2), 256); }
 size_t ws_sf(int M, int K) { return rup(rup((size_t)M, 128) * (K / 16), 256); }
 size_t ws_xl1(int M, int r) { return rup((size_t)M * klr_of(r) * 2, 256); }
@@ -353,35 +472,25 @@ extern "C" const char* svdq_status_string(svdq_status s) {
 
 extern "C" const char* svdq_version(void) { return "svdq-b200 0.1"; }
 
-extern "C" size_t svdq_act_scratch_bytes(int M, int K, int r) {
-  if (M < 0 || K <= 0 || K % 64 || r < 0 || r > 128 || (r && r % 16)) return 0;
-  if (r == 0) return 0;
-  const size_t rows = std::min((size_t)QA_MAX_SPLITS * rup((size_t)M, QA_BM),
-                               (size_t)QA_MAX_PART_ROWS);
-  return QA_CNT_BYTES + rows * (size_t)r * 4;
-}
-
 extern "C" size_t svdq_act_workspace_bytes(int M, int K, int r) {
   if (M < 0 || K <= 0 || K % 64 || r < 0 || r > 128 || (r && r % 16)) return 0;
-  return ws_scratch(M, K, r) + ws_codes(M, K) + ws_sf(M, K) + (r > 0 ? ws_xl1(M, r) : 0);
+  return ws_codes(M, K) + ws_sf(M, K) + (r > 0 ? ws_xl1(M, r) : 0);
 }
 
 extern "C" svdq_status svdq_quantize_act(const svdq_weight* w, const uint16_t* X, int M,
                                          int64_t ldx, uint8_t* codes_x, uint8_t* sf_x,
-                                         uint16_t* xl1, void* scratch, size_t scratch_bytes,
-                                         void* stream) {
+                                         uint16_t* xl1, void* stream) {
   svdq_status st = check_weight(w);
   if (st != SVDQ_OK) return st;
   if (M < 0 || ldx < w->K) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   if (!X || !codes_x || !sf_x || (w->r > 0 && !xl1)) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || ldx % 8 || !aligned16(codes_x) || !aligned16(sf_x) ||
-      (xl1 && !aligned16(xl1)) || (scratch && (reinterpret_cast<uintptr_t>(scratch) & 255)))
+      (xl1 && !aligned16(xl1)))
     return SVDQ_ERR_MISALIGNED;
   int sms = 0;
   if ((st = device_check(&sms)) != SVDQ_OK) return st;
-  return launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, scratch, scratch_bytes,
-                         (cudaStream_t)stream, sms);
+  return launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, (cudaStream_t)stream, sms);
 }
 
 extern "C" svdq_status svdq_gemm(const svdq_weight* w, const uint8_t* codes_x,
@@ -400,6 +509,74 @@ extern "C" svdq_status svdq_gemm(const svdq_weight* w, const uint8_t* codes_x,
   return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, (cudaStream_t)stream, sms);
 }
 
+extern "C" svdq_status svdq_gemm_gelu(const svdq_weight* w, const uint8_t* codes_x,
+                                      const uint8_t* sf_x, const uint16_t* xl1, int M,
+                                      uint16_t* H, int64_t ldh, void* stream) {
+  svdq_status st = check_weight(w);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || ldh < w->N) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!codes_x || !sf_x || !H || (w->r > 0 && !xl1)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(codes_x) || !aligned16(sf_x) || !aligned16(H) || ldh % 8 ||
+      (xl1 && !aligned16(xl1)))
+    return SVDQ_ERR_MISALIGNED;
+  int sms = 0;
+  if ((st = device_check(&sms)) != SVDQ_OK) return st;
+  return launch_gemm(w, codes_x, sf_x, xl1, M, H, ldh, (cudaStream_t)stream, sms, true);
+}
+
+extern "C" size_t svdq_mlp_workspace_bytes(int M, int K1, int N1, int r1, int r2) {
+  const size_t a = svdq_act_workspace_bytes(M, K1, r1), b = svdq_act_workspace_bytes(M, N1, r2);
+  if (!a || !b) return 0;
+  return std::max(a, b);
+}
+
+extern "C" svdq_status svdq_mlp_forward(const svdq_weight* w1, const svdq_weight* w2,
+                                        const uint16_t* X, int M, int64_t ldx, uint16_t* H,
+                                        int64_t ldh, uint16_t* Y, int64_t ldy, void* workspace,
+                                        size_t ws_bytes, void* stream) {
+  svdq_status st = check_weight(w1);
+  if (st != SVDQ_OK) return st;
+  if ((st = check_weight(w2)) != SVDQ_OK) return st;
+  if (w2->K != w1->N) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0 || ldx < w1->K || ldh < w1->N || ldy < w2->N) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !H || !Y || !workspace) return SVDQ_ERR_INVALID_ARG;
+  if (ws_bytes < svdq_mlp_workspace_bytes(M, w1->K, w1->N, w1->r, w2->r)) return SVDQ_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return SVDQ_ERR_MISALIGNED;
+  if (!aligned16(X) || !aligned16(H) || !aligned16(Y) || ldx % 8 || ldh % 8 || ldy % 8)
+    return SVDQ_ERR_MISALIGNED;
+  int sms = 0;
+  if ((st = device_check(&sms)) != SVDQ_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  for (int layer = 0; layer < 2; ++layer) {
+    const svdq_weight* w = layer == 0 ? w1 : w2;
+    const uint16_t* in = layer == 0 ? X : H;
+    const int64_t ldin = layer == 0 ? ldx : ldh;
+    uint8_t* codes_x = static_cast<uint8_t*>(workspace);
+    uint8_t* sf_x = codes_x + ws_codes(M, w->K);
+    uint16_t* xl1 = w->r > 0 ? reinterpret_cast<uint16_t*>(sf_x + ws_sf(M, w->K)) : nullptr;
+    if ((st = launch_quantize(w, in, M, ldin, codes_x, sf_x, xl1, s, sms)) != SVDQ_OK) return st;
+    if ((st = launch_gemm(w, codes_x, sf_x, xl1, M, layer == 0 ? H : Y, layer == 0 ? ldh : ldy, s,
+                          sms, layer == 0)) != SVDQ_OK)
+      return st;
+  }
+  return SVDQ_OK;
+}
+
+extern "C" svdq_status svdq_debug_gelu(const uint16_t* in, uint16_t* out, int64_t n,
+                                       void* stream) {
+  if (n < 0 || (n > 0 && (!in || !out))) return SVDQ_ERR_INVALID_ARG;
+  if (n == 0) return SVDQ_OK;
+  svdq_status st = device_check(nullptr);
+  if (st != SVDQ_OK) return st;
+  const int64_t blocks = (n + 255) / 256;
+  if (blocks > 0x7FFFFFFF) return SVDQ_ERR_INVALID_ARG;
+  debug_gelu_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(in, out, n,
+                                                                       gelu_consts_host());
+  return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
 extern "C" svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t* X, int M,
                                            int64_t ldx, uint16_t* Y, int64_t ldy,
                                            void* workspace, size_t ws_bytes, void* stream) {
@@ -414,15 +591,11 @@ extern "C" svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t*
   int sms = 0;
   if ((st = device_check(&sms)) != SVDQ_OK) return st;
   uint8_t* base = static_cast<uint8_t*>(workspace);
-  uint8_t* scratch = base;
-  const size_t scratch_bytes = ws_scratch(M, w->K, w->r);
-  uint8_t* codes_x = base + scratch_bytes;
+  uint8_t* codes_x = base;
   uint8_t* sf_x = codes_x + ws_codes(M, w->K);
   uint16_t* xl1 = w->r > 0 ? reinterpret_cast<uint16_t*>(sf_x + ws_sf(M, w->K)) : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
-  if ((st = launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, scratch_bytes ? scratch : nullptr,
-                            scratch_bytes, s, sms)) != SVDQ_OK)
-    return st;
+  if ((st = launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, s, sms)) != SVDQ_OK) return st;
   return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, s, sms);
 }
 

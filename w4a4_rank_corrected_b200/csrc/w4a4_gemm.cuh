@@ -44,6 +44,7 @@
 //     and row, which scattered each warp instruction over 32 rows and held
 //     the MMA issuer back.
 #pragma once
+#include "gelu.cuh"
 #include "ptx.cuh"
 
 namespace svdq_dev {
@@ -87,6 +88,8 @@ struct GemmParams {
   int M, N, K, r, klr;
   float alpha;
   uint64_t timeout_ns;
+  int gelu;          // 1: the epilogue writes GELU(bf16(y)) (first linear of an MLP pair)
+  GeluConsts gc;
 };
 
 __global__ void __launch_bounds__(G_THREADS, 1)
@@ -401,9 +404,13 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           uint32_t o[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const float y0 = fmaf(alpha, __uint_as_float(acc[ch][cb + 2 * q]), bt[c0 + 2 * q]);
-            const float y1 =
-                fmaf(alpha, __uint_as_float(acc[ch][cb + 2 * q + 1]), bt[c0 + 2 * q + 1]);
+            float y0 = fmaf(alpha, __uint_as_float(acc[ch][cb + 2 * q]), bt[c0 + 2 * q]);
+            float y1 = fmaf(alpha, __uint_as_float(acc[ch][cb + 2 * q + 1]), bt[c0 + 2 * q + 1]);
+            if (p.gelu) {
+              // the layer's bf16 output, then the MLP pair's GELU of it
+              y0 = gelu_bf16_value(__bfloat162float(__float2bfloat16_rn(y0)), p.gc);
+              y1 = gelu_bf16_value(__bfloat162float(__float2bfloat16_rn(y1)), p.gc);
+            }
             o[q] = pack_bf16x2(y0, y1);
           }
           st_shared_v4(obuf + row_t * 128 + ((j ^ (row_t & 7)) << 4), o[0], o[1], o[2], o[3]);
