@@ -231,12 +231,11 @@ svdq_status svdq_gemm(const svdq_weight* w, const uint8_t* codes_x,
  * the pages name as part of the original engine's speed ("Bringing Nunchaku
  * 4-bit diffusion inference to Diffusers", Vietnamese rendering, section
  * "Introducing Nunchaku Lite").  Writes H = bf16(GELU(bf16(alpha * acc +
- * bias))) instead of Y; GELU is the tanh form evaluated as y / (1 +
- * e^(-2u)), u = sqrt(2/pi) (y + 0.044715 y^3), in a fixed sequence of
- * round-to-nearest fp32 operations (e^x from basic operations: a degree-7
- * Taylor series of 2^f times 2^n), so it is reproducible bit for bit; see
- * svdq_debug_gelu.  H is never materialized as Y first.  Arguments and
- * errors as svdq_gemm (H in place of Y). */
+ * bias))) instead of Y: the tanh form of GELU, evaluated as y / (1 +
+ * 2^(-2 log2(e) u)), u = sqrt(2/pi) (y + 0.044715 y^3), with the hardware's
+ * approximate base-2 exponential and reciprocal (a few 1e-7 relative before
+ * the bf16 rounding; within one bf16 unit of the correctly rounded GELU, see
+ * svdq_debug_gelu).  Arguments and errors as svdq_gemm (H in place of Y). */
 svdq_status svdq_gemm_gelu(const svdq_weight* w, const uint8_t* codes_x,
                            const uint8_t* sf_x, const uint16_t* xl1, int M,
                            uint16_t* H, int64_t ldh, void* stream);

@@ -34,11 +34,11 @@ __global__ void selftest_timeout_kernel(uint64_t timeout_ns) {
 }
 
 // The epilogue's GELU on arbitrary bf16 inputs, one value per thread.
-__global__ void debug_gelu_kernel(const uint16_t* in, uint16_t* out, int64_t n, GeluConsts gc) {
+__global__ void debug_gelu_kernel(const uint16_t* in, uint16_t* out, int64_t n) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n) return;
   const float y = __uint_as_float((uint32_t)in[i] << 16);
-  const float h = gelu_bf16_value(y, gc);
+  const float h = gelu_bf16_value(y);
   out[i] = (uint16_t)(__float_as_uint(h) >> 16);
 }
 
@@ -426,7 +426,6 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   p.alpha = w->alpha;
   p.timeout_ns = kDefaultTimeoutNs;
   p.gelu = gelu ? 1 : 0;
-  p.gc = gelu_consts_host();
   const int tiles = ((M + 2 * G_BM - 1) / (2 * G_BM)) * ((N + G_BN - 1) / G_BN);
   const int pairs = std::max(1, std::min(tiles, gemm_max_pairs(sms)));
   cudaLaunchConfig_t cfg;
@@ -572,8 +571,7 @@ extern "C" svdq_status svdq_debug_gelu(const uint16_t* in, uint16_t* out, int64_
   if (st != SVDQ_OK) return st;
   const int64_t blocks = (n + 255) / 256;
   if (blocks > 0x7FFFFFFF) return SVDQ_ERR_INVALID_ARG;
-  debug_gelu_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(in, out, n,
-                                                                       gelu_consts_host());
+  debug_gelu_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(in, out, n);
   return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 

@@ -89,7 +89,6 @@ struct GemmParams {
   float alpha;
   uint64_t timeout_ns;
   int gelu;          // 1: the epilogue writes GELU(bf16(y)) (first linear of an MLP pair)
-  GeluConsts gc;
 };
 
 __global__ void __launch_bounds__(G_THREADS, 1)
@@ -408,8 +407,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
             float y1 = fmaf(alpha, __uint_as_float(acc[ch][cb + 2 * q + 1]), bt[c0 + 2 * q + 1]);
             if (p.gelu) {
               // the layer's bf16 output, then the MLP pair's GELU of it
-              y0 = gelu_bf16_value(__bfloat162float(__float2bfloat16_rn(y0)), p.gc);
-              y1 = gelu_bf16_value(__bfloat162float(__float2bfloat16_rn(y1)), p.gc);
+              y0 = gelu_bf16_value(__bfloat162float(__float2bfloat16_rn(y0)));
+              y1 = gelu_bf16_value(__bfloat162float(__float2bfloat16_rn(y1)));
             }
             o[q] = pack_bf16x2(y0, y1);
           }
