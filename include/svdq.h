@@ -268,6 +268,42 @@ svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t* X,
                                 void* workspace, size_t ws_bytes,
                                 void* stream);
 
+/* ------------------------------------------------ dynamic (per-token) --
+ * The dynamic alternative to the static activation tensor scale, for inputs
+ * outside the calibration range.  The pages fix only the static form (one
+ * fp32 tensor scale, NVFP4 of the hardware-support table of "Bringing
+ * Nunchaku 4-bit diffusion inference to Diffusers"); here each row (token)
+ * of X_hat is its own tensor for the same recipe:
+ *   A_m = max_k |fp32(x_mk smooth_k)|, g_m = fp32(2688 / A_m),
+ *   gs_m = fp32(448 / A_m) (both 1 when A_m = 0), lr_m = fp32(g_m g_w),
+ *   alpha_m = fp32(1 / lr_m);
+ * row m is quantized with g_m, gs_m (q = fp32(g_m / e4m3(sf)) per group),
+ * its low-rank operand is pre-scaled by lr_m, and the GEMM scales its
+ * output row by alpha_m.  Row scales: 16 bytes per row, {g, gs, lr, alpha}
+ * as fp32, device memory, 16-byte aligned.
+ */
+/* One pass over X: the row scales of every row (memory-bound). */
+svdq_status svdq_act_row_scales(const svdq_weight* w, const uint16_t* X, int M, int64_t ldx,
+                                void* row_scales, void* stream);
+/* svdq_quantize_act with each row's own scales (from svdq_act_row_scales). */
+svdq_status svdq_quantize_act_dynamic(const svdq_weight* w, const uint16_t* X, int M,
+                                      int64_t ldx, const void* row_scales, uint8_t* codes_x,
+                                      uint8_t* sf_x, uint16_t* xl1, void* stream);
+/* svdq_gemm with each output row scaled by its alpha_m. */
+svdq_status svdq_gemm_dynamic(const svdq_weight* w, const uint8_t* codes_x,
+                              const uint8_t* sf_x, const uint16_t* xl1,
+                              const void* row_scales, int M, uint16_t* Y, int64_t ldy,
+                              void* stream);
+/* Workspace of svdq_linear_forward_dynamic: the static forward's plus 16
+ * bytes per row (rounded to 256).  0 on bad arguments. */
+size_t svdq_dyn_workspace_bytes(int M, int K, int r);
+/* The layer with per-token scales: row scales, activation kernel, GEMM on
+ * one stream.  Arguments and errors as svdq_linear_forward (workspace >=
+ * svdq_dyn_workspace_bytes). */
+svdq_status svdq_linear_forward_dynamic(const svdq_weight* w, const uint16_t* X, int M,
+                                        int64_t ldx, uint16_t* Y, int64_t ldy,
+                                        void* workspace, size_t ws_bytes, void* stream);
+
 /* svdq_linear_forward_host: svdq_linear_forward for activations and outputs
  * that live in host memory (the drop-in layer's view of a host batch):
  * copies X_host to X_dev, runs the layer, copies Y_dev back to Y_host, all

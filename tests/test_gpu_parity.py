@@ -232,7 +232,7 @@ def test_activation_kernel_repeats_bit_identical():
 
 
 @pytest.mark.parametrize("M,K,N,r", [(15361, 320, 64, 48), (16000, 3072, 128, 32),
-                                     (15500, 192, 64, 0), (20000, 1024, 96, 128)])
+                                     (15500, 192, 64, 0), (20000, 1024, 256, 128)])
 def test_activation_kernel_128_row_tiles(M, K, N, r):
     """Batches of about 15k rows and more take the 128-row activation kernel
     (the others the 64-row one): bit-exact codes and scales on every row,
@@ -478,4 +478,62 @@ def test_mlp_pair_fused_parity():
     check_activation(codes2, sf2, xl2, Hb, op2, M, fc2.spec.K, 32)
     Y2r, _, _, _ = O.linear_reference(Hb, op2, fc2.bias_bf16, rows=rows)
     check_output(from_dev_bf16(Y)[rows], Y2r)
+    assert S.svdq_device_error() == 0
+
+
+# ------------------------------------------- dynamic per-token scales ----
+
+def _check_dynamic(S, dw, op, X, b, rows=None):
+    M, K = X.shape
+    Xd = to_dev_bf16(X)
+    rs = S.svdq_act_row_scales(dw, Xd)
+    codes, sf, xl1 = S.svdq_quantize_act_dynamic(dw, Xd, rs)
+    Y = S.svdq_linear_forward_dynamic(dw, Xd)
+    torch.cuda.synchronize()
+    xh, cq, sq, A = O.quantize_activation_dynamic(X, op.s)
+    # the row scales: g, gs bit-exact against the oracle's R4 of each row
+    r_ = rs.cpu().numpy()
+    g_ref = np.array([O.tensor_encode_scale(a) for a in A], np.float32)
+    gs_ref = np.array([O.block_scale_factor(a) for a in A], np.float32)
+    assert np.array_equal(r_[:, 0], g_ref) and np.array_equal(r_[:, 1], gs_ref)
+    assert np.array_equal(codes.cpu().numpy(), O.pack_nibbles(cq)), "dynamic codes differ"
+    assert np.array_equal(O.sf_from_mma_tiles(sf.cpu().numpy(), M, K), sq), "dynamic scales differ"
+    idx = np.arange(M) if rows is None else rows
+    Y_ref, _, _, _, _ = O.linear_reference_dynamic(X, op, b, rows=idx)
+    check_output(from_dev_bf16(Y)[idx], Y_ref)
+    return from_dev_bf16(Y)
+
+
+@pytest.mark.parametrize("name", ["flux_qkv", "sweep_r32", "sweep_m64"])
+def test_dynamic_scale_parity(name):
+    """Per-token activation scales (reading R5d) on configs 1 and 3: row
+    scales, codes and scales bit-exact against the oracle on every row; the
+    output against the oracle's per-row reference (one row of every 128-row
+    block, or every row for small M)."""
+    S = _S()
+    X, W, b, r = _workload_layer(name)
+    M = X.shape[0]
+    lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
+    _check_dynamic(S, dw, op, X, b, rows=None if M <= 1024 else rows_every_block(M, seed=3))
+    assert S.svdq_device_error() == 0
+
+
+def test_dynamic_scale_beyond_calibration():
+    """Inputs 16x beyond the calibration range: the static scale saturates
+    (E4M3 at 448, E2M1 at 6) and loses the layer; per-token scales keep it
+    within tolerance.  Large M takes the 128-row kernel."""
+    S = _S()
+    for M in (512, 16384):
+        K, N, r = 3072, 512, 32
+        Xc, W, b = SI.random_layer(60 + M, M, K, N)
+        lp, op, dw = prepare(W, SI.channel_absmax(Xc), r, b)       # calibrated on Xc
+        Xb = SI.f32_to_bf16_bits(SI.bf16_bits_to_f32(Xc) * np.float32(16.0))
+        rows = rows_every_block(M, extra=8, seed=M)
+        Yd = _check_dynamic(S, dw, op, Xb, b, rows=rows)
+        Ys = from_dev_bf16(S.svdq_linear_forward(dw, to_dev_bf16(Xb)))
+        exact = (SI.bf16_bits_to_f32(Xb).astype(np.float64)[rows] @ W.astype(np.float64).T
+                 + F.bf16_bits_to_f64(b)[None, :])
+        err_d = np.linalg.norm(F.bf16_bits_to_f64(Yd[rows]) - exact) / np.linalg.norm(exact)
+        err_s = np.linalg.norm(F.bf16_bits_to_f64(Ys[rows]) - exact) / np.linalg.norm(exact)
+        assert err_d < 0.2 * err_s, (err_d, err_s)
     assert S.svdq_device_error() == 0

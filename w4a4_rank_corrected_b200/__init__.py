@@ -28,6 +28,8 @@ __all__ = [
     "svdq_linear_forward_host", "svdq_linear_forward_static", "svdq_unswizzle_scales",
     "new_workspace", "svdq_gemm_gelu",
     "svdq_mlp_forward", "svdq_mlp_workspace_bytes", "new_mlp_workspace", "svdq_debug_gelu",
+    "svdq_act_row_scales", "svdq_quantize_act_dynamic", "svdq_gemm_dynamic",
+    "svdq_dyn_workspace_bytes", "svdq_linear_forward_dynamic",
     "svdq_device_error", "svdq_selftest_timeout", "svdq_debug_convert", "svdq_sf_tile_offset",
     "svdq_status_string", "SVDQW4A4Linear", "lib", "STATUS",
 ]
@@ -97,6 +99,12 @@ def _load() -> ctypes.CDLL:
         "svdq_selftest_timeout": (I, [I, P]),
         "svdq_debug_convert": (I, [P, P, P, I64, P]),
         "svdq_debug_gelu": (I, [P, P, I64, P]),
+        "svdq_act_row_scales": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P]),
+        "svdq_quantize_act_dynamic": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P, P, P, P]),
+        "svdq_gemm_dynamic": (I, [ctypes.POINTER(SvdqWeight), P, P, P, P, I, P, I64, P]),
+        "svdq_dyn_workspace_bytes": (SZ, [I, I, I]),
+        "svdq_linear_forward_dynamic": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P, SZ,
+                                            P]),
         "svdq_gemm_gelu": (I, [ctypes.POINTER(SvdqWeight), P, P, P, I, P, I64, P]),
         "svdq_mlp_workspace_bytes": (SZ, [I, I, I, I, I]),
         "svdq_mlp_forward": (I, [ctypes.POINTER(SvdqWeight), ctypes.POINTER(SvdqWeight), P, I, I64,
@@ -415,6 +423,76 @@ def svdq_debug_gelu(y_bf16):
     _check(lib.svdq_debug_gelu(y.data_ptr(), out.data_ptr(), y.numel(), _stream_ptr(None)),
            "svdq_debug_gelu")
     return out
+
+
+# ------------------------------------------------ dynamic (per-token) ----
+
+def svdq_act_row_scales(w: DeviceWeight, X, stream=None):
+    """Per-row scales {g, gs, lr, alpha} (fp32 [M, 4]) of the dynamic mode."""
+    import torch
+    _check_x(X, w.K)
+    M = X.shape[0]
+    rs = torch.empty((M, 4), dtype=torch.float32, device=X.device)
+    _check(lib.svdq_act_row_scales(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
+                                   rs.data_ptr(), _stream_ptr(stream)), "svdq_act_row_scales")
+    _keep_alive_on(stream, rs)
+    return rs
+
+
+def svdq_quantize_act_dynamic(w: DeviceWeight, X, row_scales, stream=None):
+    """(codes_x, sf_x, xl1) with each row's own tensor scales."""
+    import torch
+    _check_x(X, w.K)
+    M = X.shape[0]
+    klr, sf_bytes = _act_shapes(M, w.K, w.r)
+    codes_x = torch.empty((M, w.K // 2), dtype=torch.uint8, device=X.device)
+    sf_x = torch.empty(sf_bytes, dtype=torch.uint8, device=X.device)
+    xl1 = torch.empty((M, klr), dtype=torch.bfloat16, device=X.device) if w.r else None
+    _check(lib.svdq_quantize_act_dynamic(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
+                                         row_scales.data_ptr(), codes_x.data_ptr(),
+                                         sf_x.data_ptr(), _ptr(xl1), _stream_ptr(stream)),
+           "svdq_quantize_act_dynamic")
+    _keep_alive_on(stream, codes_x, sf_x, xl1)
+    return codes_x, sf_x, xl1
+
+
+def svdq_gemm_dynamic(w: DeviceWeight, codes_x, sf_x, xl1, row_scales, M: int, Y=None,
+                      stream=None):
+    import torch
+    made = []
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=codes_x.device)
+        made.append(Y)
+    _check(lib.svdq_gemm_dynamic(ctypes.byref(w.struct), codes_x.data_ptr(), sf_x.data_ptr(),
+                                 _ptr(xl1), row_scales.data_ptr(), M, Y.data_ptr(), Y.stride(0),
+                                 _stream_ptr(stream)), "svdq_gemm_dynamic")
+    _keep_alive_on(stream, *made)
+    return Y
+
+
+def svdq_dyn_workspace_bytes(M: int, K: int, r: int) -> int:
+    return int(lib.svdq_dyn_workspace_bytes(M, K, r))
+
+
+def svdq_linear_forward_dynamic(w: DeviceWeight, X, Y=None, workspace=None, stream=None):
+    """The layer with per-token activation scales."""
+    import torch
+    _check_x(X, w.K)
+    M = X.shape[0]
+    made = []
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+        made.append(Y)
+    if workspace is None:
+        workspace = torch.empty(max(svdq_dyn_workspace_bytes(M, w.K, w.r), 256),
+                                dtype=torch.uint8, device=X.device)
+        made.append(workspace)
+    _check(lib.svdq_linear_forward_dynamic(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
+                                           Y.data_ptr(), Y.stride(0), workspace.data_ptr(),
+                                           workspace.numel(), _stream_ptr(stream)),
+           "svdq_linear_forward_dynamic")
+    _keep_alive_on(stream, *made)
+    return Y
 
 
 SVDQ_STATIC_WORKSPACE_BYTES = 16 << 20

@@ -50,6 +50,7 @@
 //     kernel instead.)
 #pragma once
 #include "ptx.cuh"
+#include "row_scales.cuh"
 
 namespace svdq_dev {
 
@@ -138,6 +139,7 @@ struct QAParams {
   const float* smooth;
   uint8_t* sf_x;
   uint16_t* xl1;
+  const RowScale* row_scales;   // per-row scales (dynamic mode) or NULL (static)
   int M, K, r, klr;
   int chunks_per_split;
   int num_splits;
@@ -370,7 +372,6 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
   } else {
     // ---------------------------------------------- NVFP4 quantization ----
     const int qw = warp - QA_QWARP0;
-    const float gs = p.gs_x;
     bool ok = nchunks == 0 || mbar_wait_warp(s_bar, 0, p.timeout_ns, abort_flag, (3u << 8) | kid);
     for (int u = qw; ok && u < QA_UNITS * nchunks; u += QA_QWARPS) {
       const int i = u / QA_UNITS;
@@ -383,6 +384,14 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
       const int row_t = 32 * quarter + lane;
       const int col0 = (c_begin + cl) * 128 + 64 * box;   // first column of the unit
       const bool live = col0 < p.K;                       // else the zero box past K
+      // this row's tensor scales: the static ones, or (dynamic mode) its own
+      const int row = rb * QA_BM + row_t;
+      const bool dyn = p.row_scales != nullptr;
+      float g_row = p.g_x, gs = p.gs_x;
+      if (dyn && row < p.M) {
+        g_row = p.row_scales[row].g;
+        gs = p.row_scales[row].gs;
+      }
       uint4 xr[8];
       if (live) {
         // copy this lane's row segment into registers, then hand the stage
@@ -438,7 +447,8 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
           const float a = fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
                                 fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
           const uint32_t code = cvt_e4m3x2(__fmul_rn(a, gs), 0.0f) & 0xFF;
-          const float q = qlut[code];
+          const float q = !dyn ? qlut[code]
+                               : (code == 0 ? 0.0f : __fdiv_rn(g_row, e4m3_to_f32(code)));
           const uint64_t qq = pack_f32x2(q, q);
           float t0[8], t1[8];
 #pragma unroll
@@ -507,7 +517,8 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) sum[j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
         if (row < p.M)
-          store_hi_lo4(sum, p.lr_scale, p.xl1 + (size_t)row * p.klr + col,
+          store_hi_lo4(sum, p.row_scales ? p.row_scales[row].lr : p.lr_scale,
+                       p.xl1 + (size_t)row * p.klr + col,
                        p.xl1 + (size_t)row * p.klr + r + col);
       }
     }

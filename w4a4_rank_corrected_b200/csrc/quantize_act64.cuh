@@ -47,6 +47,7 @@
 //     up-projection.
 #pragma once
 #include "ptx.cuh"
+#include "row_scales.cuh"
 
 namespace svdq_dev {
 
@@ -121,6 +122,7 @@ struct Q64Params {
   uint8_t* codes_x;
   uint8_t* sf_x;
   uint16_t* xl1;
+  const RowScale* row_scales;   // per-row scales (dynamic mode) or NULL (static)
   int M, K, r, klr;
   int chunks_per_split;
   int num_splits;
@@ -327,7 +329,6 @@ __global__ void __launch_bounds__(Q64_THREADS, 1)
   } else {
     // ---------------------------------------------- NVFP4 quantization ----
     const int qw = warp - Q64_QWARP0;
-    const float gs = p.gs_x;
     bool ok = nchunks == 0 || mbar_wait_warp(s_bar, 0, p.timeout_ns, abort_flag, (3u << 8) | kid);
     for (int u = qw; ok && u < Q64_UNITS * nchunks; u += Q64_QWARPS) {
       const int i = u / Q64_UNITS;
@@ -338,6 +339,13 @@ __global__ void __launch_bounds__(Q64_THREADS, 1)
       if (!mbar_wait_warp(x_full0 + 8 * st, ph, p.timeout_ns, abort_flag, (3u << 8) | kid)) break;
       const int row_t = 32 * (u & 1) + lane;
       const int row = rb * Q64_BM + row_t;
+      // this row's tensor scales: the static ones, or (dynamic mode) its own
+      const bool dyn = p.row_scales != nullptr;
+      float g_row = p.g_x, gs = p.gs_x;
+      if (dyn && row < p.M) {
+        g_row = p.row_scales[row].g;
+        gs = p.row_scales[row].gs;
+      }
       const int col0 = (c_begin + cl) * 128 + 64 * box;   // first column of the unit
       const uint8_t* xrow = smem + st * Q64_X_BYTES + box * Q64_BOX_BYTES + row_t * 128;
       // copy this lane's row segment into registers, then hand the stage
@@ -390,7 +398,8 @@ __global__ void __launch_bounds__(Q64_THREADS, 1)
         const float a = fmaxf(fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3])),
                               fmaxf(fmaxf(m[4], m[5]), fmaxf(m[6], m[7])));
         const uint32_t code = cvt_e4m3x2(__fmul_rn(a, gs), 0.0f) & 0xFF;
-        const float q = qlut[code];
+        const float q = !dyn ? qlut[code]
+                             : (code == 0 ? 0.0f : __fdiv_rn(g_row, e4m3_to_f32(code)));
         const uint64_t qq = pack_f32x2(q, q);
         float t0[8], t1[8];
 #pragma unroll
@@ -440,7 +449,8 @@ __global__ void __launch_bounds__(Q64_THREADS, 1)
       for (int j = 0; j < 16; ++j) part[j] = __uint_as_float(hi[j]) + __uint_as_float(lo[j]);
       if (!reduce) {
         if (own && lrow < p.M)
-          store_hi_lo16(part, p.lr_scale, p.xl1 + (size_t)lrow * p.klr + 16 * ci,
+          store_hi_lo16(part, p.row_scales ? p.row_scales[lrow].lr : p.lr_scale,
+                        p.xl1 + (size_t)lrow * p.klr + 16 * ci,
                         p.xl1 + (size_t)lrow * p.klr + r + 16 * ci);
       } else if (split != 0) {
         // partial sums [row][r] of rank `split` into rank 0's buffer split-1
@@ -469,7 +479,8 @@ __global__ void __launch_bounds__(Q64_THREADS, 1)
               }
             }
           }
-          store_hi_lo16(part, p.lr_scale, p.xl1 + (size_t)lrow * p.klr + 16 * ci,
+          store_hi_lo16(part, p.row_scales ? p.row_scales[lrow].lr : p.lr_scale,
+                        p.xl1 + (size_t)lrow * p.klr + 16 * ci,
                         p.xl1 + (size_t)lrow * p.klr + r + 16 * ci);
         }
       }

@@ -14,6 +14,7 @@
 #include "ptx.cuh"
 #include "quantize_act.cuh"
 #include "quantize_act64.cuh"
+#include "row_scales.cuh"
 #include "w4a4_gemm.cuh"
 
 namespace svdq_dev {
@@ -216,8 +217,8 @@ int choose_splits64(int tiles, int kchunks, int r, int sms) {
 }
 
 svdq_status launch_quantize64(const svdq_weight* w, const uint16_t* X, int M, int64_t ldx,
-                            uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, cudaStream_t s,
-                            int sms) {
+                              uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, cudaStream_t s,
+                              int sms, const RowScale* rs) {
   const int K = w->K, r = w->r;
   // 64-row tiles covering whole 128-row scale atoms (padding rows get zero
   // scales)
@@ -239,6 +240,7 @@ svdq_status launch_quantize64(const svdq_weight* w, const uint16_t* X, int M, in
     return SVDQ_ERR_CUDA;
 
   Q64Params p;
+  p.row_scales = rs;
   p.smooth = w->smooth;
   p.codes_x = codes_x;
   p.sf_x = sf_x;
@@ -284,7 +286,8 @@ svdq_status launch_quantize64(const svdq_weight* w, const uint16_t* X, int M, in
 
 // The 128-row kernel: one CTA per 128-row block, all of K.
 svdq_status launch_quantize128(const svdq_weight* w, const uint16_t* X, int M, int64_t ldx,
-                               uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, cudaStream_t s) {
+                               uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, cudaStream_t s,
+                               const RowScale* rs) {
   const int K = w->K, r = w->r;
   // 128-row tiles: one scale-factor atom row each (padding rows get zero
   // scales)
@@ -310,6 +313,7 @@ svdq_status launch_quantize128(const svdq_weight* w, const uint16_t* X, int M, i
     return SVDQ_ERR_CUDA;
 
   QAParams p;
+  p.row_scales = rs;
   p.smooth = w->smooth;
   p.sf_x = sf_x;
   p.xl1 = xl1;
@@ -352,11 +356,20 @@ svdq_status launch_quantize128(const svdq_weight* w, const uint16_t* X, int M, i
 // busy.
 svdq_status launch_quantize(const svdq_weight* w, const uint16_t* X, int M, int64_t ldx,
                             uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1, cudaStream_t s,
-                            int sms) {
+                            int sms, const RowScale* rs = nullptr) {
   const int tiles128 = (M + QA_BM - 1) / QA_BM;
   if (tiles128 * 148 >= 120 * sms)
-    return launch_quantize128(w, X, M, ldx, codes_x, sf_x, xl1, s);
-  return launch_quantize64(w, X, M, ldx, codes_x, sf_x, xl1, s, sms);
+    return launch_quantize128(w, X, M, ldx, codes_x, sf_x, xl1, s, rs);
+  return launch_quantize64(w, X, M, ldx, codes_x, sf_x, xl1, s, sms, rs);
+}
+
+// The per-row scales of the dynamic mode: one warp per row, 8 rows per CTA.
+svdq_status launch_row_scales(const svdq_weight* w, const uint16_t* X, int M, int64_t ldx,
+                              RowScale* rs, cudaStream_t s, int sms) {
+  const int blocks = std::max(1, std::min((M + 7) / 8, 16 * sms));
+  row_scales_kernel<<<blocks, 256, 0, s>>>(X, ldx, w->smooth, M, w->K, w->g_w, rs);
+  if (cudaGetLastError() != cudaSuccess) return SVDQ_ERR_CUDA;
+  return SVDQ_OK;
 }
 
 int gemm_max_pairs(int sms) {
@@ -389,7 +402,7 @@ int gemm_max_pairs(int sms) {
 
 svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint8_t* sf_x,
                         const uint16_t* xl1, int M, uint16_t* Y, int64_t ldy, cudaStream_t s,
-                        int sms, bool gelu = false) {
+                        int sms, bool gelu = false, const RowScale* rs = nullptr) {
   const int N = w->N, K = w->K, r = w->r, klr = klr_of(r);
   CUtensorMap ta, tb, tsa, tsb, talr, tblr, ty;
   std::memset(&talr, 0, sizeof(talr));
@@ -426,6 +439,7 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   p.alpha = w->alpha;
   p.timeout_ns = kDefaultTimeoutNs;
   p.gelu = gelu ? 1 : 0;
+  p.row_scales = rs;
   const int tiles = ((M + 2 * G_BM - 1) / (2 * G_BM)) * ((N + G_BN - 1) / G_BN);
   const int pairs = std::max(1, std::min(tiles, gemm_max_pairs(sms)));
   cudaLaunchConfig_t cfg;
@@ -573,6 +587,86 @@ extern "C" svdq_status svdq_debug_gelu(const uint16_t* in, uint16_t* out, int64_
   if (blocks > 0x7FFFFFFF) return SVDQ_ERR_INVALID_ARG;
   debug_gelu_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(in, out, n);
   return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+extern "C" svdq_status svdq_act_row_scales(const svdq_weight* w, const uint16_t* X, int M,
+                                           int64_t ldx, void* row_scales, void* stream) {
+  svdq_status st = check_weight(w);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || ldx < w->K) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !row_scales) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || ldx % 8 || !aligned16(row_scales)) return SVDQ_ERR_MISALIGNED;
+  int sms = 0;
+  if ((st = device_check(&sms)) != SVDQ_OK) return st;
+  return launch_row_scales(w, X, M, ldx, static_cast<RowScale*>(row_scales), (cudaStream_t)stream,
+                           sms);
+}
+
+extern "C" svdq_status svdq_quantize_act_dynamic(const svdq_weight* w, const uint16_t* X, int M,
+                                                 int64_t ldx, const void* row_scales,
+                                                 uint8_t* codes_x, uint8_t* sf_x, uint16_t* xl1,
+                                                 void* stream) {
+  svdq_status st = check_weight(w);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || ldx < w->K) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !row_scales || !codes_x || !sf_x || (w->r > 0 && !xl1)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || ldx % 8 || !aligned16(codes_x) || !aligned16(sf_x) ||
+      !aligned16(row_scales) || (xl1 && !aligned16(xl1)))
+    return SVDQ_ERR_MISALIGNED;
+  int sms = 0;
+  if ((st = device_check(&sms)) != SVDQ_OK) return st;
+  return launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, (cudaStream_t)stream, sms,
+                         static_cast<const RowScale*>(row_scales));
+}
+
+extern "C" svdq_status svdq_gemm_dynamic(const svdq_weight* w, const uint8_t* codes_x,
+                                         const uint8_t* sf_x, const uint16_t* xl1,
+                                         const void* row_scales, int M, uint16_t* Y, int64_t ldy,
+                                         void* stream) {
+  svdq_status st = check_weight(w);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || ldy < w->N) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!codes_x || !sf_x || !Y || !row_scales || (w->r > 0 && !xl1)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(codes_x) || !aligned16(sf_x) || !aligned16(Y) || ldy % 8 ||
+      !aligned16(row_scales) || (xl1 && !aligned16(xl1)))
+    return SVDQ_ERR_MISALIGNED;
+  int sms = 0;
+  if ((st = device_check(&sms)) != SVDQ_OK) return st;
+  return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, (cudaStream_t)stream, sms, false,
+                     static_cast<const RowScale*>(row_scales));
+}
+
+extern "C" size_t svdq_dyn_workspace_bytes(int M, int K, int r) {
+  const size_t a = svdq_act_workspace_bytes(M, K, r);
+  if (!a) return 0;
+  return a + rup((size_t)M * sizeof(RowScale), 256);
+}
+
+extern "C" svdq_status svdq_linear_forward_dynamic(const svdq_weight* w, const uint16_t* X, int M,
+                                                   int64_t ldx, uint16_t* Y, int64_t ldy,
+                                                   void* workspace, size_t ws_bytes, void* stream) {
+  svdq_status st = check_weight(w);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || ldx < w->K || ldy < w->N) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!X || !Y || !workspace) return SVDQ_ERR_INVALID_ARG;
+  if (ws_bytes < svdq_dyn_workspace_bytes(M, w->K, w->r)) return SVDQ_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255) != 0) return SVDQ_ERR_MISALIGNED;
+  if (!aligned16(X) || !aligned16(Y) || ldx % 8 || ldy % 8) return SVDQ_ERR_MISALIGNED;
+  int sms = 0;
+  if ((st = device_check(&sms)) != SVDQ_OK) return st;
+  uint8_t* base = static_cast<uint8_t*>(workspace);
+  uint8_t* codes_x = base;
+  uint8_t* sf_x = codes_x + ws_codes(M, w->K);
+  uint16_t* xl1 = w->r > 0 ? reinterpret_cast<uint16_t*>(sf_x + ws_sf(M, w->K)) : nullptr;
+  RowScale* rs = reinterpret_cast<RowScale*>(base + svdq_act_workspace_bytes(M, w->K, w->r));
+  cudaStream_t s = (cudaStream_t)stream;
+  if ((st = launch_row_scales(w, X, M, ldx, rs, s, sms)) != SVDQ_OK) return st;
+  if ((st = launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, s, sms, rs)) != SVDQ_OK) return st;
+  return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, s, sms, false, rs);
 }
 
 extern "C" svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t* X, int M,

@@ -46,6 +46,7 @@
 #pragma once
 #include "gelu.cuh"
 #include "ptx.cuh"
+#include "row_scales.cuh"
 
 namespace svdq_dev {
 
@@ -89,6 +90,7 @@ struct GemmParams {
   float alpha;
   uint64_t timeout_ns;
   int gelu;          // 1: the epilogue writes GELU(bf16(y)) (first linear of an MLP pair)
+  const RowScale* row_scales;   // per-row output scale alpha_m (dynamic mode) or NULL
 };
 
 __global__ void __launch_bounds__(G_THREADS, 1)
@@ -344,7 +346,6 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const int quad = warp & 3;                 // tensor-memory lane quarter
     const int half = (warp - 2) >> 2;          // columns [128 half, 128 half + 128)
     const int et = threadIdx.x - 64;           // 0..255
-    const float alpha = p.alpha;
     const int row_t = quad * 32 + lane;        // this thread's row of the CTA's 128
     const uint32_t obuf = out_s + half * G_OUT_HALF_BYTES;
     const uint32_t staged = out_staged0 + 8 * half, freed = out_free0 + 8 * half;
@@ -378,6 +379,9 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(lead_acc_empty);   // accumulator free again
       const int row0 = mb * 2 * G_BM + (int)rank * G_BM;   // first row of this CTA's box
+      // the output scale: static, or this row's own (dynamic mode)
+      const float alpha = (p.row_scales && row0 + row_t < M) ? p.row_scales[row0 + row_t].alpha
+                                                             : p.alpha;
       bool ok = true;
 #pragma unroll
       for (int sb = 0; sb < 2; ++sb, ++use) {
