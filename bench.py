@@ -57,6 +57,8 @@ def parse_args():
                     help="replay each step from a CUDA graph (small layers are launch-bound)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--awq", type=int, default=0, metavar="M",
+                    help="time the AWQ W4A16 modulation linear (3072 -> 18432) at batch M instead")
     ap.add_argument("--pair", action="store_true",
                     help="time the MLP pair of the workload (fc1 -> GELU -> fc2) as one step")
     ap.add_argument("--kernel-seconds", type=float, default=1.0,
@@ -653,10 +655,69 @@ def run_pair(args):
         print(json.dumps(out), flush=True)
 
 
+def run_awq(args):
+    """The AWQ W4A16 linear of a Flux modulation projection (adanorm_zero:
+    hidden 3072 -> 6 x 3072), batch M = args.awq conditioning vectors,
+    synthetic weights N(0, 0.02^2) and inputs N(0, 1).  Memory-bound: the
+    roofline is the weight stream at the measured copy bandwidth."""
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import w4a4_rank_corrected_b200 as S
+    M, K, N, group = args.awq, 3072, 6 * 3072, 128
+    rng = np.random.default_rng(5 + rank)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    b = SI.f32_to_bf16_bits((rng.standard_normal(N) * 0.01).astype(np.float32))
+    X0 = SI.f32_to_bf16_bits(rng.standard_normal((M, K)).astype(np.float32))
+    nsets = 8     # 8 x 28 MB of weights > L2
+    ws = [S.svdq_awq_pack(W, group, bias_bf16=b).to_device(dev) for _ in range(1)]
+    ws = ws + [S.AwqWeight(N, K, group, ws[0].q, ws[0].zeros, ws[0].scales, b).to_device(dev)
+               for _ in range(nsets - 1)]
+    Xd = torch.from_numpy(X0.view(np.int16)).to(dev).view(torch.bfloat16)
+    Ys = [torch.empty((M, N), dtype=torch.bfloat16, device=dev) for _ in range(nsets)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    for i in range(max(3, args.warmup)):
+        S.svdq_awq_linear(ws[i % nsets], Xd, Ys[i % nsets])
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(200):
+            S.svdq_awq_linear(ws[i % nsets], Xd, Ys[i % nsets])
+    g.replay()
+    torch.cuda.synchronize(dev)
+    a, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = max(1, args.steps // 200)
+    a.record()
+    for _ in range(reps):
+        g.replay()
+    e.record()
+    torch.cuda.synchronize(dev)
+    clocks = sampler.stop()
+    us = a.elapsed_time(e) / (reps * 200) * 1e3
+    byts = N * K // 2 + N * (K // group) * 3 + M * K * 2 + M * N * 2 + N * 2
+    peaks, src = load_peaks()
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    out = {"metric": "AWQ W4A16 linear GB/s (weight stream) and us/layer", "value": round(byts / us / 1e3, 1),
+           "unit": "GB/s", "n_gpus": 1, "steps": reps * 200, "warmup": args.warmup,
+           "ms_per_step": round(us / 1e3, 6), "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "int4 weights x bf16", "data": "synthetic",
+           "config": {"workload": f"awq_w4a16 modulation linear K={K} N={N} group={group}, M={M}",
+                      "us_per_layer": round(us, 2)},
+           "roofline": {"bound": "hbm", "achieved": round(byts / us / 1e3, 1), "peak": hbm,
+                        "unit": "GB/s", "frac": round(byts / us / 1e3 / hbm, 4),
+                        "algorithmic_bytes": byts, "peak_source": src},
+           "gpu_launches": reps * 200, "clocks": clocks}
+    print(json.dumps(out), flush=True)
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
+    elif args.awq:
+        run_awq(args)
     elif args.pair:
         run_pair(args)
     else:

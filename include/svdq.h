@@ -350,6 +350,40 @@ svdq_status svdq_linear_forward_static(const svdq_weight* w, const uint16_t* X,
                                        int M, int64_t ldx, uint16_t* Y,
                                        int64_t ldy, void* stream);
 
+/* ------------------------------------------------------ AWQ W4A16 linear --
+ * The second kernel family of the pages: 4-bit weights with 16-bit
+ * activations, for the memory-bound, precision-sensitive modulation and
+ * adaptive-normalization projections ("Bringing Nunchaku 4-bit diffusion
+ * inference to Diffusers", Russian rendering, section "Technical details and
+ * hardware support"; the Korean rendering's kernel-family list).  The pages
+ * fix only "INT4 weights, 16-bit activations"; the format is AWQ's
+ * asymmetric INT4 per group of `group` input channels:
+ *   range [wmin, wmax] of the group widened to include 0,
+ *   scale = fp16(max(wmax - wmin, 1e-5) / 15), z = clamp(rint(-wmin/scale), 0, 15),
+ *   q = clamp(rint(w / scale) + z, 0, 15) (rint: ties to even, in double),
+ *   dequantized weight (q - z) * scale.
+ * (AWQ's activation-aware per-channel scale search is an offline step and
+ * is not part of these calls.)
+ *
+ * svdq_awq_pack (host, synchronous): W fp32 [N][K] -> q_packed u8 [N][K/2]
+ * (even k in the low nibble), zeros u8 [N][K/group], scales fp16 bit
+ * patterns [N][K/group].  group a multiple of 32 dividing K (128 is AWQ's
+ * usual group).  Errors: INVALID_ARG, NUMERIC (non-finite W). */
+svdq_status svdq_awq_pack(const float* W, int N, int K, int group, uint8_t* q_packed,
+                          uint8_t* zeros, uint16_t* scales);
+
+/* svdq_awq_linear (GPU): Y = X dequant(W)^T + bias, fp32 accumulation, one
+ * bf16 rounding.  For the batch sizes of modulation layers: 1 <= M <= 8 (a
+ * memory-bound matrix-vector product over the weight stream) and M * K * 4
+ * <= 200 KB.
+ *   q, zeros, scales  device, as svdq_awq_pack writes them (q 16-byte aligned)
+ *   bias   device bf16 [N] or NULL
+ *   X      device bf16 [M][ldx], ldx >= K;  Y device bf16 [M][ldy], ldy >= N
+ * Errors: INVALID_ARG (shapes, M > 8, NULLs), MISALIGNED, UNSUPPORTED_ARCH. */
+svdq_status svdq_awq_linear(const uint8_t* q, const uint8_t* zeros, const uint16_t* scales,
+                            const uint16_t* bias, int N, int K, int group, const uint16_t* X,
+                            int M, int64_t ldx, uint16_t* Y, int64_t ldy, void* stream);
+
 /* ------------------------------------------------------------- failure --
  * Every wait inside the kernels is bounded (about one second).  A kernel
  * that gives up records a code in a device-side word and exits cleanly

@@ -1,0 +1,68 @@
+"""AWQ W4A16 linear: host pack against the oracle (CPU, bit-exact), the
+entry points' argument checks (CPU), and the GPU kernel against the
+oracle's float64 layer (GPU)."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import svdq_inputs as SI
+import w4a4_rank_corrected_b200 as S
+from oracle import awq as A
+from oracle import formats as F
+
+
+@pytest.mark.parametrize("N,K,group,seed", [(16, 128, 128, 0), (100, 3072, 128, 1),
+                                            (33, 512, 64, 2), (8, 256, 32, 3)])
+def test_awq_pack_matches_oracle(N, K, group, seed):
+    rng = np.random.default_rng(seed)
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    W[0, :group] = 0.0                       # an all-zero group
+    W[1, :group] = 0.01                      # a constant group
+    W[2, :] *= 50.0                          # a large row
+    aw = S.svdq_awq_pack(W, group)
+    q, z, sb = A.awq_quantize(W, group)
+    assert np.array_equal(aw.scales, sb)
+    assert np.array_equal(aw.zeros, z)
+    assert np.array_equal(aw.q, A.pack_nibbles_awq(q))
+
+
+def test_awq_argument_validation():
+    L = S.lib
+    W = np.zeros((4, 128), np.float32)
+    q = np.empty((4, 64), np.uint8)
+    z = np.empty((4, 1), np.uint8)
+    sc = np.empty((4, 1), np.uint16)
+    assert L.svdq_awq_pack(W.ctypes.data, 4, 128, 48, q.ctypes.data, z.ctypes.data, sc.ctypes.data) == 1
+    assert L.svdq_awq_pack(None, 4, 128, 128, q.ctypes.data, z.ctypes.data, sc.ctypes.data) == 1
+    W[0, 0] = np.inf
+    assert L.svdq_awq_pack(W.ctypes.data, 4, 128, 128, q.ctypes.data, z.ctypes.data, sc.ctypes.data) == 7
+    Q, Z, SC, X, Y = 0x10000000, 0x20000000, 0x30000000, 0x40000000, 0x50000000
+    f = L.svdq_awq_linear
+    assert f(Q, Z, SC, None, 64, 128, 128, X, 9, 128, Y, 64, None) == 1        # M > 8
+    assert f(Q, Z, SC, None, 64, 128, 100, X, 1, 128, Y, 64, None) == 1       # group
+    assert f(Q, Z, SC, None, 64, 128, 128, X, 1, 100, Y, 64, None) == 1       # ldx < K
+    assert f(Q + 8, Z, SC, None, 64, 128, 128, X, 1, 128, Y, 64, None) == 3   # alignment
+    assert f(Q, Z, SC, None, 64, 8192, 128, X, 8, 8192, Y, 64, None) == 1     # X too big to stage
+    assert f(Q, Z, SC, None, 64, 128, 128, X, 0, 128, Y, 64, None) == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("M,K,N", [(1, 3072, 18432), (4, 3072, 18432), (3, 128, 1),
+                                   (8, 1536, 1000), (2, 12288, 3072)])
+def test_awq_linear_parity(M, K, N):
+    """The GPU layer against the oracle's float64 layer (same packed codes):
+    rel-Fro <= 2e-3 and per element 1e-2 rms + half a bf16 ulp."""
+    import torch
+    from gpu_common import check_output, from_dev_bf16, to_dev_bf16
+    rng = np.random.default_rng(M * 7 + K + N)
+    X = SI.f32_to_bf16_bits((rng.standard_normal((M, K))).astype(np.float32))
+    W = (rng.standard_normal((N, K)) * 0.02).astype(np.float32)
+    b = SI.f32_to_bf16_bits((rng.standard_normal(N) * 0.01).astype(np.float32))
+    aw = S.svdq_awq_pack(W, 128, bias_bf16=b).to_device("cuda")
+    Y = S.svdq_awq_linear(aw, to_dev_bf16(X))
+    torch.cuda.synchronize()
+    q, z, sb = A.awq_quantize(W, 128)
+    Y_ref = A.awq_linear_reference(X, q, z, sb, b)
+    check_output(from_dev_bf16(Y), Y_ref)
+    assert S.svdq_device_error() == 0

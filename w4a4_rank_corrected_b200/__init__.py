@@ -29,7 +29,8 @@ __all__ = [
     "new_workspace", "svdq_gemm_gelu",
     "svdq_mlp_forward", "svdq_mlp_workspace_bytes", "new_mlp_workspace", "svdq_debug_gelu",
     "svdq_act_row_scales", "svdq_quantize_act_dynamic", "svdq_gemm_dynamic",
-    "svdq_dyn_workspace_bytes", "svdq_linear_forward_dynamic",
+    "svdq_dyn_workspace_bytes", "svdq_linear_forward_dynamic", "svdq_awq_pack",
+    "svdq_awq_linear", "AwqWeight",
     "svdq_device_error", "svdq_selftest_timeout", "svdq_debug_convert", "svdq_sf_tile_offset",
     "svdq_status_string", "SVDQW4A4Linear", "lib", "STATUS",
 ]
@@ -99,6 +100,8 @@ def _load() -> ctypes.CDLL:
         "svdq_selftest_timeout": (I, [I, P]),
         "svdq_debug_convert": (I, [P, P, P, I64, P]),
         "svdq_debug_gelu": (I, [P, P, I64, P]),
+        "svdq_awq_pack": (I, [P, I, I, I, P, P, P]),
+        "svdq_awq_linear": (I, [P, P, P, P, I, I, I, P, I, I64, P, I64, P]),
         "svdq_act_row_scales": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P]),
         "svdq_quantize_act_dynamic": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P, P, P, P]),
         "svdq_gemm_dynamic": (I, [ctypes.POINTER(SvdqWeight), P, P, P, P, I, P, I64, P]),
@@ -491,6 +494,60 @@ def svdq_linear_forward_dynamic(w: DeviceWeight, X, Y=None, workspace=None, stre
                                            Y.data_ptr(), Y.stride(0), workspace.data_ptr(),
                                            workspace.numel(), _stream_ptr(stream)),
            "svdq_linear_forward_dynamic")
+    _keep_alive_on(stream, *made)
+    return Y
+
+
+# --------------------------------------------------------- AWQ W4A16 ----
+
+@dataclass
+class AwqWeight:
+    """A packed AWQ W4A16 weight (host numpy arrays) and, after to_device,
+    its device copies."""
+    N: int
+    K: int
+    group: int
+    q: np.ndarray          # u8 [N, K/2], even k in the low nibble
+    zeros: np.ndarray      # u8 [N, K/group]
+    scales: np.ndarray     # fp16 bits [N, K/group]
+    bias: Optional[np.ndarray] = None
+    dev: Optional[dict] = None
+
+    def to_device(self, device="cuda") -> "AwqWeight":
+        import torch
+        up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+        self.dev = {"q": up(self.q), "zeros": up(self.zeros),
+                    "scales": up(self.scales.view(np.int16)),
+                    "bias": None if self.bias is None else up(np.asarray(self.bias, np.uint16).view(np.int16))}
+        return self
+
+
+def svdq_awq_pack(W: np.ndarray, group: int = 128, bias_bf16=None) -> AwqWeight:
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    q = np.empty((N, K // 2), np.uint8)
+    z = np.empty((N, K // group), np.uint8)
+    sc = np.empty((N, K // group), np.uint16)
+    _check(lib.svdq_awq_pack(W.ctypes.data, N, K, group, q.ctypes.data, z.ctypes.data,
+                             sc.ctypes.data), "svdq_awq_pack")
+    return AwqWeight(N, K, group, q, z, sc, None if bias_bf16 is None else np.asarray(bias_bf16, np.uint16))
+
+
+def svdq_awq_linear(w: AwqWeight, X, Y=None, stream=None):
+    """Y = X dequant(W)^T + bias (bf16), 1 <= M <= 8."""
+    import torch
+    if w.dev is None:
+        raise ValueError("AwqWeight.to_device() first")
+    _check_x(X, w.K)
+    M = X.shape[0]
+    made = []
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
+        made.append(Y)
+    d = w.dev
+    _check(lib.svdq_awq_linear(d["q"].data_ptr(), d["zeros"].data_ptr(), d["scales"].data_ptr(),
+                               _ptr(d["bias"]), w.N, w.K, w.group, X.data_ptr(), M, X.stride(0),
+                               Y.data_ptr(), Y.stride(0), _stream_ptr(stream)), "svdq_awq_linear")
     _keep_alive_on(stream, *made)
     return Y
 

@@ -20,7 +20,8 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libsvdq.so")
 SOURCES = [os.path.join(HERE, "csrc", "svdq_api.cu"), os.path.join(HERE, "csrc", "pack.cpp")]
 DEPS = SOURCES + [os.path.join(HERE, "csrc", f) for f in
-                  ("ptx.cuh", "quantize_act.cuh", "w4a4_gemm.cuh")] + \
+                  ("ptx.cuh", "quantize_act.cuh", "quantize_act64.cuh", "w4a4_gemm.cuh",
+                   "gelu.cuh", "row_scales.cuh", "awq_gemv.cuh")] + \
        [os.path.join(ROOT, "include", "svdq.h")]
 
 

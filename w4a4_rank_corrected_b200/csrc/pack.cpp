@@ -476,3 +476,66 @@ extern "C" svdq_status svdq_pack_weight(const float* W, const float* x_absmax,
   }
   return SVDQ_OK;
 }
+
+// ----------------------------------------------------------------- AWQ ----
+// binary16 (1 sign, 5 exponent bits with bias 15, 10 fraction bits;
+// subnormals k * 2^-24) nearest to a double, ties to even.
+static uint16_t half_from_double(double x) {
+  const uint16_t sign = std::signbit(x) ? 0x8000 : 0;
+  const double a = std::fabs(x);
+  if (a == 0.0) return sign;
+  if (!(a < 65520.0)) return (uint16_t)(sign | 0x7C00);   // rounds past 65504
+  if (a < std::ldexp(1.0, -14)) {
+    const double k = std::rint(std::ldexp(a, 24));          // 0 .. 1024 (1024: smallest normal)
+    return (uint16_t)(sign | (uint16_t)k);
+  }
+  int e = 0;
+  const double m = std::frexp(a, &e);                      // a = m 2^e, m in [0.5, 1)
+  double r = std::rint(std::ldexp(m, 11));                 // 1024 .. 2048
+  int ex = e - 1;
+  if (r == 2048.0) {
+    r = 1024.0;
+    ex += 1;
+  }
+  if (ex > 15) return (uint16_t)(sign | 0x7C00);
+  return (uint16_t)(sign | ((ex + 15) << 10) | ((int)r - 1024));
+}
+
+static double half_to_double(uint16_t h) {
+  const int e = (h >> 10) & 31, f = h & 1023;
+  const double v = e == 0 ? std::ldexp((double)f, -24) : std::ldexp(1.0 + f / 1024.0, e - 15);
+  return (h & 0x8000) ? -v : v;
+}
+
+extern "C" svdq_status svdq_awq_pack(const float* W, int N, int K, int group, uint8_t* q_packed,
+                                     uint8_t* zeros, uint16_t* scales) {
+  if (!W || !q_packed || !zeros || !scales || N <= 0 || K <= 0 || group <= 0 || group % 32 ||
+      K % group)
+    return SVDQ_ERR_INVALID_ARG;
+  for (size_t i = 0; i < (size_t)N * K; ++i)
+    if (!std::isfinite(W[i])) return SVDQ_ERR_NUMERIC;
+  const int G = K / group;
+#pragma omp parallel for schedule(static)
+  for (int n = 0; n < N; ++n) {
+    for (int gi = 0; gi < G; ++gi) {
+      const float* w = W + (size_t)n * K + (size_t)gi * group;
+      double wmin = 0.0, wmax = 0.0;   // the range includes 0
+      for (int j = 0; j < group; ++j) {
+        wmin = std::min(wmin, (double)w[j]);
+        wmax = std::max(wmax, (double)w[j]);
+      }
+      const uint16_t hb = half_from_double(std::max(wmax - wmin, 1e-5) / 15.0);
+      const double scale = half_to_double(hb);
+      const double z = std::min(15.0, std::max(0.0, std::rint(-wmin / scale)));
+      scales[(size_t)n * G + gi] = hb;
+      zeros[(size_t)n * G + gi] = (uint8_t)z;
+      for (int j = 0; j < group; j += 2) {
+        const double q0 = std::min(15.0, std::max(0.0, std::rint((double)w[j] / scale) + z));
+        const double q1 = std::min(15.0, std::max(0.0, std::rint((double)w[j + 1] / scale) + z));
+        q_packed[(size_t)n * (K / 2) + ((size_t)gi * group + j) / 2] =
+            (uint8_t)((int)q0 | ((int)q1 << 4));
+      }
+    }
+  }
+  return SVDQ_OK;
+}

@@ -15,6 +15,7 @@
 #include "quantize_act.cuh"
 #include "quantize_act64.cuh"
 #include "row_scales.cuh"
+#include "awq_gemv.cuh"
 #include "w4a4_gemm.cuh"
 
 namespace svdq_dev {
@@ -667,6 +668,56 @@ extern "C" svdq_status svdq_linear_forward_dynamic(const svdq_weight* w, const u
   if ((st = launch_row_scales(w, X, M, ldx, rs, s, sms)) != SVDQ_OK) return st;
   if ((st = launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, s, sms, rs)) != SVDQ_OK) return st;
   return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, s, sms, false, rs);
+}
+
+template <int MT>
+svdq_status launch_awq(const uint8_t* q, const uint8_t* zeros, const uint16_t* scales,
+                       const uint16_t* bias, int N, int K, int group, const uint16_t* X,
+                       int64_t ldx, uint16_t* Y, int64_t ldy, cudaStream_t s, int sms) {
+  const size_t smem = (size_t)MT * K * 4;
+  if (cudaFuncSetAttribute(awq_gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess) {
+    cudaGetLastError();
+    return SVDQ_ERR_CUDA;
+  }
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, awq_gemv_kernel<MT>, AWQ_THREADS,
+                                                    smem) != cudaSuccess ||
+      per_sm <= 0) {
+    cudaGetLastError();
+    per_sm = 1;
+  }
+  const int warps = AWQ_THREADS / 32;
+  const int blocks = std::max(1, std::min((N + warps - 1) / warps, per_sm * sms));
+  awq_gemv_kernel<MT><<<blocks, AWQ_THREADS, smem, s>>>(q, zeros, scales, bias, N, K, group, X,
+                                                        ldx, Y, ldy);
+  return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+extern "C" svdq_status svdq_awq_linear(const uint8_t* q, const uint8_t* zeros,
+                                       const uint16_t* scales, const uint16_t* bias, int N, int K,
+                                       int group, const uint16_t* X, int M, int64_t ldx,
+                                       uint16_t* Y, int64_t ldy, void* stream) {
+  if (N <= 0 || K <= 0 || group <= 0 || group % 32 || K % group) return SVDQ_ERR_INVALID_ARG;
+  if (M < 0 || M > AWQ_MAX_M || ldx < K || ldy < N) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!q || !zeros || !scales || !X || !Y) return SVDQ_ERR_INVALID_ARG;
+  if ((size_t)M * K * 4 > 200u * 1024u) return SVDQ_ERR_INVALID_ARG;   // X staged in smem
+  if (!aligned16(q)) return SVDQ_ERR_MISALIGNED;
+  int sms = 0;
+  svdq_status st = device_check(&sms);
+  if (st != SVDQ_OK) return st;
+  cudaStream_t s = (cudaStream_t)stream;
+  switch (M) {
+    case 1: return launch_awq<1>(q, zeros, scales, bias, N, K, group, X, ldx, Y, ldy, s, sms);
+    case 2: return launch_awq<2>(q, zeros, scales, bias, N, K, group, X, ldx, Y, ldy, s, sms);
+    case 3: return launch_awq<3>(q, zeros, scales, bias, N, K, group, X, ldx, Y, ldy, s, sms);
+    case 4: return launch_awq<4>(q, zeros, scales, bias, N, K, group, X, ldx, Y, ldy, s, sms);
+    case 5: return launch_awq<5>(q, zeros, scales, bias, N, K, group, X, ldx, Y, ldy, s, sms);
+    case 6: return launch_awq<6>(q, zeros, scales, bias, N, K, group, X, ldx, Y, ldy, s, sms);
+    case 7: return launch_awq<7>(q, zeros, scales, bias, N, K, group, X, ldx, Y, ldy, s, sms);
+    default: return launch_awq<8>(q, zeros, scales, bias, N, K, group, X, ldx, Y, ldy, s, sms);
+  }
 }
 
 extern "C" svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t* X, int M,
