@@ -521,9 +521,12 @@ def test_dynamic_scale_parity(name):
 
 
 def test_dynamic_scale_beyond_calibration():
-    """Inputs 16x beyond the calibration range: the static scale saturates
-    (E4M3 at 448, E2M1 at 6) and loses the layer; per-token scales keep it
-    within tolerance.  Large M takes the 128-row kernel."""
+    """Inputs 16x beyond the calibration range.  Per-token scales are
+    invariant to a power-of-two scaling of X: the codes and scales of 16 X
+    equal those of X bit for bit, and the output error against the exact
+    X W^T + b stays at the in-range 4-bit floor.  The static scale
+    saturates (E4M3 at 448, E2M1 at 6): its error at 16x is at least twice
+    the in-range one.  Large M takes the 128-row kernel."""
     S = _S()
     for M in (512, 16384):
         K, N, r = 3072, 512, 32
@@ -532,10 +535,17 @@ def test_dynamic_scale_beyond_calibration():
         Xb = SI.f32_to_bf16_bits(SI.bf16_bits_to_f32(Xc) * np.float32(16.0))
         rows = rows_every_block(M, extra=8, seed=M)
         Yd = _check_dynamic(S, dw, op, Xb, b, rows=rows)
-        Ys = from_dev_bf16(S.svdq_linear_forward(dw, to_dev_bf16(Xb)))
-        exact = (SI.bf16_bits_to_f32(Xb).astype(np.float64)[rows] @ W.astype(np.float64).T
-                 + F.bf16_bits_to_f64(b)[None, :])
-        err_d = np.linalg.norm(F.bf16_bits_to_f64(Yd[rows]) - exact) / np.linalg.norm(exact)
-        err_s = np.linalg.norm(F.bf16_bits_to_f64(Ys[rows]) - exact) / np.linalg.norm(exact)
-        assert err_d < 0.2 * err_s, (err_d, err_s)
+        c1, s1, _ = S.svdq_quantize_act_dynamic(dw, to_dev_bf16(Xc), S.svdq_act_row_scales(dw, to_dev_bf16(Xc)))
+        c16, s16, _ = S.svdq_quantize_act_dynamic(dw, to_dev_bf16(Xb), S.svdq_act_row_scales(dw, to_dev_bf16(Xb)))
+        assert torch.equal(c1, c16) and torch.equal(s1, s16)
+        Ys1 = from_dev_bf16(S.svdq_linear_forward(dw, to_dev_bf16(Xc)))
+        Ys16 = from_dev_bf16(S.svdq_linear_forward(dw, to_dev_bf16(Xb)))
+        w64 = W.astype(np.float64).T
+        bias = F.bf16_bits_to_f64(b)[None, :]
+        ex1 = SI.bf16_bits_to_f32(Xc).astype(np.float64)[rows] @ w64 + bias
+        ex16 = SI.bf16_bits_to_f32(Xb).astype(np.float64)[rows] @ w64 + bias
+        rel = lambda Y, ex: np.linalg.norm(F.bf16_bits_to_f64(Y[rows]) - ex) / np.linalg.norm(ex)
+        e_s1, e_s16, e_d16 = rel(Ys1, ex1), rel(Ys16, ex16), rel(Yd, ex16)
+        assert e_d16 <= 1.1 * e_s1, (e_d16, e_s1)
+        assert e_s16 >= 2.0 * e_s1, (e_s16, e_s1)
     assert S.svdq_device_error() == 0
