@@ -374,8 +374,8 @@ svdq_status svdq_awq_pack(const float* W, int N, int K, int group, uint8_t* q_pa
 
 /* svdq_awq_linear (GPU): Y = X dequant(W)^T + bias, fp32 accumulation, one
  * bf16 rounding.  For the batch sizes of modulation layers: 1 <= M <= 8 (a
- * memory-bound matrix-vector product over the weight stream) and M * K * 4
- * <= 200 KB.
+ * memory-bound matrix-vector product over the weight stream) and
+ * M * K * 4.5 <= 200 KB (X is staged in shared memory).
  *   q, zeros, scales  device, as svdq_awq_pack writes them (q 16-byte aligned)
  *   bias   device bf16 [N] or NULL
  *   X      device bf16 [M][ldx], ldx >= K;  Y device bf16 [M][ldy], ldy >= N

@@ -48,7 +48,7 @@ def test_awq_argument_validation():
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("M,K,N", [(1, 3072, 18432), (4, 3072, 18432), (3, 128, 1),
+@pytest.mark.parametrize("M,K,N", [(1, 3072, 18432), (4, 3072, 18432), (3, 128, 64),
                                    (8, 1536, 1000), (2, 12288, 3072)])
 def test_awq_linear_parity(M, K, N):
     """The GPU layer against the oracle's float64 layer (same packed codes):

@@ -11,8 +11,12 @@
 // CUDA cores: one warp per output row at a time, each lane streaming 16
 // bytes (32 codes) of the row per step, dequantizing in registers (exact in
 // fp32: a small integer times an fp16 scale) and accumulating the M dot
-// products in fp32; X is staged once per CTA in shared memory as fp32; the
-// lanes' partial sums meet in a warp reduction.  A persistent grid (a few
+// products in fp32; X is staged once per CTA in shared memory as fp32, each
+// 32-value chunk padded to 36 floats (lane l reads chunk l: with a 144-byte
+// chunk stride the 32 lanes' 16-byte reads fall on distinct bank groups,
+// where the unpadded 128-byte stride put all of them on the same banks and
+// cost 8x in shared-memory wavefronts); the lanes' partial sums meet in a
+// warp reduction.  A persistent grid (a few
 // CTAs per SM) keeps enough loads in flight to cover the memory latency.
 #pragma once
 #include <cuda_fp16.h>
@@ -22,6 +26,7 @@ namespace svdq_dev {
 
 constexpr int AWQ_THREADS = 256;
 constexpr int AWQ_MAX_M = 8;
+constexpr int AWQ_CHUNK_PAD = 36;   // floats per staged 32-value chunk of X
 
 template <int MT>
 __global__ void __launch_bounds__(AWQ_THREADS)
@@ -29,10 +34,11 @@ __global__ void __launch_bounds__(AWQ_THREADS)
                     const uint16_t* __restrict__ scales, const uint16_t* __restrict__ bias, int N,
                     int K, int group, const uint16_t* __restrict__ X, int64_t ldx,
                     uint16_t* __restrict__ Y, int64_t ldy) {
-  extern __shared__ float xs[];   // [MT][K] fp32
+  extern __shared__ float xs[];   // [MT][K / 32][36] fp32 (chunks padded)
+  const int KP = (K >> 5) * AWQ_CHUNK_PAD;
   for (int i = threadIdx.x; i < MT * K; i += blockDim.x) {
     const int m = i / K, k = i - m * K;
-    xs[i] = bf16_lo_f32(X[(size_t)m * ldx + k]);
+    xs[m * KP + (k >> 5) * AWQ_CHUNK_PAD + (k & 31)] = bf16_lo_f32(X[(size_t)m * ldx + k]);
   }
   __syncthreads();
   const int lane = threadIdx.x & 31;
@@ -59,18 +65,24 @@ __global__ void __launch_bounds__(AWQ_THREADS)
         if (c >= chunks) break;
         const int gi = c / cpg;
         const float sc = __half2float(__ushort_as_half(scales[(size_t)n * G + gi]));
-        const float zf = (float)zeros[(size_t)n * G + gi];
+        const float nzs = -(float)zeros[(size_t)n * G + gi] * sc;   // exact: z * fp16
         const uint32_t words[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
         float v[32];
 #pragma unroll
         for (int t = 0; t < 4; ++t)
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            v[8 * t + j] = ((float)((words[t] >> (4 * j)) & 15u) - zf) * sc;
-        const int k0 = c * 32;
+          for (int j = 0; j < 8; ++j) {
+            // the code as a float without a conversion instruction: the bits
+            // of 2^23 + q, minus 2^23 (exact); then (q - z) scale = q scale -
+            // z scale, exact in one fused operation (every term is a small
+            // integer times the fp16 scale)
+            const float qf =
+                __uint_as_float(0x4B000000u | ((words[t] >> (4 * j)) & 15u)) - 8388608.0f;
+            v[8 * t + j] = fmaf(qf, sc, nzs);
+          }
 #pragma unroll
         for (int m = 0; m < MT; ++m) {
-          const float4* x4 = reinterpret_cast<const float4*>(xs + m * K + k0);
+          const float4* x4 = reinterpret_cast<const float4*>(xs + m * KP + c * AWQ_CHUNK_PAD);
           float a = acc[m];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {

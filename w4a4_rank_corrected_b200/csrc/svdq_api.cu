@@ -674,7 +674,7 @@ template <int MT>
 svdq_status launch_awq(const uint8_t* q, const uint8_t* zeros, const uint16_t* scales,
                        const uint16_t* bias, int N, int K, int group, const uint16_t* X,
                        int64_t ldx, uint16_t* Y, int64_t ldy, cudaStream_t s, int sms) {
-  const size_t smem = (size_t)MT * K * 4;
+  const size_t smem = (size_t)MT * (K / 32) * AWQ_CHUNK_PAD * 4;
   if (cudaFuncSetAttribute(awq_gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess) {
     cudaGetLastError();
@@ -702,7 +702,8 @@ extern "C" svdq_status svdq_awq_linear(const uint8_t* q, const uint8_t* zeros,
   if (M < 0 || M > AWQ_MAX_M || ldx < K || ldy < N) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   if (!q || !zeros || !scales || !X || !Y) return SVDQ_ERR_INVALID_ARG;
-  if ((size_t)M * K * 4 > 200u * 1024u) return SVDQ_ERR_INVALID_ARG;   // X staged in smem
+  if ((size_t)M * (K / 32) * AWQ_CHUNK_PAD * 4 > 200u * 1024u)
+    return SVDQ_ERR_INVALID_ARG;   // X staged in smem
   if (!aligned16(q)) return SVDQ_ERR_MISALIGNED;
   int sms = 0;
   svdq_status st = device_check(&sms);
