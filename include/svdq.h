@@ -372,13 +372,29 @@ svdq_status svdq_linear_forward_static(const svdq_weight* w, const uint16_t* X,
 svdq_status svdq_awq_pack(const float* W, int N, int K, int group, uint8_t* q_packed,
                           uint8_t* zeros, uint16_t* scales);
 
-/* svdq_awq_linear (GPU): Y = X dequant(W)^T + bias, fp32 accumulation, one
- * bf16 rounding.  For the batch sizes of modulation layers: 1 <= M <= 8 (a
- * memory-bound matrix-vector product over the weight stream) and
- * M * K * 4.5 <= 200 KB (X is staged in shared memory).
- *   q, zeros, scales  device, as svdq_awq_pack writes them (q 16-byte aligned)
+/* svdq_awq_tile_codes (host, synchronous): the codes in the layout the
+ * GPU layer reads.  q_rowmajor as svdq_awq_pack writes it ([N][K/2], even k
+ * in the low nibble); q_tiled: ceil(N/16) * 16 * K / 2 bytes.  Per 16-row
+ * block rb and 64-deep block of K, 512 bytes = 32 lanes x 16 bytes; lane
+ * l = 4 g + c holds one 32-bit word per 16-deep k-step ks (4 per block, at
+ * byte ((rb * K/64 + ks/4) * 32 + l) * 16 + (ks % 4) * 4), and nibble j of
+ * that word is the code of row 16 rb + g + 8 (j % 2), column
+ * 16 ks + 2 c + 8 ((j % 4) / 2) + j / 4 (the elements a warp's tensor-core
+ * fragment takes from lane l); rows past N hold code 0.  K % 64 == 0.
+ * Errors: INVALID_ARG. */
+svdq_status svdq_awq_tile_codes(const uint8_t* q_rowmajor, int N, int K, uint8_t* q_tiled);
+
+/* svdq_awq_linear (GPU): Y = X dequant(W)^T + bias, one bf16 rounding.  Per
+ * group the sum of (q - z) x is accumulated in fp32 (products exact), then
+ * scaled by the group's fp16 scale and added in fp32.  For the batch sizes
+ * of modulation layers: 1 <= M <= 8 (a memory-bound product over the weight
+ * stream), group a multiple of 64 dividing K, and 8 KB + M * K * 2 bytes
+ * <= 216 KB (X is staged in shared memory).
+ *   q      device, tiled as svdq_awq_tile_codes writes it (16-byte aligned)
+ *   zeros, scales  device, as svdq_awq_pack writes them ([N][K/group])
  *   bias   device bf16 [N] or NULL
- *   X      device bf16 [M][ldx], ldx >= K;  Y device bf16 [M][ldy], ldy >= N
+ *   X      device bf16 [M][ldx], 16-byte aligned, ldx >= K, ldx % 8 == 0
+ *   Y      device bf16 [M][ldy], ldy >= N
  * Errors: INVALID_ARG (shapes, M > 8, NULLs), MISALIGNED, UNSUPPORTED_ARCH. */
 svdq_status svdq_awq_linear(const uint8_t* q, const uint8_t* zeros, const uint16_t* scales,
                             const uint16_t* bias, int N, int K, int group, const uint16_t* X,

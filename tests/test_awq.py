@@ -27,6 +27,35 @@ def test_awq_pack_matches_oracle(N, K, group, seed):
     assert np.array_equal(aw.q, A.pack_nibbles_awq(q))
 
 
+@pytest.mark.parametrize("N,K,seed", [(16, 64, 0), (40, 256, 1), (1000, 1536, 2)])
+def test_awq_tile_codes_layout(N, K, seed):
+    """The tiled code layout read back the way a warp's m16n8k16 A fragment
+    takes it: lane l = 4 g + c, register r holds (row g + 8 (r % 2),
+    columns 2 c + 8 (r // 2) + {0, 1}) of each 16 x 16 tile; in the word,
+    register r's low half is nibble r and its high half nibble r + 4."""
+    rng = np.random.default_rng(seed)
+    q = rng.integers(0, 16, (N, K), dtype=np.uint8)
+    tiled = S.svdq_awq_tile_codes(A.pack_nibbles_awq(q), N, K)
+    N16 = (N + 15) // 16 * 16
+    assert tiled.shape == (N16 * K // 2,)
+    words = tiled.view(np.uint32)
+    back = np.full((N16, K), 255, np.int32)
+    for rb in range(N16 // 16):
+        for ks in range(K // 16):
+            for lane in range(32):
+                g, c = divmod(lane, 4)
+                w = int(words[((rb * (K // 64) + ks // 4) * 32 + lane) * 4 + ks % 4])
+                for r in range(4):
+                    for half in range(2):
+                        nib = (w >> (4 * (r + 4 * half))) & 15
+                        row = 16 * rb + g + 8 * (r % 2)
+                        col = 16 * ks + 2 * c + 8 * (r // 2) + half
+                        assert back[row, col] == 255
+                        back[row, col] = nib
+    assert np.array_equal(back[:N], q)
+    assert np.all(back[N:] == 0)
+
+
 def test_awq_argument_validation():
     L = S.lib
     W = np.zeros((4, 128), np.float32)
@@ -41,9 +70,10 @@ def test_awq_argument_validation():
     f = L.svdq_awq_linear
     assert f(Q, Z, SC, None, 64, 128, 128, X, 9, 128, Y, 64, None) == 1        # M > 8
     assert f(Q, Z, SC, None, 64, 128, 100, X, 1, 128, Y, 64, None) == 1       # group
+    assert f(Q, Z, SC, None, 64, 128, 32, X, 1, 128, Y, 64, None) == 1        # group % 64
     assert f(Q, Z, SC, None, 64, 128, 128, X, 1, 100, Y, 64, None) == 1       # ldx < K
     assert f(Q + 8, Z, SC, None, 64, 128, 128, X, 1, 128, Y, 64, None) == 3   # alignment
-    assert f(Q, Z, SC, None, 64, 8192, 128, X, 8, 8192, Y, 64, None) == 1     # X too big to stage
+    assert f(Q, Z, SC, None, 64, 16384, 128, X, 8, 16384, Y, 64, None) == 1   # X too big to stage
     assert f(Q, Z, SC, None, 64, 128, 128, X, 0, 128, Y, 64, None) == 0
 
 

@@ -30,7 +30,7 @@ __all__ = [
     "svdq_mlp_forward", "svdq_mlp_workspace_bytes", "new_mlp_workspace", "svdq_debug_gelu",
     "svdq_act_row_scales", "svdq_quantize_act_dynamic", "svdq_gemm_dynamic",
     "svdq_dyn_workspace_bytes", "svdq_linear_forward_dynamic", "svdq_awq_pack",
-    "svdq_awq_linear", "AwqWeight",
+    "svdq_awq_linear", "svdq_awq_tile_codes", "AwqWeight",
     "svdq_device_error", "svdq_selftest_timeout", "svdq_debug_convert", "svdq_sf_tile_offset",
     "svdq_status_string", "SVDQW4A4Linear", "lib", "STATUS",
 ]
@@ -101,6 +101,7 @@ def _load() -> ctypes.CDLL:
         "svdq_debug_convert": (I, [P, P, P, I64, P]),
         "svdq_debug_gelu": (I, [P, P, I64, P]),
         "svdq_awq_pack": (I, [P, I, I, I, P, P, P]),
+        "svdq_awq_tile_codes": (I, [P, I, I, P]),
         "svdq_awq_linear": (I, [P, P, P, P, I, I, I, P, I, I64, P, I64, P]),
         "svdq_act_row_scales": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P]),
         "svdq_quantize_act_dynamic": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P, P, P, P]),
@@ -514,9 +515,10 @@ class AwqWeight:
     dev: Optional[dict] = None
 
     def to_device(self, device="cuda") -> "AwqWeight":
+        """Device copies; the codes go up in the GPU layer's tiled layout."""
         import torch
         up = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
-        self.dev = {"q": up(self.q), "zeros": up(self.zeros),
+        self.dev = {"q": up(svdq_awq_tile_codes(self.q, self.N, self.K)), "zeros": up(self.zeros),
                     "scales": up(self.scales.view(np.int16)),
                     "bias": None if self.bias is None else up(np.asarray(self.bias, np.uint16).view(np.int16))}
         return self
@@ -531,6 +533,17 @@ def svdq_awq_pack(W: np.ndarray, group: int = 128, bias_bf16=None) -> AwqWeight:
     _check(lib.svdq_awq_pack(W.ctypes.data, N, K, group, q.ctypes.data, z.ctypes.data,
                              sc.ctypes.data), "svdq_awq_pack")
     return AwqWeight(N, K, group, q, z, sc, None if bias_bf16 is None else np.asarray(bias_bf16, np.uint16))
+
+
+def svdq_awq_tile_codes(q_rowmajor: np.ndarray, N: int, K: int) -> np.ndarray:
+    """[N, K/2] codes -> the GPU layer's tiled layout (ceil(N/16)*16*K/2 bytes)."""
+    q_rowmajor = np.ascontiguousarray(q_rowmajor, dtype=np.uint8)
+    if q_rowmajor.shape != (N, K // 2):
+        raise ValueError("codes must have shape [N, K/2]")
+    out = np.empty(((N + 15) // 16 * 16 * K // 2,), np.uint8)
+    _check(lib.svdq_awq_tile_codes(q_rowmajor.ctypes.data, N, K, out.ctypes.data),
+           "svdq_awq_tile_codes")
+    return out
 
 
 def svdq_awq_linear(w: AwqWeight, X, Y=None, stream=None):

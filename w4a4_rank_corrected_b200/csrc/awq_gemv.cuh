@@ -6,18 +6,37 @@
 //
 // Y = X W^T + bias with W stored as asymmetric INT4 per group of `group`
 // input channels: w = (q - z) * scale, q and z integers 0..15, scale fp16.
-// At the batch sizes of those layers (a few conditioning vectors) the layer
-// is a matrix-vector product bound by the weight stream, so it runs on the
-// CUDA cores: one warp per output row at a time, each lane streaming 16
-// bytes (32 codes) of the row per step, dequantizing in registers (exact in
-// fp32: a small integer times an fp16 scale) and accumulating the M dot
-// products in fp32; X is staged once per CTA in shared memory as fp32, each
-// 32-value chunk padded to 36 floats (lane l reads chunk l: with a 144-byte
-// chunk stride the 32 lanes' 16-byte reads fall on distinct bank groups,
-// where the unpadded 128-byte stride put all of them on the same banks and
-// cost 8x in shared-memory wavefronts); the lanes' partial sums meet in a
-// warp reduction.  A persistent grid (a few
-// CTAs per SM) keeps enough loads in flight to cover the memory latency.
+// At the batch sizes of those layers (M <= 8 conditioning vectors) the
+// layer is bound by the weight stream: about 22 bytes, 45 weights, per SM
+// clock at the HBM rate.  A CUDA-core dot product spends an FMA per weight
+// and batch row plus the code's conversion -- more issue slots than an SM
+// has at that rate.  So the contraction runs on the tensor core with
+// register operands (mma.sync m16n8k16, bf16 in, fp32 accumulate): a warp's
+// 16 x 16 weight tile is dequantized in registers and meets the batch
+// (padded to 8 columns) in one instruction.  The dequantized weights never
+// touch shared or tensor memory (the weight stream's rate would saturate
+// either), which is why this is not a tcgen05 kernel.
+//
+//   * codes arrive pre-tiled (svdq_awq_tile_codes): per 16-row block and
+//     four 16-deep k-steps, 512 bytes in which lane l's 16 bytes are its
+//     four 32-bit words, one per k-step; the eight codes of a word are that
+//     lane's eight A-fragment elements, nibbles j and j + 4 forming register
+//     j of the fragment (low and high half);
+//   * a pair of codes becomes the bf16 pair (128 + q, 128 + q') with one
+//     shift and one bitwise op (the nibble lands in the low mantissa bits
+//     of 128.0), then q - z exactly with one bf16x2 subtraction of
+//     (128 + z, 128 + z);
+//   * per group the MMA accumulator holds sum_k (q_k - z) x_k (products
+//     exact, fp32 accumulation); it is scaled by the group's fp16 scale and
+//     added to the running sum (one FMA per output);
+//   * X is staged once per CTA in shared memory (16-byte loads), per k-step
+//     and batch row 16 values in B-fragment order (lane c's four values
+//     adjacent: one 8-byte load);
+//   * a CTA's eight warps cover 8 / S row blocks, S warps splitting K per
+//     block (S chosen by the host so the grid has enough warps); their
+//     partial sums meet in shared memory, bias is added and Y is rounded
+//     once to bf16.  Each warp keeps eight 512-byte code blocks (with their
+//     scales and zeros) in flight ahead of the one it computes.
 #pragma once
 #include <cuda_fp16.h>
 #include "ptx.cuh"
@@ -25,91 +44,234 @@
 namespace svdq_dev {
 
 constexpr int AWQ_THREADS = 256;
+constexpr int AWQ_WARPS = AWQ_THREADS / 32;
 constexpr int AWQ_MAX_M = 8;
-constexpr int AWQ_CHUNK_PAD = 36;   // floats per staged 32-value chunk of X
+constexpr int AWQ_PF = 8;                                // code blocks in flight per warp
+constexpr uint32_t AWQ_SMEM_MAX = 216u * 1024u;
+constexpr int AWQ_RED_FLOATS = 2 * AWQ_WARPS * 32 * 4;   // two buffers of partial fragments
+
+// Shared memory of one CTA: the partial-sum buffers, then X (bf16 [K/16][M][16]).
+__host__ __device__ inline size_t awq_smem_bytes(int M, int K) {
+  return (size_t)AWQ_RED_FLOATS * 4 + (size_t)K * (size_t)M * 2;
+}
+
+// Byte offset of lane l's word for k-step ks of row block rb in the tiled codes.
+__host__ __device__ inline size_t awq_tile_word_offset(int rb, int ks, int lane, int K) {
+  return (((size_t)rb * (size_t)(K / 64) + (size_t)(ks >> 2)) * 32 + (size_t)lane) * 16 +
+         (size_t)(ks & 3) * 4;
+}
+
+// D += A * B, m16n8k16, bf16 inputs, fp32 accumulate.
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4],
+                                               uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t bf16x2_sub(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// The codes of nibbles j and j + 4 (the word shifted right by 4 j) as the
+// bf16 pair (128 + q_j, 128 + q_{j+4}).
+__device__ __forceinline__ uint32_t awq_pair128(uint32_t shifted) {
+  return (shifted & 0x000F000Fu) | 0x43004300u;
+}
+
+struct AwqSlot {   // one code block in flight: codes, and its group's scales and zeros
+  uint4 w;
+  uint32_t s;      // fp16 bits: row g (low half), row g + 8 (high half)
+  uint32_t z;      // zeros: row g (bits 0..7), row g + 8 (bits 16..23)
+};
 
 template <int MT>
-__global__ void __launch_bounds__(AWQ_THREADS)
+__global__ void __launch_bounds__(AWQ_THREADS, 2)
     awq_gemv_kernel(const uint8_t* __restrict__ q, const uint8_t* __restrict__ zeros,
                     const uint16_t* __restrict__ scales, const uint16_t* __restrict__ bias, int N,
-                    int K, int group, const uint16_t* __restrict__ X, int64_t ldx,
+                    int K, int group, int S, const uint16_t* __restrict__ X, int64_t ldx,
                     uint16_t* __restrict__ Y, int64_t ldy) {
-  extern __shared__ float xs[];   // [MT][K / 32][36] fp32 (chunks padded)
-  const int KP = (K >> 5) * AWQ_CHUNK_PAD;
-  for (int i = threadIdx.x; i < MT * K; i += blockDim.x) {
-    const int m = i / K, k = i - m * K;
-    xs[m * KP + (k >> 5) * AWQ_CHUNK_PAD + (k & 31)] = bf16_lo_f32(X[(size_t)m * ldx + k]);
-  }
-  __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const int warps = blockDim.x >> 5;
-  const int chunks = K >> 5;                 // 32 codes (16 bytes) per chunk
+  extern __shared__ __align__(16) uint8_t awq_smem[];
+  float* red = reinterpret_cast<float*>(awq_smem);                            // [2][8][32][4]
+  uint16_t* xs = reinterpret_cast<uint16_t*>(awq_smem + AWQ_RED_FLOATS * 4);  // [K/16][MT][16]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, c = lane & 3;
   const int G = K / group;
-  const int cpg = group >> 5;                // chunks per group
-  for (int n = blockIdx.x * warps + (threadIdx.x >> 5); n < N; n += gridDim.x * warps) {
-    const uint4* row = reinterpret_cast<const uint4*>(q + (size_t)n * (K / 2));
-    float acc[MT];
+  const int bpg = group >> 6;                 // 64-deep code blocks per group
+  const int R = AWQ_WARPS / S;                // row blocks per CTA per round
+  const int rb_total = (N + 15) >> 4;
+  const int rounds = (rb_total + R - 1) / R;
+  const int my_rounds =
+      (int)blockIdx.x < rounds ? (rounds - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+  const int sub = warp % S, rloc = warp / S;
+  const int gps = (G + S - 1) / S;            // groups per K slice
+  const int g0 = min(G, sub * gps), g1 = min(G, g0 + gps);
+  const int nblk = (g1 - g0) * bpg;           // this warp's code blocks per round
+  const int total = my_rounds * nblk;
+
+  // ---- fetch side of this warp's sequence of (round, block): pointers
+  // advanced per block (no per-block index arithmetic) ----
+  const int kb0 = g0 * bpg;                   // first 64-deep block of this warp's slice
+  int f_round = 0, f_blk = 0, f_ing = 0;      // round, block in the round, block in the group
+  bool f_ok = false, f_ok0 = false, f_ok1 = false;
+  const uint4* f_q = nullptr;
+  const uint16_t *f_s0 = scales, *f_s1 = scales;
+  const uint8_t *f_z0 = zeros, *f_z1 = zeros;
+  auto f_start_round = [&]() {
+    const int rb = ((int)blockIdx.x + f_round * (int)gridDim.x) * R + rloc;
+    const int n0 = rb * 16 + g;
+    f_ok = rb < rb_total;
+    f_ok0 = n0 < N;
+    f_ok1 = n0 + 8 < N;
+    f_q = reinterpret_cast<const uint4*>(q + awq_tile_word_offset(f_ok ? rb : 0, 4 * kb0, lane, K));
+    const size_t r0 = f_ok0 ? (size_t)n0 * G + g0 : 0, r1 = f_ok1 ? (size_t)(n0 + 8) * G + g0 : 0;
+    f_s0 = scales + r0;
+    f_s1 = scales + r1;
+    f_z0 = zeros + r0;
+    f_z1 = zeros + r1;
+    f_ing = 0;
+  };
+  auto fetch = [&](AwqSlot& sl) {
+    sl.w = f_ok ? __ldcs(f_q) : make_uint4(0, 0, 0, 0);
+    sl.s = (f_ok0 ? (uint32_t)__ldg(f_s0) : 0u) | ((f_ok1 ? (uint32_t)__ldg(f_s1) : 0u) << 16);
+    sl.z = (f_ok0 ? (uint32_t)__ldg(f_z0) : 0u) | ((f_ok1 ? (uint32_t)__ldg(f_z1) : 0u) << 16);
+    f_q += 32;                                // the next 512-byte block of this row block
+    if (++f_ing == bpg) {
+      f_ing = 0;
+      ++f_s0, ++f_s1, ++f_z0, ++f_z1;
+    }
+    if (++f_blk == nblk) {
+      f_blk = 0;
+      ++f_round;
+      f_start_round();
+    }
+  };
+  if (nblk > 0) f_start_round();
+  AwqSlot ring[AWQ_PF];
 #pragma unroll
-    for (int m = 0; m < MT; ++m) acc[m] = 0.0f;
-    for (int c0 = lane; c0 < chunks; c0 += 4 * 32) {
-      // up to four chunks per lane in flight before any arithmetic
-      uint4 w[4];
+  for (int j = 0; j < AWQ_PF; ++j)
+    if (j < total) fetch(ring[j]);            // in flight while X is staged
+
+  // ---- X into shared memory, each k-step's 16 values in B-fragment order:
+  // value j of a k-step goes to 4 ((j % 8) / 2) + 2 (j / 8) + j % 2, so each
+  // aligned pair stays a pair.  16-byte loads, four in flight per thread.
+  {
+    const int cpr = K >> 3;                   // 8-value chunks per row
+    uint32_t* xs32 = reinterpret_cast<uint32_t*>(xs);
+    for (int i0 = threadIdx.x; i0 < MT * cpr; i0 += 4 * AWQ_THREADS) {
+      uint4 v[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int c = c0 + 32 * u;
-        w[u] = c < chunks ? __ldcs(row + c) : make_uint4(0, 0, 0, 0);
+        const int i = i0 + u * AWQ_THREADS;
+        if (i < MT * cpr) {
+          const int m = i / cpr, ch = i - m * cpr;
+          v[u] = __ldg(reinterpret_cast<const uint4*>(X + (size_t)m * ldx) + ch);
+        }
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int c = c0 + 32 * u;
-        if (c >= chunks) break;
-        const int gi = c / cpg;
-        const float sc = __half2float(__ushort_as_half(scales[(size_t)n * G + gi]));
-        const float nzs = -(float)zeros[(size_t)n * G + gi] * sc;   // exact: z * fp16
-        const uint32_t words[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
-        float v[32];
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            // the code as a float without a conversion instruction: the bits
-            // of 2^23 + q, minus 2^23 (exact); then (q - z) scale = q scale -
-            // z scale, exact in one fused operation (every term is a small
-            // integer times the fp16 scale)
-            const float qf =
-                __uint_as_float(0x4B000000u | ((words[t] >> (4 * j)) & 15u)) - 8388608.0f;
-            v[8 * t + j] = fmaf(qf, sc, nzs);
-          }
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          const float4* x4 = reinterpret_cast<const float4*>(xs + m * KP + c * AWQ_CHUNK_PAD);
-          float a = acc[m];
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 xv = x4[j];
-            a = fmaf(xv.x, v[4 * j], a);
-            a = fmaf(xv.y, v[4 * j + 1], a);
-            a = fmaf(xv.z, v[4 * j + 2], a);
-            a = fmaf(xv.w, v[4 * j + 3], a);
-          }
-          acc[m] = a;
+        const int i = i0 + u * AWQ_THREADS;
+        if (i < MT * cpr) {
+          const int m = i / cpr, ch = i - m * cpr;
+          const int ks = ch >> 1, hi8 = ch & 1;   // the chunk is values 8 hi8 .. 8 hi8 + 7
+          uint32_t* dst = xs32 + ((size_t)ks * MT + m) * 8 + hi8;
+          dst[0] = v[u].x;
+          dst[2] = v[u].y;
+          dst[4] = v[u].z;
+          dst[6] = v[u].w;
         }
       }
     }
+  }
+  __syncthreads();
+
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  float cg[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  int c_round = 0, c_blk = 0, c_ing = 0;
+  // this lane's B fragment: batch row g, values 4c .. 4c+3 of each k-step's 16
+  const bool has_b = g < MT;
+  const uint2* xl0 = reinterpret_cast<const uint2*>(xs + (size_t)(has_b ? g : 0) * 16 + 4 * c) +
+                     (size_t)kb0 * 4 * MT * 4;
+  const uint2* xl = xl0;
+  // a warp without code blocks still takes one step per round (the CTA's
+  // barrier is passed by every warp once per round)
+  const int steps = nblk > 0 ? total : my_rounds;
+  for (int base = 0; base < steps; base += AWQ_PF) {
 #pragma unroll
-    for (int m = 0; m < MT; ++m) {
-      float a = acc[m];
+    for (int j = 0; j < AWQ_PF; ++j) {
+      const int item = base + j;
+      if (item < steps) {
+        bool round_end = true;
+        if (nblk > 0) {
+          const AwqSlot sl = ring[j];
+          if (item + AWQ_PF < total) fetch(ring[j]);
+          // (128 + z) in both halves, for each of this lane's two rows
+          const uint32_t zz0 = ((sl.z & 0xFFu) * 0x00010001u) | 0x43004300u;
+          const uint32_t zz1 = ((sl.z >> 16) * 0x00010001u) | 0x43004300u;
+          const uint32_t words[4] = {sl.w.x, sl.w.y, sl.w.z, sl.w.w};
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
-      acc[m] = a;
-    }
-    if (lane < MT) {
-      float a = acc[0];
-#pragma unroll
-      for (int m = 1; m < MT; ++m)
-        if (lane == m) a = acc[m];
-      if (bias) a += bf16_lo_f32(bias[n]);
-      Y[(size_t)lane * ldy + n] = (uint16_t)(__float_as_uint(__bfloat162float(__float2bfloat16_rn(a))) >> 16);
+          for (int t = 0; t < 4; ++t) {
+            const uint32_t wd = words[t];
+            uint32_t a[4];
+            a[0] = bf16x2_sub(awq_pair128(wd), zz0);         // row g,     k 2c, 2c+1
+            a[1] = bf16x2_sub(awq_pair128(wd >> 4), zz1);    // row g + 8, k 2c, 2c+1
+            a[2] = bf16x2_sub(awq_pair128(wd >> 8), zz0);    // row g,     k 2c+8, 2c+9
+            a[3] = bf16x2_sub(awq_pair128(wd >> 12), zz1);   // row g + 8, k 2c+8, 2c+9
+            uint32_t b0 = 0, b1 = 0;
+            if (has_b) {
+              const uint2 xv = xl[t * MT * 4];   // k-step t of the block: MT rows of 16 values
+              b0 = xv.x;
+              b1 = xv.y;
+            }
+            mma_bf16_16816(cg, a, b0, b1);
+          }
+          xl += 4 * MT * 4;
+          if (++c_ing == bpg) {
+            c_ing = 0;
+            // the group's sum of (q - z) x, times its scale
+            const float s0 = __half2float(__ushort_as_half((unsigned short)(sl.s & 0xFFFFu)));
+            const float s1 = __half2float(__ushort_as_half((unsigned short)(sl.s >> 16)));
+            acc[0] = fmaf(s0, cg[0], acc[0]);
+            acc[1] = fmaf(s0, cg[1], acc[1]);
+            acc[2] = fmaf(s1, cg[2], acc[2]);
+            acc[3] = fmaf(s1, cg[3], acc[3]);
+            cg[0] = cg[1] = cg[2] = cg[3] = 0.0f;
+          }
+          round_end = ++c_blk == nblk;
+          if (round_end) {
+            c_blk = 0;
+            xl = xl0;
+          }
+        }
+        if (round_end) {
+          // the S warps of each row block add their partial sums
+          float* buf = red + (c_round & 1) * (AWQ_WARPS * 32 * 4);
+          *reinterpret_cast<float4*>(buf + (warp * 32 + lane) * 4) =
+              make_float4(acc[0], acc[1], acc[2], acc[3]);
+          acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+          named_barrier_sync(1, AWQ_THREADS);
+          const int rbase = ((int)blockIdx.x + c_round * (int)gridDim.x) * R;
+          for (int o = threadIdx.x; o < R * 16 * MT; o += AWQ_THREADS) {
+            const int rl = o / (16 * MT), rem = o - rl * (16 * MT);
+            const int row = rem / MT, m = rem - row * MT;
+            const int src = (row & 7) * 4 + (m >> 1);      // the fragment's lane
+            const int idx = (row >> 3) * 2 + (m & 1);      // and element
+            float y = 0.0f;
+            for (int s = 0; s < S; ++s) y += buf[((rl * S + s) * 32 + src) * 4 + idx];
+            const int n = (rbase + rl) * 16 + row;
+            if (rbase + rl < rb_total && n < N) {
+              if (bias) y += bf16_lo_f32(bias[n]);
+              Y[(size_t)m * ldy + n] =
+                  (uint16_t)(__float_as_uint(__bfloat162float(__float2bfloat16_rn(y))) >> 16);
+            }
+          }
+          ++c_round;
+        }
+      }
     }
   }
 }

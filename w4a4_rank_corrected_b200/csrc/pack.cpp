@@ -507,6 +507,38 @@ static double half_to_double(uint16_t h) {
   return (h & 0x8000) ? -v : v;
 }
 
+// The AWQ GEMV's code layout: per 16-row block and 64-deep block of K, 512
+// bytes = 32 lanes x 16 bytes; lane l = 4 g + c holds one 32-bit word per
+// 16-deep k-step ks (4 per block), and nibble j of the word is the code of
+//   row 16 rb + g + 8 (j % 2),  column 16 ks + 2 c + 8 ((j % 4) / 2) + j / 4
+// (the m16n8k16 A-fragment element of register j % 4, half j / 4).  Rows
+// past N hold code 0.
+extern "C" svdq_status svdq_awq_tile_codes(const uint8_t* q_rowmajor, int N, int K,
+                                           uint8_t* q_tiled) {
+  if (!q_rowmajor || !q_tiled || N <= 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
+  const int RB = (N + 15) / 16, KS = K / 16;
+#pragma omp parallel for schedule(static)
+  for (int rb = 0; rb < RB; ++rb)
+    for (int ks = 0; ks < KS; ++ks)
+      for (int l = 0; l < 32; ++l) {
+        const int g = l >> 2, c = l & 3;
+        uint32_t word = 0;
+        for (int j = 0; j < 8; ++j) {
+          const int n = 16 * rb + g + 8 * (j & 1);
+          const int k = 16 * ks + 2 * c + 8 * ((j & 3) >> 1) + (j >> 2);
+          uint32_t code = 0;
+          if (n < N) {
+            const uint8_t b = q_rowmajor[(size_t)n * (K / 2) + k / 2];
+            code = (k & 1) ? (b >> 4) : (b & 15u);
+          }
+          word |= code << (4 * j);
+        }
+        const size_t off = (((size_t)rb * (K / 64) + (ks >> 2)) * 32 + l) * 16 + (ks & 3) * 4;
+        std::memcpy(q_tiled + off, &word, 4);
+      }
+  return SVDQ_OK;
+}
+
 extern "C" svdq_status svdq_awq_pack(const float* W, int N, int K, int group, uint8_t* q_packed,
                                      uint8_t* zeros, uint16_t* scales) {
   if (!W || !q_packed || !zeros || !scales || N <= 0 || K <= 0 || group <= 0 || group % 32 ||

@@ -674,7 +674,7 @@ template <int MT>
 svdq_status launch_awq(const uint8_t* q, const uint8_t* zeros, const uint16_t* scales,
                        const uint16_t* bias, int N, int K, int group, const uint16_t* X,
                        int64_t ldx, uint16_t* Y, int64_t ldy, cudaStream_t s, int sms) {
-  const size_t smem = (size_t)MT * (K / 32) * AWQ_CHUNK_PAD * 4;
+  const size_t smem = awq_smem_bytes(MT, K);
   if (cudaFuncSetAttribute(awq_gemv_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess) {
     cudaGetLastError();
@@ -687,10 +687,17 @@ svdq_status launch_awq(const uint8_t* q, const uint8_t* zeros, const uint16_t* s
     cudaGetLastError();
     per_sm = 1;
   }
-  const int warps = AWQ_THREADS / 32;
-  const int blocks = std::max(1, std::min((N + warps - 1) / warps, per_sm * sms));
-  awq_gemv_kernel<MT><<<blocks, AWQ_THREADS, smem, s>>>(q, zeros, scales, bias, N, K, group, X,
-                                                        ldx, Y, ldy);
+  // S warps per 16-row block split K: the smallest split that gives every
+  // resident warp slot a block (while each K slice keeps a group)
+  const int rb_total = (N + 15) / 16, G = K / group;
+  const long long slots = (long long)per_sm * sms * AWQ_WARPS;
+  int S = 1;
+  while (S < AWQ_WARPS && (long long)rb_total * S < slots && 2 * S <= G) S *= 2;
+  const int R = AWQ_WARPS / S;
+  const int rounds = (rb_total + R - 1) / R;
+  const int blocks = std::max(1, std::min(rounds, per_sm * sms));
+  awq_gemv_kernel<MT><<<blocks, AWQ_THREADS, smem, s>>>(q, zeros, scales, bias, N, K, group, S,
+                                                        X, ldx, Y, ldy);
   return cudaGetLastError() == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 
@@ -698,13 +705,12 @@ extern "C" svdq_status svdq_awq_linear(const uint8_t* q, const uint8_t* zeros,
                                        const uint16_t* scales, const uint16_t* bias, int N, int K,
                                        int group, const uint16_t* X, int M, int64_t ldx,
                                        uint16_t* Y, int64_t ldy, void* stream) {
-  if (N <= 0 || K <= 0 || group <= 0 || group % 32 || K % group) return SVDQ_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || group <= 0 || group % 64 || K % group) return SVDQ_ERR_INVALID_ARG;
   if (M < 0 || M > AWQ_MAX_M || ldx < K || ldy < N) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   if (!q || !zeros || !scales || !X || !Y) return SVDQ_ERR_INVALID_ARG;
-  if ((size_t)M * (K / 32) * AWQ_CHUNK_PAD * 4 > 200u * 1024u)
-    return SVDQ_ERR_INVALID_ARG;   // X staged in smem
-  if (!aligned16(q)) return SVDQ_ERR_MISALIGNED;
+  if (awq_smem_bytes(M, K) > AWQ_SMEM_MAX) return SVDQ_ERR_INVALID_ARG;   // X staged in smem
+  if (!aligned16(q) || !aligned16(X) || ldx % 8) return SVDQ_ERR_MISALIGNED;
   int sms = 0;
   svdq_status st = device_check(&sms);
   if (st != SVDQ_OK) return st;
