@@ -388,7 +388,7 @@ svdq_status svdq_awq_tile_codes(const uint8_t* q_rowmajor, int N, int K, uint8_t
  * group the sum of (q - z) x is accumulated in fp32 (products exact), then
  * scaled by the group's fp16 scale and added in fp32.  For the batch sizes
  * of modulation layers: 1 <= M <= 8 (a memory-bound product over the weight
- * stream), group a multiple of 64 dividing K, and 8 KB + M * K * 2 bytes
+ * stream), group a multiple of 128 dividing K, and 8 KB + M * K * 2 bytes
  * <= 216 KB (X is staged in shared memory).
  *   q      device, tiled as svdq_awq_tile_codes writes it (16-byte aligned)
  *   zeros, scales  device, as svdq_awq_pack writes them ([N][K/group])

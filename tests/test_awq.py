@@ -70,7 +70,7 @@ def test_awq_argument_validation():
     f = L.svdq_awq_linear
     assert f(Q, Z, SC, None, 64, 128, 128, X, 9, 128, Y, 64, None) == 1        # M > 8
     assert f(Q, Z, SC, None, 64, 128, 100, X, 1, 128, Y, 64, None) == 1       # group
-    assert f(Q, Z, SC, None, 64, 128, 32, X, 1, 128, Y, 64, None) == 1        # group % 64
+    assert f(Q, Z, SC, None, 64, 128, 64, X, 1, 128, Y, 64, None) == 1        # group % 128
     assert f(Q, Z, SC, None, 64, 128, 128, X, 1, 100, Y, 64, None) == 1       # ldx < K
     assert f(Q + 8, Z, SC, None, 64, 128, 128, X, 1, 128, Y, 64, None) == 3   # alignment
     assert f(Q, Z, SC, None, 64, 16384, 128, X, 8, 16384, Y, 64, None) == 1   # X too big to stage

@@ -26,17 +26,18 @@
 //     shift and one bitwise op (the nibble lands in the low mantissa bits
 //     of 128.0), then q - z exactly with one bf16x2 subtraction of
 //     (128 + z, 128 + z);
-//   * per group the MMA accumulator holds sum_k (q_k - z) x_k (products
-//     exact, fp32 accumulation); it is scaled by the group's fp16 scale and
-//     added to the running sum (one FMA per output);
+//   * per group the MMA accumulators (two, for even and odd k-steps) hold
+//     sum_k (q_k - z) x_k (products exact, fp32 accumulation); the group's
+//     fp16 scale multiplies it into the running sum (one FMA per output);
 //   * X is staged once per CTA in shared memory (16-byte loads), per k-step
 //     and batch row 16 values in B-fragment order (lane c's four values
 //     adjacent: one 8-byte load);
 //   * a CTA's eight warps cover 8 / S row blocks, S warps splitting K per
 //     block (S chosen by the host so the grid has enough warps); their
 //     partial sums meet in shared memory, bias is added and Y is rounded
-//     once to bf16.  Each warp keeps eight 512-byte code blocks (with their
-//     scales and zeros) in flight ahead of the one it computes.
+//     once to bf16.  A warp works in 128-deep slots (two 512-byte blocks of
+//     codes, one group's scales and zeros; the group size is a multiple of
+//     128) and keeps four slots in flight ahead of the one it computes.
 #pragma once
 #include <cuda_fp16.h>
 #include "ptx.cuh"
@@ -46,7 +47,7 @@ namespace svdq_dev {
 constexpr int AWQ_THREADS = 256;
 constexpr int AWQ_WARPS = AWQ_THREADS / 32;
 constexpr int AWQ_MAX_M = 8;
-constexpr int AWQ_PF = 8;                                // code blocks in flight per warp
+constexpr int AWQ_PF = 4;                                // 1 KB slots in flight per warp
 constexpr uint32_t AWQ_SMEM_MAX = 216u * 1024u;
 constexpr int AWQ_RED_FLOATS = 2 * AWQ_WARPS * 32 * 4;   // two buffers of partial fragments
 
@@ -83,8 +84,8 @@ __device__ __forceinline__ uint32_t awq_pair128(uint32_t shifted) {
   return (shifted & 0x000F000Fu) | 0x43004300u;
 }
 
-struct AwqSlot {   // one code block in flight: codes, and its group's scales and zeros
-  uint4 w;
+struct AwqSlot {   // one 128-deep slot in flight: codes, and its group's scales and zeros
+  uint4 w0, w1;    // the slot's two 512-byte blocks (this lane's 16 bytes of each)
   uint32_t s;      // fp16 bits: row g (low half), row g + 8 (high half)
   uint32_t z;      // zeros: row g (bits 0..7), row g + 8 (bits 16..23)
 };
@@ -101,7 +102,7 @@ __global__ void __launch_bounds__(AWQ_THREADS, 2)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, c = lane & 3;
   const int G = K / group;
-  const int bpg = group >> 6;                 // 64-deep code blocks per group
+  const int spg = group >> 7;                 // 128-deep slots per group
   const int R = AWQ_WARPS / S;                // row blocks per CTA per round
   const int rb_total = (N + 15) >> 4;
   const int rounds = (rb_total + R - 1) / R;
@@ -110,15 +111,15 @@ __global__ void __launch_bounds__(AWQ_THREADS, 2)
   const int sub = warp % S, rloc = warp / S;
   const int gps = (G + S - 1) / S;            // groups per K slice
   const int g0 = min(G, sub * gps), g1 = min(G, g0 + gps);
-  const int nblk = (g1 - g0) * bpg;           // this warp's code blocks per round
-  const int total = my_rounds * nblk;
+  const int nsl = (g1 - g0) * spg;            // this warp's slots per round
+  const int total = my_rounds * nsl;
+  const int sk0 = g0 * spg;                   // first slot of this warp's K slice
 
-  // ---- fetch side of this warp's sequence of (round, block): pointers
-  // advanced per block (no per-block index arithmetic) ----
-  const int kb0 = g0 * bpg;                   // first 64-deep block of this warp's slice
-  int f_round = 0, f_blk = 0, f_ing = 0;      // round, block in the round, block in the group
+  // ---- fetch side of this warp's sequence of (round, slot): pointers
+  // advanced per slot, recomputed once per round ----
+  int f_round = 0, f_sl = 0, f_ing = 0;       // round, slot in the round, slot in the group
   bool f_ok = false, f_ok0 = false, f_ok1 = false;
-  const uint4* f_q = nullptr;
+  const uint4* f_q = reinterpret_cast<const uint4*>(q);
   const uint16_t *f_s0 = scales, *f_s1 = scales;
   const uint8_t *f_z0 = zeros, *f_z1 = zeros;
   auto f_start_round = [&]() {
@@ -127,7 +128,7 @@ __global__ void __launch_bounds__(AWQ_THREADS, 2)
     f_ok = rb < rb_total;
     f_ok0 = n0 < N;
     f_ok1 = n0 + 8 < N;
-    f_q = reinterpret_cast<const uint4*>(q + awq_tile_word_offset(f_ok ? rb : 0, 4 * kb0, lane, K));
+    f_q = reinterpret_cast<const uint4*>(q + awq_tile_word_offset(f_ok ? rb : 0, 8 * sk0, lane, K));
     const size_t r0 = f_ok0 ? (size_t)n0 * G + g0 : 0, r1 = f_ok1 ? (size_t)(n0 + 8) * G + g0 : 0;
     f_s0 = scales + r0;
     f_s1 = scales + r1;
@@ -136,21 +137,26 @@ __global__ void __launch_bounds__(AWQ_THREADS, 2)
     f_ing = 0;
   };
   auto fetch = [&](AwqSlot& sl) {
-    sl.w = f_ok ? __ldcs(f_q) : make_uint4(0, 0, 0, 0);
+    if (f_ok) {
+      sl.w0 = __ldcs(f_q);
+      sl.w1 = __ldcs(f_q + 32);               // the next 512-byte block
+    } else {
+      sl.w0 = sl.w1 = make_uint4(0, 0, 0, 0);
+    }
     sl.s = (f_ok0 ? (uint32_t)__ldg(f_s0) : 0u) | ((f_ok1 ? (uint32_t)__ldg(f_s1) : 0u) << 16);
     sl.z = (f_ok0 ? (uint32_t)__ldg(f_z0) : 0u) | ((f_ok1 ? (uint32_t)__ldg(f_z1) : 0u) << 16);
-    f_q += 32;                                // the next 512-byte block of this row block
-    if (++f_ing == bpg) {
+    f_q += 64;
+    if (++f_ing == spg) {
       f_ing = 0;
       ++f_s0, ++f_s1, ++f_z0, ++f_z1;
     }
-    if (++f_blk == nblk) {
-      f_blk = 0;
+    if (++f_sl == nsl) {
+      f_sl = 0;
       ++f_round;
       f_start_round();
     }
   };
-  if (nblk > 0) f_start_round();
+  if (nsl > 0) f_start_round();
   AwqSlot ring[AWQ_PF];
 #pragma unroll
   for (int j = 0; j < AWQ_PF; ++j)
@@ -190,60 +196,66 @@ __global__ void __launch_bounds__(AWQ_THREADS, 2)
   __syncthreads();
 
   float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  float cg[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  int c_round = 0, c_blk = 0, c_ing = 0;
-  // this lane's B fragment: batch row g, values 4c .. 4c+3 of each k-step's 16
+  float ce[4] = {0.0f, 0.0f, 0.0f, 0.0f}, co[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // even / odd k-steps
+  int c_round = 0, c_sl = 0, c_ing = 0;
+  // this lane's B fragment: batch row g, values 4c .. 4c+3 of each k-step's
+  // 16; a lane past the batch keeps zeros
   const bool has_b = g < MT;
   const uint2* xl0 = reinterpret_cast<const uint2*>(xs + (size_t)(has_b ? g : 0) * 16 + 4 * c) +
-                     (size_t)kb0 * 4 * MT * 4;
+                     (size_t)sk0 * 8 * MT * 4;
   const uint2* xl = xl0;
-  // a warp without code blocks still takes one step per round (the CTA's
-  // barrier is passed by every warp once per round)
-  const int steps = nblk > 0 ? total : my_rounds;
+  uint32_t b0 = 0, b1 = 0;
+  // a warp without slots still takes one step per round (the CTA's barrier
+  // is passed by every warp once per round)
+  const int steps = nsl > 0 ? total : my_rounds;
   for (int base = 0; base < steps; base += AWQ_PF) {
 #pragma unroll
     for (int j = 0; j < AWQ_PF; ++j) {
       const int item = base + j;
       if (item < steps) {
         bool round_end = true;
-        if (nblk > 0) {
+        if (nsl > 0) {
           const AwqSlot sl = ring[j];
           if (item + AWQ_PF < total) fetch(ring[j]);
           // (128 + z) in both halves, for each of this lane's two rows
           const uint32_t zz0 = ((sl.z & 0xFFu) * 0x00010001u) | 0x43004300u;
           const uint32_t zz1 = ((sl.z >> 16) * 0x00010001u) | 0x43004300u;
-          const uint32_t words[4] = {sl.w.x, sl.w.y, sl.w.z, sl.w.w};
+          const uint32_t words[8] = {sl.w0.x, sl.w0.y, sl.w0.z, sl.w0.w,
+                                     sl.w1.x, sl.w1.y, sl.w1.z, sl.w1.w};
 #pragma unroll
-          for (int t = 0; t < 4; ++t) {
+          for (int t = 0; t < 8; ++t) {
             const uint32_t wd = words[t];
             uint32_t a[4];
             a[0] = bf16x2_sub(awq_pair128(wd), zz0);         // row g,     k 2c, 2c+1
             a[1] = bf16x2_sub(awq_pair128(wd >> 4), zz1);    // row g + 8, k 2c, 2c+1
             a[2] = bf16x2_sub(awq_pair128(wd >> 8), zz0);    // row g,     k 2c+8, 2c+9
             a[3] = bf16x2_sub(awq_pair128(wd >> 12), zz1);   // row g + 8, k 2c+8, 2c+9
-            uint32_t b0 = 0, b1 = 0;
             if (has_b) {
-              const uint2 xv = xl[t * MT * 4];   // k-step t of the block: MT rows of 16 values
+              const uint2 xv = xl[t * MT * 4];   // k-step t of the slot: MT rows of 16 values
               b0 = xv.x;
               b1 = xv.y;
             }
-            mma_bf16_16816(cg, a, b0, b1);
+            if (t & 1)
+              mma_bf16_16816(co, a, b0, b1);
+            else
+              mma_bf16_16816(ce, a, b0, b1);
           }
-          xl += 4 * MT * 4;
-          if (++c_ing == bpg) {
+          xl += 8 * MT * 4;
+          if (++c_ing == spg) {
             c_ing = 0;
             // the group's sum of (q - z) x, times its scale
             const float s0 = __half2float(__ushort_as_half((unsigned short)(sl.s & 0xFFFFu)));
             const float s1 = __half2float(__ushort_as_half((unsigned short)(sl.s >> 16)));
-            acc[0] = fmaf(s0, cg[0], acc[0]);
-            acc[1] = fmaf(s0, cg[1], acc[1]);
-            acc[2] = fmaf(s1, cg[2], acc[2]);
-            acc[3] = fmaf(s1, cg[3], acc[3]);
-            cg[0] = cg[1] = cg[2] = cg[3] = 0.0f;
+            acc[0] = fmaf(s0, ce[0] + co[0], acc[0]);
+            acc[1] = fmaf(s0, ce[1] + co[1], acc[1]);
+            acc[2] = fmaf(s1, ce[2] + co[2], acc[2]);
+            acc[3] = fmaf(s1, ce[3] + co[3], acc[3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) ce[e] = co[e] = 0.0f;
           }
-          round_end = ++c_blk == nblk;
+          round_end = ++c_sl == nsl;
           if (round_end) {
-            c_blk = 0;
+            c_sl = 0;
             xl = xl0;
           }
         }
@@ -261,7 +273,7 @@ __global__ void __launch_bounds__(AWQ_THREADS, 2)
             const int src = (row & 7) * 4 + (m >> 1);      // the fragment's lane
             const int idx = (row >> 3) * 2 + (m & 1);      // and element
             float y = 0.0f;
-            for (int s = 0; s < S; ++s) y += buf[((rl * S + s) * 32 + src) * 4 + idx];
+            for (int s2 = 0; s2 < S; ++s2) y += buf[((rl * S + s2) * 32 + src) * 4 + idx];
             const int n = (rbase + rl) * 16 + row;
             if (rbase + rl < rb_total && n < N) {
               if (bias) y += bf16_lo_f32(bias[n]);

@@ -705,7 +705,7 @@ extern "C" svdq_status svdq_awq_linear(const uint8_t* q, const uint8_t* zeros,
                                        const uint16_t* scales, const uint16_t* bias, int N, int K,
                                        int group, const uint16_t* X, int M, int64_t ldx,
                                        uint16_t* Y, int64_t ldy, void* stream) {
-  if (N <= 0 || K <= 0 || group <= 0 || group % 64 || K % group) return SVDQ_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || group <= 0 || group % 128 || K % group) return SVDQ_ERR_INVALID_ARG;
   if (M < 0 || M > AWQ_MAX_M || ldx < K || ldy < N) return SVDQ_ERR_INVALID_ARG;
   if (M == 0) return SVDQ_OK;
   if (!q || !zeros || !scales || !X || !Y) return SVDQ_ERR_INVALID_ARG;
