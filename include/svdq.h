@@ -226,6 +226,35 @@ svdq_status svdq_gemm(const svdq_weight* w, const uint8_t* codes_x,
                       const uint8_t* sf_x, const uint16_t* xl1, int M,
                       uint16_t* Y, int64_t ldy, void* stream);
 
+/* Bytes of the workspace of svdq_gemm_splitk for an M x N x K layer (the
+ * partials: tiles x parts x 256 x 256 fp32); 0 when the GEMM does not split
+ * (32 or more 256 x 256 output tiles, or a single 256-deep K stage). */
+size_t svdq_gemm_workspace_bytes(int M, int N, int K);
+
+/* svdq_gemm_splitk: svdq_gemm for layers with few output tiles (small M,
+ * where whole-K tiles would leave most SMs idle; the pages' small-batch
+ * latency concern, Vietnamese rendering, "End-to-end latency and memory").
+ * Each tile's K stages are split into up to 8 parts ("units") run by
+ * different CTA pairs (about 64 units in all); every unit stores its fp32
+ * partial accumulator in the workspace, and a second kernel (chained by
+ * programmatic dependent launch, the whole GPU wide) adds the partials in
+ * part order -- Y is deterministic -- and applies alpha, bias and the bf16
+ * store.  The low-rank branch is accumulated by the last K part.  Same
+ * result as svdq_gemm up to the fp32 summation order.  Two launches.
+ *   workspace  device, 256-byte aligned, >= svdq_gemm_workspace_bytes(M, N, K)
+ *              (may be NULL when that is 0); contents need not be preserved
+ * Errors as svdq_gemm, plus SVDQ_ERR_WORKSPACE. */
+svdq_status svdq_gemm_splitk(const svdq_weight* w, const uint8_t* codes_x,
+                             const uint8_t* sf_x, const uint16_t* xl1, int M,
+                             uint16_t* Y, int64_t ldy, void* workspace, size_t ws_bytes,
+                             void* stream);
+
+/* Bytes of a svdq_linear_forward workspace that also holds the split-K
+ * partials (svdq_act_workspace_bytes rounded up to 256, plus
+ * svdq_gemm_workspace_bytes); equal to svdq_act_workspace_bytes when the
+ * GEMM does not split.  0 on bad arguments. */
+size_t svdq_forward_workspace_bytes(const svdq_weight* w, int M);
+
 /* svdq_gemm_gelu: svdq_gemm for the first linear of an MLP pair, with the
  * pair's GELU fused into the epilogue.  Source: the fused GELU/MLP kernels
  * the pages name as part of the original engine's speed ("Bringing Nunchaku
@@ -262,7 +291,9 @@ svdq_status svdq_mlp_forward(const svdq_weight* w1, const svdq_weight* w2,
  * + bias ("Background: SVDQuant and Nunchaku"; the runtime SVDQW4A4Linear
  * layer that replaces nn.Linear in "Loading natively in Diffusers"):
  * svdq_quantize_act then svdq_gemm on one stream, with the intermediates in
- * `workspace` (device, >= svdq_act_workspace_bytes, 256-byte aligned). */
+ * `workspace` (device, >= svdq_act_workspace_bytes, 256-byte aligned).  With
+ * a workspace of svdq_forward_workspace_bytes(w, M) the GEMM runs split-K
+ * (svdq_gemm_splitk) when the layer has few output tiles. */
 svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t* X,
                                 int M, int64_t ldx, uint16_t* Y, int64_t ldy,
                                 void* workspace, size_t ws_bytes,

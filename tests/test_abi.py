@@ -70,6 +70,43 @@ def test_workspace_bytes():
     assert S.svdq_act_workspace_bytes(100, 3000, 32) == 0
 
 
+def test_split_k_workspace_rule():
+    """svdq_gemm_workspace_bytes restated: at most 16 output tiles of
+    256 x 256 and at least 24 stages of 256 along K split each tile's K into
+    min(8, 64 // tiles, stages // 6) parts; partials are
+    [tiles][parts][2][128][256] fp32."""
+    def rule(M, N, K):
+        tiles = -(-M // 256) * -(-N // 256)
+        stages = -(-(K // 64) // 4)
+        if tiles > 16 or stages < 24:
+            return 0
+        parts = max(1, min(8, 64 // tiles, stages // 6))
+        if parts <= 1:
+            return 0
+        return tiles * parts * 2 * 128 * 256 * 4
+    for M, N, K in [(64, 3072, 3072), (4608, 9216, 3072), (256, 12288, 3072), (512, 3072, 12288),
+                    (1, 16, 64), (129, 272, 320), (300, 784, 768), (257, 3072, 3072),
+                    (2048, 3072, 12288), (64, 128, 12288), (64, 3072, 12288), (200, 256, 6144),
+                    (64, 4096, 6144), (16, 640, 6144)]:
+        assert S.svdq_gemm_workspace_bytes(M, N, K) == rule(M, N, K), (M, N, K)
+    assert S.svdq_gemm_workspace_bytes(64, 3072, 12288) == 12 * 5 * 262144
+    assert S.svdq_gemm_workspace_bytes(64, 3072, 3072) == 0
+    # the forward workspace adds it after the activation workspace (256-aligned)
+    w = _fake_weight(N=3072, K=12288, r=32)
+    a = S.svdq_act_workspace_bytes(64, 12288, 32)
+    assert S.lib.svdq_forward_workspace_bytes(ctypes.byref(w), 64) == \
+        -(-a // 256) * 256 + rule(64, 3072, 12288)
+    assert S.lib.svdq_forward_workspace_bytes(ctypes.byref(w), 4608) == \
+        S.svdq_act_workspace_bytes(4608, 12288, 32)
+    # a split GEMM refuses a short workspace before touching the device
+    C, SF, XL = 0x30000000, 0x40000000, 0x50000000
+    need = S.svdq_gemm_workspace_bytes(64, 3072, 12288)
+    assert S.lib.svdq_gemm_splitk(ctypes.byref(w), C, SF, XL, 64, 0x60000000, 3072,
+                                  0x70000000, need - 1, None) == 4
+    assert S.lib.svdq_gemm_splitk(ctypes.byref(w), C, SF, XL, 64, 0x60000000, 3072,
+                                  None, 0, None) == 4
+
+
 def _fake_weight(N=256, K=256, r=32, base=0x10000000):
     w = S.SvdqWeight()
     w.N, w.K, w.r = N, K, r

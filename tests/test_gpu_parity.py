@@ -164,6 +164,38 @@ def test_linear_forward_parity(M, K, N, r):
     check_output(from_dev_bf16(Y), Y_ref)
 
 
+SPLIT_CASES = [  # M, K, N, r: few output tiles and long K, so the GEMM splits K
+    (64, 12288, 3072, 32), (200, 6144, 256, 0), (300, 8192, 512, 32), (16, 6144, 640, 128),
+]
+
+
+@pytest.mark.parametrize("M,K,N,r", SPLIT_CASES)
+def test_gemm_splitk_parity_and_determinism(M, K, N, r):
+    """Split-K GEMM: within tolerance of the oracle, bit-identical across
+    calls (the partials are added in part order), with a workspace that
+    starts out as garbage."""
+    S = _S()
+    need = S.svdq_gemm_workspace_bytes(M, N, K)
+    assert need > 0
+    X, W, b = SI.random_layer(M + 7 * K + N, M, K, N)
+    lp, op, dw = prepare(W, SI.channel_absmax(X), r, b)
+    codes, sf, xl1 = S.svdq_quantize_act(dw, to_dev_bf16(X))
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device="cuda")
+    Y1 = S.svdq_gemm_splitk(dw, codes, sf, xl1, M, workspace=ws).clone()
+    Y2 = S.svdq_gemm_splitk(dw, codes, sf, xl1, M, workspace=ws)
+    Y0 = S.svdq_gemm(dw, codes, sf, xl1, M)
+    torch.cuda.synchronize()
+    assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+    Y_ref, _, _, _ = O.linear_reference(X, op, b)
+    check_output(from_dev_bf16(Y1), Y_ref)
+    check_output(from_dev_bf16(Y0), Y_ref)
+    # the forward with a workspace that has room for the partials splits too
+    Yf = S.svdq_linear_forward(dw, to_dev_bf16(X))
+    torch.cuda.synchronize()
+    assert torch.equal(Yf.view(torch.int16), Y1.view(torch.int16))
+    assert S.svdq_device_error() == 0
+
+
 def test_zero_input_gives_bias_exactly():
     S = _S()
     M, K, N, r = 130, 256, 512, 32
@@ -364,7 +396,9 @@ def test_host_forward_strided_host_buffers():
     Yh = Yh_full[:, :N]
     Xd = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
     Yd = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
-    ws = S.new_workspace(M, K, r)
+    # the same workspace size as the reference call below (with room for the
+    # split-K partials), so both take the same GEMM path
+    ws = S.new_forward_workspace(dw, M)
     S.svdq_linear_forward_host(dw, Xh, Yh, Xd, Yd, ws)
     torch.cuda.synchronize()
     ref = from_dev_bf16(S.svdq_linear_forward(dw, to_dev_bf16(X)))

@@ -26,7 +26,8 @@ __all__ = [
     "SvdqError", "PackedWeight", "DeviceWeight", "svdq_query_sizes", "svdq_pack_weight",
     "svdq_quantize_act", "svdq_gemm", "svdq_linear_forward", "svdq_act_workspace_bytes",
     "svdq_linear_forward_host", "svdq_linear_forward_static", "svdq_unswizzle_scales",
-    "new_workspace", "svdq_gemm_gelu",
+    "new_workspace", "svdq_gemm_gelu", "svdq_gemm_splitk", "svdq_gemm_workspace_bytes",
+    "svdq_forward_workspace_bytes", "new_forward_workspace",
     "svdq_mlp_forward", "svdq_mlp_workspace_bytes", "new_mlp_workspace", "svdq_debug_gelu",
     "svdq_act_row_scales", "svdq_quantize_act_dynamic", "svdq_gemm_dynamic",
     "svdq_dyn_workspace_bytes", "svdq_linear_forward_dynamic", "svdq_awq_pack",
@@ -94,6 +95,9 @@ def _load() -> ctypes.CDLL:
         "svdq_act_workspace_bytes": (SZ, [I, I, I]),
         "svdq_quantize_act": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, P, P, P]),
         "svdq_gemm": (I, [ctypes.POINTER(SvdqWeight), P, P, P, I, P, I64, P]),
+        "svdq_gemm_workspace_bytes": (SZ, [I, I, I]),
+        "svdq_gemm_splitk": (I, [ctypes.POINTER(SvdqWeight), P, P, P, I, P, I64, P, SZ, P]),
+        "svdq_forward_workspace_bytes": (SZ, [ctypes.POINTER(SvdqWeight), I]),
         "svdq_linear_forward": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P, SZ, P]),
         "svdq_linear_forward_static": (I, [ctypes.POINTER(SvdqWeight), P, I, I64, P, I64, P]),
         "svdq_device_error": (I, [P, ctypes.POINTER(I)]),
@@ -148,9 +152,26 @@ def svdq_act_workspace_bytes(M: int, K: int, r: int) -> int:
 
 
 def new_workspace(M: int, K: int, r: int, device="cuda"):
-    """A forward workspace of svdq_act_workspace_bytes(M, K, r) bytes."""
+    """A forward workspace of svdq_act_workspace_bytes(M, K, r) bytes (the
+    minimum: the GEMM then never splits K)."""
     import torch
     return torch.empty(max(svdq_act_workspace_bytes(M, K, r), 256), dtype=torch.uint8,
+                       device=device)
+
+
+def svdq_gemm_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib.svdq_gemm_workspace_bytes(M, N, K))
+
+
+def svdq_forward_workspace_bytes(w: "DeviceWeight", M: int) -> int:
+    return int(lib.svdq_forward_workspace_bytes(ctypes.byref(w.struct), M))
+
+
+def new_forward_workspace(w: "DeviceWeight", M: int, device="cuda"):
+    """A forward workspace with room for the split-K partials when the layer
+    has few output tiles (svdq_forward_workspace_bytes)."""
+    import torch
+    return torch.empty(max(svdq_forward_workspace_bytes(w, M), 256), dtype=torch.uint8,
                        device=device)
 
 
@@ -361,12 +382,32 @@ def svdq_linear_forward(w: DeviceWeight, X, Y=None, workspace=None, stream=None)
         Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=X.device)
         made.append(Y)
     if workspace is None:
-        workspace = new_workspace(M, w.K, w.r, X.device)
+        workspace = new_forward_workspace(w, M, X.device)
         made.append(workspace)
     _check(lib.svdq_linear_forward(ctypes.byref(w.struct), X.data_ptr(), M, X.stride(0),
                                    Y.data_ptr(), Y.stride(0), workspace.data_ptr(),
                                    workspace.numel(), _stream_ptr(stream)),
            "svdq_linear_forward")
+    _keep_alive_on(stream, *made)
+    return Y
+
+
+def svdq_gemm_splitk(w: DeviceWeight, codes_x, sf_x, xl1, M: int, Y=None, workspace=None,
+                     stream=None):
+    """svdq_gemm with K split across CTA pairs when the output has few tiles."""
+    import torch
+    made = []
+    if Y is None:
+        Y = torch.empty((M, w.N), dtype=torch.bfloat16, device=codes_x.device)
+        made.append(Y)
+    need = svdq_gemm_workspace_bytes(M, w.N, w.K)
+    if workspace is None and need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=codes_x.device)
+        made.append(workspace)
+    _check(lib.svdq_gemm_splitk(ctypes.byref(w.struct), codes_x.data_ptr(), sf_x.data_ptr(),
+                                _ptr(xl1), M, Y.data_ptr(), Y.stride(0), _ptr(workspace),
+                                0 if workspace is None else workspace.numel(),
+                                _stream_ptr(stream)), "svdq_gemm_splitk")
     _keep_alive_on(stream, *made)
     return Y
 
@@ -620,7 +661,7 @@ class HostStreamer:
         self.w, self.M = w, M
         self.X = [torch.empty((M, w.K), dtype=torch.bfloat16, device=device) for _ in range(2)]
         self.Y = [torch.empty((M, w.N), dtype=torch.bfloat16, device=device) for _ in range(2)]
-        self.ws = [new_workspace(M, w.K, w.r, device) for _ in range(2)]
+        self.ws = [new_forward_workspace(w, M, device) for _ in range(2)]
         self.streams = [torch.cuda.Stream(device=device) for _ in range(2)]
         self.n = 0
 
@@ -684,8 +725,8 @@ class SVDQW4A4Linear(_linear_module_base()):
         lead = X.shape[:-1]
         X2 = X.reshape(-1, X.shape[-1])
         M = X2.shape[0]
-        need = svdq_act_workspace_bytes(M, self.packed.K, self.packed.r)
+        need = svdq_forward_workspace_bytes(self.dev, M)
         if self._ws is None or self._ws.numel() < need or self._ws.device != X.device:
-            self._ws = new_workspace(M, self.packed.K, self.packed.r, X.device)
+            self._ws = new_forward_workspace(self.dev, M, X.device)
         Y = svdq_linear_forward(self.dev, X2, workspace=self._ws)
         return Y.reshape(*lead, self.out_features)

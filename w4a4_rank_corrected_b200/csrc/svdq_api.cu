@@ -401,13 +401,39 @@ int gemm_max_pairs(int sms) {
   return std::max(1, cached);
 }
 
+// Split-K for few output tiles and long K: with at most 16 tiles of
+// 256 x 256 (the GEMM has 74 CTA pairs on a B200) and at least 24 stages of
+// 256 along K, each tile's K is split into min(8, 64 / tiles, stages / 6)
+// parts.  The split adds a second kernel and a round trip of fp32 partials
+// through L2, about 5 us; measured, it pays at K = 12288 (M = 64: 16.5 against
+// 21.2 us whole-K; M = 256: 18.5 against 22.0 us), breaks even at 24 tiles and
+// loses at K = 3072 (12.4 against 9.2 us).  The rule depends on the shapes
+// only, so the workspace size does too.
+constexpr int kSplitTileLimit = 16;
+constexpr int kSplitMinStages = 24;
+constexpr int kSplitUnits = 64;
+constexpr int kSplitMax = 8;
+int gemm_tiles(int M, int N) { return ((M + 2 * G_BM - 1) / (2 * G_BM)) * ((N + G_BN - 1) / G_BN); }
+int gemm_ksplit(int M, int N, int K) {
+  const int tiles = gemm_tiles(M, N), kb_total = (K / 64 + 3) / 4;
+  if (tiles > kSplitTileLimit || kb_total < kSplitMinStages) return 1;
+  return std::max(1, std::min(std::min(kSplitMax, kSplitUnits / tiles), kb_total / 6));
+}
+// partials [tiles][ksplit][2][128][256] fp32
+size_t gemm_split_ws_bytes(int M, int N, int K) {
+  if (M <= 0 || gemm_ksplit(M, N, K) <= 1) return 0;
+  return (size_t)gemm_tiles(M, N) * gemm_ksplit(M, N, K) * 2 * G_BM * G_BN * 4;
+}
+
 svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint8_t* sf_x,
                         const uint16_t* xl1, int M, uint16_t* Y, int64_t ldy, cudaStream_t s,
-                        int sms, bool gelu = false, const RowScale* rs = nullptr) {
+                        int sms, bool gelu = false, const RowScale* rs = nullptr,
+                        void* split_ws = nullptr) {
   const int N = w->N, K = w->K, r = w->r, klr = klr_of(r);
-  CUtensorMap ta, tb, tsa, tsb, talr, tblr, ty;
+  CUtensorMap ta, tb, tsa, tsb, talr, tblr, ty, tpart;
   std::memset(&talr, 0, sizeof(talr));
   std::memset(&tblr, 0, sizeof(tblr));
+  std::memset(&tpart, 0, sizeof(tpart));
   // scale buffers as rows of 256 bytes (half a 512-byte atom), unswizzled
   const uint64_t sfa_rows = rup((size_t)M, 128) * (K / 16) / 256;
   const uint64_t sfb_rows = rup((size_t)N, 256) * (K / 16) / 256;
@@ -441,8 +467,17 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   p.timeout_ns = kDefaultTimeoutNs;
   p.gelu = gelu ? 1 : 0;
   p.row_scales = rs;
-  const int tiles = ((M + 2 * G_BM - 1) / (2 * G_BM)) * ((N + G_BN - 1) / G_BN);
-  const int pairs = std::max(1, std::min(tiles, gemm_max_pairs(sms)));
+  const int tiles = gemm_tiles(M, N);
+  // (the split is for the plain layer: not with GELU or per-row scales)
+  p.ksplit = (split_ws && !gelu && !rs) ? gemm_ksplit(M, N, K) : 1;
+  p.partials = p.ksplit > 1 ? static_cast<float*>(split_ws) : nullptr;
+  // the partials as a 2-D fp32 tensor [tiles * ksplit * 256 rows][256], stored
+  // in 128-row x 32-column boxes (128-byte swizzle, as the Y boxes)
+  if (p.ksplit > 1 &&
+      !make_map(&tpart, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, p.partials, (uint64_t)G_BN,
+                (uint64_t)tiles * p.ksplit * 2 * G_BM, (uint64_t)G_BN * 4, 32, G_BM))
+    return SVDQ_ERR_CUDA;
+  const int pairs = std::max(1, std::min(tiles * p.ksplit, gemm_max_pairs(sms)));
   cudaLaunchConfig_t cfg;
   std::memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
@@ -457,9 +492,27 @@ svdq_status launch_gemm(const svdq_weight* w, const uint8_t* codes_x, const uint
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  if (cudaLaunchKernelEx(&cfg, w4a4_gemm_kernel, ta, tb, tsa, tsb, talr, tblr, ty, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, w4a4_gemm_kernel, ta, tb, tsa, tsb, talr, tblr, ty, tpart, p) !=
+      cudaSuccess) {
     cudaGetLastError();
     return SVDQ_ERR_CUDA;
+  }
+  if (p.ksplit > 1) {
+    // the partials -> Y, chained to the GEMM by programmatic dependent launch
+    const long long threads = (long long)M * (N / 8);
+    cudaLaunchConfig_t rc;
+    std::memset(&rc, 0, sizeof(rc));
+    rc.gridDim = dim3((unsigned)std::max(1LL, std::min((threads + 255) / 256, 4LL * sms)), 1, 1);
+    rc.blockDim = dim3(256, 1, 1);
+    rc.stream = s;
+    cudaLaunchAttribute ra = pdl_attr();
+    rc.attrs = &ra;
+    rc.numAttrs = 1;
+    if (cudaLaunchKernelEx(&rc, splitk_reduce_kernel, (const float*)p.partials, M, N, p.ksplit,
+                           p.alpha, p.bias, Y, ldy) != cudaSuccess) {
+      cudaGetLastError();
+      return SVDQ_ERR_CUDA;
+    }
   }
   return SVDQ_OK;
 }
@@ -521,6 +574,39 @@ extern "C" svdq_status svdq_gemm(const svdq_weight* w, const uint8_t* codes_x,
   int sms = 0;
   if ((st = device_check(&sms)) != SVDQ_OK) return st;
   return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, (cudaStream_t)stream, sms);
+}
+
+extern "C" size_t svdq_gemm_workspace_bytes(int M, int N, int K) {
+  if (M < 0 || N <= 0 || K <= 0 || K % 64) return 0;
+  return gemm_split_ws_bytes(M, N, K);
+}
+
+extern "C" svdq_status svdq_gemm_splitk(const svdq_weight* w, const uint8_t* codes_x,
+                                        const uint8_t* sf_x, const uint16_t* xl1, int M,
+                                        uint16_t* Y, int64_t ldy, void* workspace,
+                                        size_t ws_bytes, void* stream) {
+  svdq_status st = check_weight(w);
+  if (st != SVDQ_OK) return st;
+  if (M < 0 || ldy < w->N) return SVDQ_ERR_INVALID_ARG;
+  if (M == 0) return SVDQ_OK;
+  if (!codes_x || !sf_x || !Y || (w->r > 0 && !xl1)) return SVDQ_ERR_INVALID_ARG;
+  const size_t need = gemm_split_ws_bytes(M, w->N, w->K);
+  if (need && (!workspace || ws_bytes < need)) return SVDQ_ERR_WORKSPACE;
+  if (!aligned16(codes_x) || !aligned16(sf_x) || !aligned16(Y) || ldy % 8 ||
+      (xl1 && !aligned16(xl1)) || (reinterpret_cast<uintptr_t>(workspace) & 255) != 0)
+    return SVDQ_ERR_MISALIGNED;
+  int sms = 0;
+  if ((st = device_check(&sms)) != SVDQ_OK) return st;
+  return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, (cudaStream_t)stream, sms, false, nullptr,
+                     need ? workspace : nullptr);
+}
+
+extern "C" size_t svdq_forward_workspace_bytes(const svdq_weight* w, int M) {
+  if (!w || M < 0) return 0;
+  const size_t a = svdq_act_workspace_bytes(M, w->K, w->r);
+  if (!a && M > 0) return 0;
+  const size_t g = gemm_split_ws_bytes(M, w->N, w->K);
+  return g ? rup(a, 256) + g : a;
 }
 
 extern "C" svdq_status svdq_gemm_gelu(const svdq_weight* w, const uint8_t* codes_x,
@@ -746,7 +832,11 @@ extern "C" svdq_status svdq_linear_forward(const svdq_weight* w, const uint16_t*
   uint16_t* xl1 = w->r > 0 ? reinterpret_cast<uint16_t*>(sf_x + ws_sf(M, w->K)) : nullptr;
   cudaStream_t s = (cudaStream_t)stream;
   if ((st = launch_quantize(w, X, M, ldx, codes_x, sf_x, xl1, s, sms)) != SVDQ_OK) return st;
-  return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, s, sms);
+  // split-K for few output tiles when the workspace has room for it
+  const size_t a = rup(svdq_act_workspace_bytes(M, w->K, w->r), 256);
+  const size_t g = gemm_split_ws_bytes(M, w->N, w->K);
+  void* split_ws = (g && ws_bytes >= a + g) ? static_cast<void*>(base + a) : nullptr;
+  return launch_gemm(w, codes_x, sf_x, xl1, M, Y, ldy, s, sms, false, nullptr, split_ws);
 }
 
 extern "C" svdq_status svdq_linear_forward_host(const svdq_weight* w, const uint16_t* X_host,

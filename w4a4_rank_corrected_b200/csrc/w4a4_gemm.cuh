@@ -83,6 +83,7 @@ __host__ __device__ inline uint32_t gemm_smem_bytes() {
 static_assert(1024u + G_STAGES * G_STAGE_BYTES + G_OUT_BYTES + G_BIAS_BYTES + 256u <= 232448u,
               "GEMM shared memory above the 227 KB a CTA may use");
 static_assert((G_STAGES * G_STAGE_BYTES) % 1024 == 0, "output boxes need 1024-byte alignment");
+static_assert((2 * G_STAGES + 12) * 8 <= 256, "barriers and words past the 256-byte barrier area");
 
 struct GemmParams {
   const uint16_t* bias;
@@ -91,7 +92,18 @@ struct GemmParams {
   uint64_t timeout_ns;
   int gelu;          // 1: the epilogue writes GELU(bf16(y)) (first linear of an MLP pair)
   const RowScale* row_scales;   // per-row output scale alpha_m (dynamic mode) or NULL
+  // split-K (few output tiles): each tile's K stages are split into ksplit
+  // parts ("units"); every unit stores its fp32 partial accumulator instead
+  // of Y, and splitk_reduce_kernel adds them in part order and writes Y
+  int ksplit;                   // 1: no split
+  float* partials;              // [tiles][ksplit][2 CTAs][128 rows][256 cols] fp32
 };
+
+// The 256-deep stages [lo, hi) of part `part` of a K split in `ksplit` parts.
+__device__ __forceinline__ void split_stages(int part, int ksplit, int kb_total, int& lo, int& hi) {
+  lo = (int)(((long long)part * kb_total) / ksplit);
+  hi = (int)(((long long)(part + 1) * kb_total) / ksplit);
+}
 
 __global__ void __launch_bounds__(G_THREADS, 1)
     w4a4_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
@@ -99,7 +111,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
                      const __grid_constant__ CUtensorMap tm_sfb,
                      const __grid_constant__ CUtensorMap tm_alr,
                      const __grid_constant__ CUtensorMap tm_blr,
-                     const __grid_constant__ CUtensorMap tm_y, const GemmParams p) {
+                     const __grid_constant__ CUtensorMap tm_y,
+                     const __grid_constant__ CUtensorMap tm_part, const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -132,14 +145,16 @@ __global__ void __launch_bounds__(G_THREADS, 1)
   const int num_m = (M + 2 * G_BM - 1) / (2 * G_BM);
   const int num_n = (N + G_BN - 1) / G_BN;
   const int num_tiles = num_m * num_n;
+  const int ksplit = p.ksplit > 1 ? p.ksplit : 1;
+  const int num_units = num_tiles * ksplit;   // unit u: tile u / ksplit, part u % ksplit
   const int pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
   // Each pair takes a contiguous run of tiles in M-major order (tile t is
   // M block t / num_n, N block t % num_n), so consecutive tiles mostly share
   // their activation rows and those rows' scales stay in tensor memory.
-  const int t_begin = (int)(((long long)pair * num_tiles) / num_pairs);
-  const int t_end = (int)(((long long)(pair + 1) * num_tiles) / num_pairs);
+  const int t_begin = (int)(((long long)pair * num_units) / num_pairs);   // this pair's units
+  const int t_end = (int)(((long long)(pair + 1) * num_units) / num_pairs);
   const int k64 = K >> 6;
-  const bool sfa_res = k64 <= G_SFA_RES_MAX_K64;
+  const bool sfa_res = ksplit == 1 && k64 <= G_SFA_RES_MAX_K64;
   const int kb_total = (k64 + 3) >> 2;
   const int lr_chunks = has_lr ? (p.klr >> 6) : 0;
   const unsigned int kid = 2;
@@ -195,13 +210,17 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     // ---------------------------------------------- TMA producer (warp) ----
     int it = 0;
     bool stop = false;
-    for (int tile = t_begin; tile < t_end && !stop; ++tile) {
+    for (int u = t_begin; u < t_end && !stop; ++u) {
+      const int tile = u / ksplit, part = u - tile * ksplit;
+      int kb_lo, kb_hi;
+      split_stages(part, ksplit, kb_total, kb_lo, kb_hi);
+      const int lr_here = part == ksplit - 1 ? lr_chunks : 0;   // the low-rank stage: last part
       const int mb = tile / num_n, nb = tile % num_n;
-      const bool load_sfa = !sfa_res || tile == t_begin || nb == 0;
+      const bool load_sfa = !sfa_res || u == t_begin || nb == 0;
       const int row0 = mb * 2 * G_BM + (int)rank * G_BM;     // this CTA's A rows
       const int brow0 = nb * G_BN + (int)rank * G_BN_CTA;    // this CTA's B rows
       const int sfa_blk = mb * 2 + (int)rank;                // 128-row scale block
-      for (int kb = 0; kb < kb_total; ++kb, ++it) {
+      for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
         const int st = it % G_STAGES;
         const uint32_t ph = (it / G_STAGES) & 1;
         if (!mbar_wait_warp(empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) {
@@ -225,7 +244,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
         __syncwarp();
         issued = it + 1;
       }
-      for (int c = 0; c < lr_chunks && !stop; ++c, ++it) {
+      for (int c = 0; c < lr_here && !stop; ++c, ++it) {
         const int st = it % G_STAGES;
         const uint32_t ph = (it / G_STAGES) & 1;
         if (!mbar_wait_warp(empty0 + 8 * st, ph ^ 1, p.timeout_ns, abort_flag, (1u << 8) | kid)) {
@@ -262,15 +281,19 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       // made right after the previous stage was issued (its latency then
       // overlaps the tensor-core work instead of preceding the next issue)
       bool ready = false;
-      for (int tile = t_begin; tile < t_end && !stop; ++tile, ++tcount) {
+      for (int u = t_begin; u < t_end && !stop; ++u, ++tcount) {
         // (the accumulator is free only once every MMA of the previous tile
         // has completed, so resident scales may be overwritten after this)
         if (!mbar_wait_warp(acc_empty, (tcount & 1) ^ 1, p.timeout_ns, abort_flag, (2u << 8) | kid))
           break;
         tc_fence_after();
-        const bool load_sfa = !sfa_res || tile == t_begin || tile % num_n == 0;
+        const int tile = u / ksplit, part = u - tile * ksplit;
+        int kb_lo, kb_hi;
+        split_stages(part, ksplit, kb_total, kb_lo, kb_hi);
+        const int lr_here = part == ksplit - 1 ? lr_chunks : 0;
+        const bool load_sfa = !sfa_res || u == t_begin || tile % num_n == 0;
         uint32_t accumulate = 0;
-        for (int kb = 0; kb < kb_total; ++kb, ++it) {
+        for (int kb = kb_lo; kb < kb_hi; ++kb, ++it) {
           const int st = it % G_STAGES;
           const uint32_t ph = (it / G_STAGES) & 1;
           // the stage's TMA bytes have landed (complete_tx); the MMAs and
@@ -316,7 +339,7 @@ __global__ void __launch_bounds__(G_THREADS, 1)
           if (elect_one()) tc_commit_pair(empty0 + 8 * st, 0x3);
           __syncwarp();
         }
-        for (int c = 0; c < lr_chunks && !stop; ++c, ++it) {
+        for (int c = 0; c < lr_here && !stop; ++c, ++it) {
           const int st = it % G_STAGES;
           const uint32_t ph = (it / G_STAGES) & 1;
           if (!ready &&
@@ -353,7 +376,8 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     const bool issuer = ((warp - 2) & 3) == 0 && lane == 0;
     int use = 0;                               // boxes this group has staged
     int tcount = 0;
-    for (int tile = t_begin; tile < t_end; ++tile, ++tcount) {
+    for (int u = t_begin; u < t_end; ++u, ++tcount) {
+      const int tile = u / ksplit, part = u - tile * ksplit;
       const int mb = tile / num_n, nb = tile % num_n;
       // stage this tile's bias (fp32) while the main loop runs.  Buffer
       // tcount&1 was last read for tile tcount-2, which every thread had
@@ -383,6 +407,47 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       const float alpha = (p.row_scales && row0 + row_t < M) ? p.row_scales[row0 + row_t].alpha
                                                              : p.alpha;
       bool ok = true;
+      if (ksplit > 1) {
+        // split-K: this unit's fp32 partial instead of Y, through the same
+        // staging buffer and bulk stores: four 128-row x 32-column boxes per
+        // half (rows past M are written but never read)
+        const int prow = ((tile * ksplit + part) * 2 + (int)rank) * G_BM;
+#pragma unroll
+        for (int sb = 0; sb < 4; ++sb, ++use) {
+          if (use > 0) {
+            if (issuer) {
+              bulk_wait_read_all();
+              mbar_arrive(freed);
+            }
+            __syncwarp();
+            if (!mbar_wait_warp(freed, (use - 1) & 1, p.timeout_ns, abort_flag, (7u << 8) | kid)) {
+              ok = false;
+              break;
+            }
+          }
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(obuf + row_t * 128 + ((j ^ (row_t & 7)) << 4), acc[sb][4 * j],
+                         acc[sb][4 * j + 1], acc[sb][4 * j + 2], acc[sb][4 * j + 3]);
+          fence_proxy_async_shared();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(staged);
+          if (issuer) {
+            if (mbar_wait(staged, use & 1, p.timeout_ns, abort_flag, (8u << 8) | kid)) {
+              if (row0 < M) {
+                tma_store_2d(&tm_part, obuf, half * 128 + sb * 32, prow);
+                bulk_commit_group();
+              }
+            } else {
+              ok = false;
+            }
+          }
+          ok = __all_sync(0xffffffffu, ok) != 0;
+          if (!ok) break;
+        }
+        if (!ok) break;
+        continue;
+      }
 #pragma unroll
       for (int sb = 0; sb < 2; ++sb, ++use) {
         // the buffer is free once the store issued from it has read it
@@ -454,15 +519,26 @@ __global__ void __launch_bounds__(G_THREADS, 1)
       mbar_wait_drain_cluster(peer_bar, 0, p.timeout_ns);
       const int peer = *peer_issued;
       const int hi = max(issued, peer);
-      const int per_tile = kb_total + lr_chunks;
       for (int i = max(0, hi - G_STAGES); i < hi; ++i) {
         const uint32_t fb = full0 + 8 * (i % G_STAGES);
         if (i >= issued) {
-          // the stage's bytes follow from its place in the tile sequence
+          // the stage's bytes follow from its place in the unit sequence
           // (the same rule the producers use)
-          const int tile = t_begin + i / per_tile;
-          const bool lr_stage = (i % per_tile) >= kb_total;
-          const bool with_sfa = !sfa_res || tile == t_begin || tile % num_n == 0;
+          int u = t_begin, j = i;
+          bool lr_stage = false;
+          while (u < t_end) {
+            const int tl = u / ksplit, pt = u - tl * ksplit;
+            int lo, hi2;
+            split_stages(pt, ksplit, kb_total, lo, hi2);
+            const int n_fp4 = hi2 - lo, n_lr = pt == ksplit - 1 ? lr_chunks : 0;
+            if (j < n_fp4 + n_lr) {
+              lr_stage = j >= n_fp4;
+              break;
+            }
+            j -= n_fp4 + n_lr;
+            ++u;
+          }
+          const bool with_sfa = !sfa_res || u == t_begin || (u / ksplit) % num_n == 0;
           mbar_arrive_expect_tx(fb, (lr_stage ? G_LR_TX : with_sfa ? G_FP4_TX : G_FP4_TX_NOSFA) / 2);
         }
         mbar_wait_drain(fb, (i / G_STAGES) & 1, p.timeout_ns);
@@ -484,6 +560,57 @@ __global__ void __launch_bounds__(G_THREADS, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem, G_TMEM_COLS);
   }
+}
+
+// Split-K reduction: Y[m][n] = bf16(alpha * sum_p partial_p[m][n] + bias[n]),
+// the parts added in part order (so Y does not depend on which unit of the
+// GEMM finished first).  One thread per 8 consecutive outputs of a row: all
+// parts' 32 bytes are loaded before the sum (up to 8 parts in flight).
+// Launched right after the GEMM with programmatic dependent launch.
+__global__ void __launch_bounds__(256)
+    splitk_reduce_kernel(const float* __restrict__ partials, int M, int N, int ksplit,
+                         float alpha, const uint16_t* __restrict__ bias, uint16_t* __restrict__ Y,
+                         int64_t ldy) {
+  grid_dependency_wait();
+  const int num_n = (N + G_BN - 1) / G_BN;
+  const int groups = N >> 3;   // N % 8 == 0
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < (long long)M * groups;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int m = (int)(i / groups), n = (int)(i - (long long)m * groups) * 8;
+    const int tile = (m / (2 * G_BM)) * num_n + n / G_BN;
+    const int rank = (m % (2 * G_BM)) / G_BM, row = m % G_BM, col = n % G_BN;
+    const float* src = partials + (((size_t)tile * ksplit * 2 + rank) * G_BM + row) * G_BN + col;
+    const size_t stride = (size_t)2 * G_BM * G_BN;
+    float4 v[2 * 8];
+#pragma unroll
+    for (int pp = 0; pp < 8; ++pp)
+      if (pp < ksplit) {
+        v[2 * pp] = ld_cg_f4(src + pp * stride);
+        v[2 * pp + 1] = ld_cg_f4(src + pp * stride + 4);
+      }
+    float y[8] = {v[0].x, v[0].y, v[0].z, v[0].w, v[1].x, v[1].y, v[1].z, v[1].w};
+#pragma unroll
+    for (int pp = 1; pp < 8; ++pp)
+      if (pp < ksplit) {
+        y[0] += v[2 * pp].x;
+        y[1] += v[2 * pp].y;
+        y[2] += v[2 * pp].z;
+        y[3] += v[2 * pp].w;
+        y[4] += v[2 * pp + 1].x;
+        y[5] += v[2 * pp + 1].y;
+        y[6] += v[2 * pp + 1].z;
+        y[7] += v[2 * pp + 1].w;
+      }
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float b0 = bias ? bf16_lo_f32(bias[n + 2 * q]) : 0.0f;
+      const float b1 = bias ? bf16_lo_f32(bias[n + 2 * q + 1]) : 0.0f;
+      o[q] = pack_bf16x2(fmaf(alpha, y[2 * q], b0), fmaf(alpha, y[2 * q + 1], b1));
+    }
+    *reinterpret_cast<uint4*>(Y + (size_t)m * ldy + n) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  grid_launch_dependents();
 }
 
 }  // namespace svdq_dev
