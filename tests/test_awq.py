@@ -96,3 +96,18 @@ def test_awq_linear_parity(M, K, N):
     Y_ref = A.awq_linear_reference(X, q, z, sb, b)
     check_output(from_dev_bf16(Y), Y_ref)
     assert S.svdq_device_error() == 0
+
+
+def test_awq_code_to_bf16_trick_is_exact():
+    """The GEMV's dequantization, restated on the host: the bit pattern
+    0x4300 | q is the bf16 number 128 + q for every 4-bit q, and the bf16
+    difference (128 + q) - (128 + z) is q - z exactly (no rounding: every
+    operand and result is an integer of at most 8 significant bits)."""
+    import torch
+    q = torch.arange(16, dtype=torch.int32)
+    as_bf16 = (q | 0x4300).to(torch.int16).view(torch.bfloat16)
+    assert torch.equal(as_bf16.float(), 128.0 + q.float())
+    for z in range(16):
+        zz = torch.full((16,), 0x4300 | z, dtype=torch.int16).view(torch.bfloat16)
+        d = (as_bf16 - zz)                    # bf16 subtraction, round to nearest
+        assert torch.equal(d.float(), (q - z).float())
