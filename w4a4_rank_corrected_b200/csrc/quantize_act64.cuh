@@ -303,19 +303,22 @@ __global__ void __launch_bounds__(Q64_THREADS, 1)
         // the async proxy
         if (!mbar_wait_warp(x_full0 + 8 * xs, xph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
         if (!mbar_wait_warp(l_full0 + 8 * ls, lph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
-#pragma unroll
-        for (int b = 0; b < Q64_BOXES; ++b) {
-          const uint64_t da = sdesc_sw128(smem_u32(smem + xs * Q64_X_BYTES + b * Q64_BOX_BYTES));
-          const uint64_t db =
-              sdesc_sw128(smem_u32(smem + L.l1_off + ls * L.l1_bytes + b * (L.l1_bytes / Q64_BOXES)));
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {  // K = 16 bf16 = 32 bytes per MMA
-            if (elect_one())
-              mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (i | b | kk) != 0 ? 1u : 0u);
-            __syncwarp();
-          }
-        }
+        // the chunk's eight MMAs and both releases from one elected lane: this
+        // warp shares its sub-partition with busy quantize warps, and each
+        // stage's release waits for its MMAs, so the fewer issue slots the
+        // chunk costs here the sooner the X ring turns over (an elect and a
+        // warp sync per MMA left this warp about 1.8 us behind the
+        // quantize warps at the end of a 4608 x 3072 launch)
         if (elect_one()) {
+#pragma unroll
+          for (int b = 0; b < Q64_BOXES; ++b) {
+            const uint64_t da = sdesc_sw128(smem_u32(smem + xs * Q64_X_BYTES + b * Q64_BOX_BYTES));
+            const uint64_t db = sdesc_sw128(
+                smem_u32(smem + L.l1_off + ls * L.l1_bytes + b * (L.l1_bytes / Q64_BOXES)));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)  // K = 16 bf16 = 32 bytes per MMA
+              mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (i | b | kk) != 0 ? 1u : 0u);
+          }
           tc_commit(x_empty0 + 8 * xs);
           tc_commit(l_empty0 + 8 * ls);
         }
