@@ -346,19 +346,19 @@ __global__ void __launch_bounds__(QA_THREADS, 1)
         // the async proxy
         if (!mbar_wait_warp(x_full0 + 8 * xs, xph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
         if (!mbar_wait_warp(l_full0 + 8 * ls, lph, p.timeout_ns, abort_flag, (2u << 8) | kid)) break;
-#pragma unroll
-        for (int b = 0; b < QA_BOXES; ++b) {
-          const uint64_t da = sdesc_sw128(smem_u32(smem + xs * QA_X_BYTES + b * QA_BOX_BYTES));
-          const uint64_t db =
-              sdesc_sw128(smem_u32(smem + L.l1_off + ls * L.l1_bytes + b * (L.l1_bytes / QA_BOXES)));
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {  // K = 16 bf16 = 32 bytes per MMA
-            if (elect_one())
-              mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (i | b | kk) != 0 ? 1u : 0u);
-            __syncwarp();
-          }
-        }
+        // the chunk's MMAs and both releases from one elected lane (fewer
+        // issue slots on a sub-partition shared with the quantize warps, so
+        // the X ring turns over sooner)
         if (elect_one()) {
+#pragma unroll
+          for (int b = 0; b < QA_BOXES; ++b) {
+            const uint64_t da = sdesc_sw128(smem_u32(smem + xs * QA_X_BYTES + b * QA_BOX_BYTES));
+            const uint64_t db = sdesc_sw128(
+                smem_u32(smem + L.l1_off + ls * L.l1_bytes + b * (L.l1_bytes / QA_BOXES)));
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)  // K = 16 bf16 = 32 bytes per MMA
+              mma_bf16(tmem, da + 2 * kk, db + 2 * kk, idesc, (i | b | kk) != 0 ? 1u : 0u);
+          }
           tc_commit(x_empty0 + 8 * xs);
           tc_commit(l_empty0 + 8 * ls);
         }
