@@ -22,7 +22,8 @@
  *
  * Conventions for every call:
  *   - All pointers are caller-owned.  The library never allocates, frees or
- *     retains device or host memory and never synchronizes a stream.
+ *     retains device or host memory and never synchronizes a stream (except
+ *     svdq_device_error, whose job is to read the kernels' error word).
  *   - "device" pointers must be global memory of the current CUDA device;
  *     "host" pointers are ordinary host memory.
  *   - bf16 tensors are passed as uint16_t bit patterns.
