@@ -217,3 +217,19 @@ def test_pack_rejects_bad_input():
     with pytest.raises(S.SvdqError) as e:
         S.svdq_pack_weight(W, cx, 16)
     assert e.value.status == 7
+
+
+def test_split_k_argument_checks():
+    """svdq_gemm_splitk checks its workspace's size and alignment before
+    touching a device; a shape that does not split needs no workspace."""
+    L = S.lib
+    w = _fake_weight(N=3072, K=12288, r=32)
+    C, SF, XL, Y = 0x30000000, 0x40000000, 0x50000000, 0x60000000
+    need = S.svdq_gemm_workspace_bytes(64, 3072, 12288)
+    assert need > 0
+    assert L.svdq_gemm_splitk(ctypes.byref(w), C, SF, XL, 64, Y, 3072, 0x70000010, need,
+                              None) == 3                                  # not 256-aligned
+    assert L.svdq_gemm_splitk(ctypes.byref(w), C, SF, XL, 0, Y, 3072, None, 0, None) == 0
+    assert L.svdq_gemm_splitk(ctypes.byref(w), C, SF, XL, 64, Y, 3000, 0x70000000, need,
+                              None) == 1                                  # ldy < N
+    assert S.svdq_gemm_workspace_bytes(64, 3072, 100) == 0                # K % 64

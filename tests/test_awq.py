@@ -111,3 +111,15 @@ def test_awq_code_to_bf16_trick_is_exact():
         zz = torch.full((16,), 0x4300 | z, dtype=torch.int16).view(torch.bfloat16)
         d = (as_bf16 - zz)                    # bf16 subtraction, round to nearest
         assert torch.equal(d.float(), (q - z).float())
+
+
+def test_awq_tile_codes_validation():
+    L = S.lib
+    q = np.zeros((16, 32), np.uint8)
+    out = np.zeros(16 * 32, np.uint8)
+    assert L.svdq_awq_tile_codes(q.ctypes.data, 16, 64, out.ctypes.data) == 0
+    assert L.svdq_awq_tile_codes(q.ctypes.data, 16, 96, out.ctypes.data) == 1      # K % 64
+    assert L.svdq_awq_tile_codes(None, 16, 64, out.ctypes.data) == 1
+    assert L.svdq_awq_tile_codes(q.ctypes.data, 0, 64, out.ctypes.data) == 1
+    with pytest.raises(ValueError):
+        S.svdq_awq_tile_codes(q[:, :16], 16, 64)                                   # shape
