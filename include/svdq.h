@@ -405,7 +405,9 @@ svdq_status svdq_awq_pack(const float* W, int N, int K, int group, uint8_t* q_pa
                           uint8_t* zeros, uint16_t* scales);
 
 /* svdq_awq_tile_codes (host, synchronous): the codes in the layout the
- * GPU layer reads.  q_rowmajor as svdq_awq_pack writes it ([N][K/2], even k
+ * GPU layer reads (a permutation only: the layer is the awq_w4a16 family of
+ * "Bringing Nunchaku 4-bit diffusion inference to Diffusers", Russian
+ * rendering, "Technical details and hardware support").  q_rowmajor as svdq_awq_pack writes it ([N][K/2], even k
  * in the low nibble); q_tiled: ceil(N/16) * 16 * K / 2 bytes.  Per 16-row
  * block rb and 64-deep block of K, 512 bytes = 32 lanes x 16 bytes; lane
  * l = 4 g + c holds one 32-bit word per 16-deep k-step ks (4 per block, at
